@@ -1,0 +1,194 @@
+"""Python access to the CPU oracle of the weight fake-quantizer.
+
+TEST INFRASTRUCTURE ONLY: tests, the smoke check and the benchmark's CPU
+baseline leg call this module; the product path never imports it. The oracle
+itself is the plain C file next to this one (``pq_oracle.c``); this module
+compiles it with gcc on first use (no FMA contraction, no fast-math) and wraps
+its functions for numpy arrays.
+
+Quantizer arithmetic lives only in the C file; this wrapper marshals arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "pq_oracle.c")
+_LIB = os.path.join(_HERE, "libpq_oracle.so")
+CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c11",
+          "-shared", "-fPIC", "-Wall", "-Wextra"]
+
+# Quantizer identifiers (same numbering as the library's C ABI).
+BINARY, TERNARY, SEQ2, SEQ2_B, LSQ2, LSQ3, LSQ4 = 1, 2, 3, 4, 5, 6, 7
+ALL_QUANTIZERS = (BINARY, TERNARY, SEQ2, SEQ2_B, LSQ2, LSQ3, LSQ4)
+
+_lock = threading.Lock()
+_default = None
+
+
+def compile_source(src: str, out: str) -> str:
+    """Compile an oracle C source into a shared library at ``out``."""
+    tmp = out + f".{os.getpid()}.tmp"
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``libpq_oracle.so`` (if missing or stale)."""
+    stale = (not os.path.exists(_LIB)
+             or os.path.getmtime(_LIB) < os.path.getmtime(SRC))
+    if force or stale:
+        compile_source(SRC, _LIB)
+    return _LIB
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """One loaded copy of the oracle library."""
+
+    def __init__(self, path: str):
+        L = ctypes.CDLL(path)
+        i64, p = ctypes.c_int64, ctypes.c_void_p
+        L.pqo_fwd.argtypes = [ctypes.c_int, i64, i64, p, p, p, p, p]
+        L.pqo_fwd.restype = ctypes.c_int
+        L.pqo_bwd.argtypes = [ctypes.c_int, i64, i64, p, p, p, p, p,
+                              ctypes.c_float, p]
+        L.pqo_bwd.restype = ctypes.c_int
+        L.pqo_pack.argtypes = [ctypes.c_int, i64, i64, p, p, p]
+        L.pqo_pack.restype = ctypes.c_int
+        L.pqo_default_grad_scale.argtypes = [ctypes.c_int, i64]
+        L.pqo_default_grad_scale.restype = ctypes.c_float
+        L.pqo_code_bits.argtypes = [ctypes.c_int]
+        L.pqo_code_bits.restype = ctypes.c_int
+        L.pqo_bf16_rne.argtypes = [ctypes.c_float]
+        L.pqo_bf16_rne.restype = ctypes.c_uint16
+        L.pqo_quantize_scalar.argtypes = [
+            ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float),
+            ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int),
+            ctypes.POINTER(ctypes.c_float)]
+        L.pqo_quantize_scalar.restype = ctypes.c_int
+        self.lib = L
+        self.path = path
+
+    def code_bits(self, q: int) -> int:
+        return int(self.lib.pqo_code_bits(q))
+
+    def fwd(self, q: int, w, alpha, pack: bool = False):
+        """Returns (wq_bf16 bits uint16 [R,C], codes int8 [R,C], packed uint8
+        [R, C*bits/8] or None)."""
+        w = np.ascontiguousarray(w, np.float32)
+        rows, cols = w.shape
+        alpha = np.ascontiguousarray(alpha, np.float32).reshape(rows)
+        wq = np.empty((rows, cols), np.uint16)
+        codes = np.empty((rows, cols), np.int8)
+        packed = (np.empty((rows, cols * self.code_bits(q) // 8), np.uint8)
+                  if pack else None)
+        rc = self.lib.pqo_fwd(q, rows, cols, _ptr(w), _ptr(alpha), _ptr(wq),
+                              _ptr(codes), _ptr(packed))
+        if rc != 0:
+            raise ValueError(f"oracle fwd rejected q={q} shape={w.shape} "
+                             f"pack={pack}")
+        return wq, codes, packed
+
+    def bwd(self, q: int, w, alpha, g_bf16, grad_scale: float):
+        """Returns (dw fp32 [R,C], dalpha fp32 [R], row_abs fp64 [R]) where
+        row_abs is the per-row sum of |term| before grad_scale."""
+        w = np.ascontiguousarray(w, np.float32)
+        rows, cols = w.shape
+        alpha = np.ascontiguousarray(alpha, np.float32).reshape(rows)
+        g = np.ascontiguousarray(g_bf16).view(np.uint16)
+        assert g.shape == w.shape
+        dw = np.empty((rows, cols), np.float32)
+        da = np.empty(rows, np.float32)
+        row_abs = np.empty(rows, np.float64)
+        rc = self.lib.pqo_bwd(q, rows, cols, _ptr(w), _ptr(alpha), _ptr(g),
+                              _ptr(dw), _ptr(da), ctypes.c_float(grad_scale),
+                              _ptr(row_abs))
+        if rc != 0:
+            raise ValueError(f"oracle bwd rejected q={q}")
+        return dw, da, row_abs
+
+    def pack(self, q: int, w, alpha):
+        w = np.ascontiguousarray(w, np.float32)
+        rows, cols = w.shape
+        alpha = np.ascontiguousarray(alpha, np.float32).reshape(rows)
+        out = np.empty((rows, cols * self.code_bits(q) // 8), np.uint8)
+        rc = self.lib.pqo_pack(q, rows, cols, _ptr(w), _ptr(alpha), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle pack rejected q={q} shape={w.shape}")
+        return out
+
+    def quantize_scalar(self, q: int, w: float, alpha: float,
+                        clip_hi: float = 0.0):
+        """One element: dict(code, level, wq32, inside, x). ``clip_hi`` > 0
+        replaces the symmetric SEQ/ternary clip value."""
+        c, lev, wq = ctypes.c_int(), ctypes.c_float(), ctypes.c_float()
+        ins, x = ctypes.c_int(), ctypes.c_float()
+        rc = self.lib.pqo_quantize_scalar(q, w, alpha, clip_hi,
+                                          ctypes.byref(c), ctypes.byref(lev),
+                                          ctypes.byref(wq), ctypes.byref(ins),
+                                          ctypes.byref(x))
+        if rc != 0:
+            raise ValueError(f"unknown quantizer {q}")
+        return dict(code=c.value, level=lev.value, wq32=wq.value,
+                    inside=bool(ins.value), x=x.value)
+
+    def bf16_rne(self, f) -> np.ndarray:
+        """Elementwise fp32 -> bf16 bits via the oracle's own conversion."""
+        f = np.asarray(f, np.float32).ravel()
+        return np.array([self.lib.pqo_bf16_rne(float(v)) for v in f],
+                        np.uint16)
+
+    def default_grad_scale(self, q: int, cols: int) -> float:
+        return float(self.lib.pqo_default_grad_scale(q, cols))
+
+
+def default() -> Oracle:
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+def fwd(q, w, alpha, pack=False):
+    return default().fwd(q, w, alpha, pack)
+
+
+def bwd(q, w, alpha, g_bf16, grad_scale):
+    return default().bwd(q, w, alpha, g_bf16, grad_scale)
+
+
+def pack(q, w, alpha):
+    return default().pack(q, w, alpha)
+
+
+def quantize_scalar(q, w, alpha, clip_hi=0.0):
+    return default().quantize_scalar(q, w, alpha, clip_hi)
+
+
+def bf16_rne(f):
+    return default().bf16_rne(f)
+
+
+def default_grad_scale(q, cols):
+    return default().default_grad_scale(q, cols)
+
+
+def code_bits(q):
+    return default().code_bits(q)
+
+
+def bf16_bits_to_float(h) -> np.ndarray:
+    """bf16 bit patterns -> fp32 values (exact widening)."""
+    return (np.asarray(h).view(np.uint16).astype(np.uint32) << 16).view(np.float32)
