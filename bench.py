@@ -1,0 +1,457 @@
+"""Benchmark of the quantizer step: forward + STE backward over the
+Llama-3-8B-shaped linear set (32 layers of q/o 4096x4096, k/v 1024x4096,
+gate/up 14336x4096, down 4096x14336; 2-bit SEQ, bf16 dequant output).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward over every matrix, then one backward over every
+matrix, with all inputs resident in HBM (synthetic, seeded; about 84 GB per
+GPU, far larger than L2, so no flush is needed between steps). Each rank
+runs the full set on its own GPU (weak scaling; the quantizer shards by
+matrix and row and needs no collective). Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain C reference used by
+the tests) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantizer fwd+bwd Gweights/s per step and % of B200 HBM roofline"
+UNIT = "Gweights/s"
+WORKLOAD = "llama3_8b_linear_set_seq2_fwd_ste_bwd"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0,
+                   help="target CPU time of the oracle baseline sample")
+    return p.parse_args()
+
+
+def config_dict(n_gpus, weights_per_gpu):
+    return {"workload": WORKLOAD,
+            "matrices": "32 layers x {q,o 4096x4096; k,v 1024x4096; "
+                        "gate,up 14336x4096; down 4096x14336}",
+            "quantizer": "seq2 (2-bit SEQ, levels +-0.25, +-0.75 alpha)",
+            "weights_per_gpu": weights_per_gpu,
+            "global_weights": weights_per_gpu * n_gpus,
+            "parallelism": f"replicas x{n_gpus} (each GPU its own layer set)",
+            "l2": "inputs larger than L2 (about 84 GB resident per GPU)"}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantization_aware_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per weight of the backward kernel from an ncu capture,
+    valid only while the kernel sources are unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return d
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clocks and throttle reasons during the timed
+    region (read only; no GPU setting is changed)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- reference
+def workload_weights():
+    from bit_quantization_aware_b200 import inputs as I
+    return I.total_weights(I.llama3_8b_set())
+
+
+def sample_rows_for_oracle(cpu_seconds):
+    """Rows drawn from every matrix kind of one layer so that the oracle's
+    forward + backward takes about ``cpu_seconds`` on one core."""
+    import numpy as np
+
+    from bit_quantization_aware_b200 import inputs as I
+    from oracle import pq_oracle
+    import torch
+
+    mats = [m for m in I.llama3_8b_set() if m.layer == 0]
+    q = I.SEQ2
+    # calibrate with 8 rows of the widest matrix
+    w = I.normal_weights(8, 14336, seed=0, stream=6, device="cpu")
+    a = I.alpha_init(w, q)
+    g = I.grad_bf16(8, 14336, seed=0, stream=70, device="cpu")
+    gn = g.view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    pq_oracle.fwd(q, w.numpy(), a.numpy())
+    pq_oracle.bwd(q, w.numpy(), a.numpy(), gn, 1.0)
+    per_weight = (time.perf_counter() - t0) / w.numel()
+    total = cpu_seconds / max(per_weight, 1e-12)
+    per_kind = total / len(mats)
+    sample = []
+    for m in mats:
+        rows = max(1, min(m.rows, int(per_kind // m.cols)))
+        wm = I.normal_weights(rows, m.cols, seed=0, stream=m.proj, device="cpu")
+        am = I.alpha_init(wm, q)
+        gm = I.grad_bf16(rows, m.cols, seed=0, stream=m.proj + 64, device="cpu")
+        sample.append((m, wm.numpy(), am.numpy(), gm.view(torch.int16).numpy().view(np.uint16)))
+    return sample
+
+
+def time_oracle(sample):
+    from oracle import pq_oracle
+    q = 3  # SEQ2
+    t0 = time.perf_counter()
+    n = 0
+    for m, w, a, g in sample:
+        pq_oracle.fwd(q, w, a)
+        pq_oracle.bwd(q, w, a, g, pq_oracle.default_grad_scale(q, m.cols))
+        n += w.size
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+def describe_sample(sample):
+    rows = {m.name.split(".")[-1]: w.shape[0] for m, w, _, _ in sample}
+    n = sum(w.size for _, w, _, _ in sample)
+    return (f"{n} weights: rows {rows} of layer 0's matrices (full width), "
+            f"SEQ2 forward + backward, single thread")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    # each step is a bounded sample: the whole run stays near two minutes
+    per_step = max(0.5, min(10.0, 120.0 / max(1, args.steps)))
+    sample = sample_rows_for_oracle(per_step)
+    for _ in range(args.warmup):
+        time_oracle(sample[:1])
+    times, n = [], 0
+    for _ in range(args.steps):
+        n, dt = time_oracle(sample)
+        times.append(dt)
+    total = sum(times)
+    value = n * args.steps / total / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_dict(args.gpus, workload_weights()),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1,
+                             "kind": "oracle", "sample": describe_sample(sample)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.step import QuantStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    pq.lib()  # fail loudly if the CUDA library is missing
+
+    mats = I.llama3_8b_set()
+    step = QuantStep(mats, pq.PQ_SEQ2, device=f"cuda:{local}")
+    step.generate(seed=3 + rank)
+    stream = torch.cuda.current_stream()
+    weights = step.weights
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        step.run()
+    torch.cuda.synchronize()
+
+    n_b = len(step.bufs)
+    ev_start = torch.cuda.Event(enable_timing=True)
+    ev_end = torch.cuda.Event(enable_timing=True)
+    bwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    gpu_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            gpu_index = int(vis.split(",")[local])
+        except ValueError:
+            pass
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.3)
+
+    barrier()
+    torch.cuda.synchronize()
+    ev_start.record(stream)
+    for k in range(args.steps):
+        step.fwd_all()
+        bwd_ev[k][0].record(stream)
+        step.bwd_all()
+        bwd_ev[k][1].record(stream)
+    ev_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+
+    ms_total = ev_start.elapsed_time(ev_end)
+    bwd_ms = sum(a.elapsed_time(b) for a, b in bwd_ev)
+    t = torch.tensor([ms_total, bwd_ms], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, bwd_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+    value = weights * world / (ms_step * 1e-3) / 1e9
+
+    # roofline of the dominant kernel (the backward: 10 of 16 bytes/weight)
+    peak, peak_kind = measured_peaks()
+    bwd_bytes_step = step.bytes_bwd()
+    bwd_s_step = bwd_ms * 1e-3 / args.steps
+    achieved = bwd_bytes_step / bwd_s_step / 1e9
+    tr = recorded_traffic()
+    traffic = None
+    if tr is not None:
+        traffic = tr["dram_bytes_per_weight"] * weights / n_b
+    roofline = {"bound": "hbm", "kernel": "pq::bwd_kernel<SEQ2, vec>",
+                "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_kind} hbm_gbs (STREAM-style copy)",
+                "algorithmic_bytes_per_launch": bwd_bytes_step / n_b,
+                "avg_launch_us": bwd_s_step / n_b * 1e6,
+                "fwd_bwd_frac_of_peak": (step.bytes_fwd() + bwd_bytes_step)
+                / (ms_step * 1e-3) / 1e9 / peak}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(step, args, local, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = sample_rows_for_oracle(args.cpu_seconds)
+        n, dt = time_oracle(sample)
+        cpu = {"value": n / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": describe_sample(sample), "seconds": dt}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic (seeded N(0,0.02) weights, "
+                "bf16 N(0,1e-3) upstream grads, alpha = max|w_row|)",
+                "config": config_dict(world, weights),
+                "gpu_launches": step.launches_per_step * args.steps,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(step, args, local, world):
+    """Same metric through the public API from host buffers: every step
+    copies each layer's W and dWq from pinned host memory, runs the forward
+    and backward calls, and copies Wq, dW and d(alpha) back to pinned host
+    memory. Copies in and out run on their own streams and overlap compute
+    across layers."""
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantization_aware_b200 import pq
+
+    layers = sorted({b.m.layer for b in step.bufs})
+    by_layer = {l: [b for b in step.bufs if b.m.layer == l] for l in layers}
+    n_layer = sum(b.m.numel for b in by_layer[layers[0]])
+    rows_layer = sum(b.m.rows for b in by_layer[layers[0]])
+    pin = dict(pin_memory=True)
+    h_w = torch.empty(n_layer, dtype=torch.float32, **pin)
+    h_g = torch.empty(n_layer, dtype=torch.bfloat16, **pin)
+    h_wq = torch.empty(n_layer, dtype=torch.bfloat16, **pin)
+    h_dw = torch.empty(n_layer, dtype=torch.float32, **pin)
+    h_da = torch.empty(rows_layer, dtype=torch.float32, **pin)
+    # start from the device data so that host inputs are realistic
+    o = 0
+    for b in by_layer[layers[0]]:
+        h_w[o:o + b.m.numel].copy_(b.w.reshape(-1))
+        h_g[o:o + b.m.numel].copy_(b.g.reshape(-1))
+        o += b.m.numel
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def one_step():
+        done_in, done_cmp = {}, {}
+        for l in layers:
+            with torch.cuda.stream(s_in):
+                o = 0
+                for b in by_layer[l]:
+                    b.w.view(-1).copy_(h_w[o:o + b.m.numel], non_blocking=True)
+                    b.g.view(-1).copy_(h_g[o:o + b.m.numel], non_blocking=True)
+                    o += b.m.numel
+                e = torch.cuda.Event()
+                e.record(s_in)
+                done_in[l] = e
+        for l in layers:
+            s_cmp.wait_event(done_in[l])
+            for b in by_layer[l]:
+                pq.pq_fakequant_fwd(step.q, b.w, b.alpha, b.wq, None, s_cmp)
+            for b in by_layer[l]:
+                pq.pq_fakequant_bwd(step.q, b.w, b.alpha, b.g, b.dw, b.dalpha,
+                                    b.grad_scale, s_cmp)
+            e = torch.cuda.Event()
+            e.record(s_cmp)
+            done_cmp[l] = e
+        with torch.cuda.stream(s_out):
+            for l in layers:
+                s_out.wait_event(done_cmp[l])
+                o, ro = 0, 0
+                for b in by_layer[l]:
+                    h_wq[o:o + b.m.numel].copy_(b.wq.view(-1), non_blocking=True)
+                    h_dw[o:o + b.m.numel].copy_(b.dw.view(-1), non_blocking=True)
+                    h_da[ro:ro + b.m.rows].copy_(b.dalpha, non_blocking=True)
+                    o += b.m.numel
+                    ro += b.m.rows
+
+    one_step()
+    torch.cuda.synchronize()
+    k = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for _ in range(k):
+        one_step()
+        # the next step's inputs may only land after this step's outputs left
+        s_in.wait_stream(s_out)
+    end.record(s_in)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    wall = (time.perf_counter() - t0) * 1e3
+    t = torch.tensor([max(ms, 0.0)], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t[0])
+    ms_step = ms / k
+    bi = sum(b.m.numel * 6 for b in step.bufs)
+    bo = sum(b.m.numel * 6 + b.m.rows * 4 for b in step.bufs)
+    return {"value": step.weights * world / (ms_step * 1e-3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "ms_per_step": ms_step, "steps": k, "wall_ms_per_step": wall / k,
+            "how": "pinned host W, dWq -> device; pq_fakequant_fwd/bwd per matrix; "
+                   "Wq, dW, dalpha -> pinned host; three streams, layer-pipelined"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

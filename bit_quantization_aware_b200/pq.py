@@ -1,0 +1,167 @@
+"""Thin ctypes binding over the C ABI in ``include/pq.h`` (``lib/libpq.so``).
+
+Argument marshalling only: every step of the quantizer runs in the CUDA
+kernels of the library. Tensors are passed as device pointers; torch is used
+for device memory and streams. There is no CPU fallback: loading fails
+loudly when the library is missing.
+
+Function names match the C entry points. Each takes torch tensors (CUDA,
+contiguous) and an optional stream (torch.cuda.Stream or a raw cudaStream_t
+int; default: torch's current stream), and raises ``PQError`` on a non-OK
+status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libpq.so")
+
+PQ_BINARY, PQ_TERNARY, PQ_SEQ2, PQ_SEQ2_B, PQ_LSQ2, PQ_LSQ3, PQ_LSQ4 = range(1, 8)
+QUANTIZERS = {"binary": PQ_BINARY, "ternary": PQ_TERNARY, "seq2": PQ_SEQ2,
+              "seq2_b": PQ_SEQ2_B, "lsq2": PQ_LSQ2, "lsq3": PQ_LSQ3,
+              "lsq4": PQ_LSQ4}
+PQ_OK, PQ_ERR_INVALID_ARG, PQ_ERR_UNSUPPORTED, PQ_ERR_MISALIGNED, \
+    PQ_ERR_CUDA, PQ_ERR_TIMEOUT = range(6)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class PQError(RuntimeError):
+    def __init__(self, fn, status, cuda_err=0):
+        msg = f"{fn}: status {status} ({status_string(status)})"
+        if status == PQ_ERR_CUDA:
+            msg += f", cudaError {cuda_err}"
+        super().__init__(msg)
+        self.status = status
+
+
+def _declare(L):
+    i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.pq_fakequant_fwd.argtypes = [i32, i64, i64, p, p, p, p, p]
+    L.pq_fakequant_fwd.restype = i32
+    L.pq_fakequant_bwd.argtypes = [i32, i64, i64, p, p, p, p, p, f32, p]
+    L.pq_fakequant_bwd.restype = i32
+    L.pq_pack_codes.argtypes = [i32, i64, i64, p, p, p, p]
+    L.pq_pack_codes.restype = i32
+    L.pq_code_bits.argtypes = [i32]
+    L.pq_code_bits.restype = i32
+    L.pq_default_grad_scale.argtypes = [i32, i64]
+    L.pq_default_grad_scale.restype = f32
+    L.pq_status_string.argtypes = [i32]
+    L.pq_status_string.restype = ctypes.c_char_p
+    L.pq_last_cuda_error.argtypes = []
+    L.pq_last_cuda_error.restype = i32
+    return L
+
+
+def lib(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise ImportError(
+                    f"CUDA library {path} is missing; build it with "
+                    "`python -m bit_quantization_aware_b200.build` (there is no "
+                    "CPU fallback)")
+            _lib = _declare(ctypes.CDLL(path))
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, status):
+    if status != PQ_OK:
+        raise PQError(fn, status, lib().pq_last_cuda_error())
+
+
+def _shape(w, rows, cols):
+    if rows is None or cols is None:
+        rows, cols = w.shape
+    return int(rows), int(cols)
+
+
+def pq_fakequant_fwd(q, w, alpha, wq_out, packed_out=None, stream=None,
+                     rows=None, cols=None):
+    """Forward: ``wq_out`` (bf16 [rows, cols]) and optional ``packed_out``
+    (uint8 [rows, cols*bits/8])."""
+    rows, cols = _shape(w, rows, cols)
+    _check("pq_fakequant_fwd", lib().pq_fakequant_fwd(
+        q, rows, cols, _ptr(w), _ptr(alpha), _ptr(wq_out), _ptr(packed_out),
+        _stream(stream)))
+
+
+def pq_fakequant_bwd(q, w, alpha, g, dw_out, dalpha_out, grad_scale,
+                     stream=None, rows=None, cols=None):
+    """Backward: ``dw_out`` (fp32 [rows, cols]) and ``dalpha_out`` (fp32
+    [rows]) from the bf16 upstream gradient ``g``."""
+    rows, cols = _shape(w, rows, cols)
+    _check("pq_fakequant_bwd", lib().pq_fakequant_bwd(
+        q, rows, cols, _ptr(w), _ptr(alpha), _ptr(g), _ptr(dw_out),
+        _ptr(dalpha_out), ctypes.c_float(grad_scale), _stream(stream)))
+
+
+def pq_pack_codes(q, w, alpha, packed_out, stream=None, rows=None, cols=None):
+    """Packed code export only."""
+    rows, cols = _shape(w, rows, cols)
+    _check("pq_pack_codes", lib().pq_pack_codes(
+        q, rows, cols, _ptr(w), _ptr(alpha), _ptr(packed_out),
+        _stream(stream)))
+
+
+def pq_code_bits(q) -> int:
+    return int(lib().pq_code_bits(q))
+
+
+def pq_default_grad_scale(q, cols) -> float:
+    return float(lib().pq_default_grad_scale(q, cols))
+
+
+def status_string(status) -> str:
+    return lib().pq_status_string(status).decode()
+
+
+# --------------------------------------------------------------- conveniences
+def fakequant_fwd(q, w, alpha, pack=False, stream=None):
+    """Allocate outputs and run the forward; returns (wq bf16, packed|None)."""
+    rows, cols = w.shape
+    wq = torch.empty((rows, cols), dtype=torch.bfloat16, device=w.device)
+    packed = (torch.empty((rows, cols * pq_code_bits(q) // 8), dtype=torch.uint8,
+                          device=w.device) if pack else None)
+    pq_fakequant_fwd(q, w, alpha, wq, packed, stream)
+    return wq, packed
+
+
+def fakequant_bwd(q, w, alpha, g, grad_scale=None, stream=None):
+    """Allocate outputs and run the backward; returns (dw fp32, dalpha fp32)."""
+    rows, cols = w.shape
+    if grad_scale is None:
+        grad_scale = pq_default_grad_scale(q, cols)
+    dw = torch.empty((rows, cols), dtype=torch.float32, device=w.device)
+    da = torch.empty((rows,), dtype=torch.float32, device=w.device)
+    pq_fakequant_bwd(q, w, alpha, g, dw, da, grad_scale, stream)
+    return dw, da

@@ -1,0 +1,166 @@
+/*
+ * pq.h - C ABI of the B200 (sm_100a) ParetoQ-style weight fake-quantizer.
+ *
+ * The library quantizes the fp32 "shadow" weights of one linear layer per
+ * call, the way quantization-aware training does on every forward, and runs
+ * the matching straight-through-estimator backward. All arithmetic runs in
+ * CUDA kernels for sm_100a; there is no CPU fallback.
+ *
+ * Notation (one weight matrix):
+ *   W      fp32 [rows, cols], row-major, contiguous; rows = output channels
+ *   alpha  fp32 [rows], the learnable per-output-channel scale
+ *   x      fl(w / alpha), IEEE fp32 division
+ *   G      upstream gradient dWq, bf16 [rows, cols], row-major
+ *
+ * Conventions shared by every entry point:
+ *   - All array arguments are DEVICE pointers owned by the caller. The
+ *     library allocates nothing and keeps no state between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and the call returns after the launch. Outputs are
+ *     ready when the stream reaches that point.
+ *   - rows == 0 or cols == 0 is valid and launches nothing, except that the
+ *     backward writes d(alpha) = 0 for rows > 0, cols == 0.
+ *   - Any alignment is accepted. The fast path needs cols % 8 == 0, 16-byte
+ *     aligned fp32/bf16 arrays and a packed buffer aligned to 2 bytes
+ *     (2-bit codes) or 4 bytes (4-bit codes); otherwise a slower element
+ *     path with the same results runs.
+ *   - Preconditions not checked on the device: w finite, alpha finite and
+ *     > 0, and output buffers that alias no input. Violations give
+ *     unspecified results (no fault for in-bounds buffers).
+ *   - Outputs are overwritten, never accumulated into. The same inputs give
+ *     the same output bits on every run (fixed reduction order).
+ *   - Errors: arguments are checked on the host before any launch; a bad
+ *     argument returns PQ_ERR_INVALID_ARG or PQ_ERR_UNSUPPORTED and enqueues
+ *     nothing. A failed launch returns PQ_ERR_CUDA; pq_last_cuda_error()
+ *     then gives the cudaError_t value of the calling thread's last failure.
+ *
+ * Sources, by page title and section:
+ *   [P1] "ParetoQ, the strongest low-bit QAT I could find" (modelfoundations.com)
+ *   [P3] "ParetoQ: Improving Scaling Laws in Extremely Low-bit LLM
+ *        Quantization" (paperhub.cn, authors' rebuttal)
+ *   [P4] "Meta's ParetoQ compares five bit widths and puts the accuracy
+ *        cliff at 1 bit" (llmobile ticker)
+ */
+#ifndef PQ_H_
+#define PQ_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PQ_API __attribute__((visibility("default")))
+#else
+#define PQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Quantizer (level set). [P1 "Finding 3"; P1 "Paper vs. code", the dispatch
+ * SEQ for 1.58/2-bit, LSQ for 3/4-bit; P3 "why SEQ is better than LSQ"].
+ *
+ *   enum        clip on x          code c                         level (alpha units)
+ *   PQ_BINARY   [-1, 1] mask only  x >= 0 ? +1 : -1               c
+ *   PQ_TERNARY  [-0.99f, 0.99f]    rint(xc*1.5)                   c/1.5  = {-2/3, 0, 2/3}
+ *   PQ_SEQ2     [-0.99f, 0.99f]    rint(xc*2 - 0.5)               (c+0.5)/2 = {+-0.25, +-0.75}
+ *   PQ_SEQ2_B   [-0.99f, 0.99f]    rint(xc*1.5 - 0.5)             (c+0.5)/1.5 = {+-1/3, +-1}
+ *   PQ_LSQ2/3/4 [-2^(b-1), 2^(b-1)-1]  rint(xc)                   c (integer grid)
+ *
+ * rint rounds half to even; each fp32 step rounds on its own (no FMA);
+ * xc = min(max(x, lo), hi). PQ_SEQ2 is the 2-bit SEQ grid as printed on
+ * [P1]; PQ_SEQ2_B is the alternative reading whose levels are
+ * {-1.5,-0.5,0.5,1.5}/1.5. A negative argument that rounds to zero gives
+ * the level -0.0 (and a dequantized -0.0), as the floating-point formula
+ * does. The clip 0.99 is the code's 1 - 1e-2 [P1 "Paper vs. code"]. */
+typedef enum {
+    PQ_BINARY = 1,
+    PQ_TERNARY = 2,
+    PQ_SEQ2 = 3,
+    PQ_SEQ2_B = 4,
+    PQ_LSQ2 = 5,
+    PQ_LSQ3 = 6,
+    PQ_LSQ4 = 7
+} pq_quant_t;
+
+typedef enum {
+    PQ_OK = 0,
+    PQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, bad pack shape */
+    PQ_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve */
+    PQ_ERR_MISALIGNED = 3,  /* reserved: misaligned input is served by the element path */
+    PQ_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    PQ_ERR_TIMEOUT = 5      /* reserved for bounded device-side waits */
+} pq_status_t;
+
+/* Forward fake-quantization of one weight matrix.
+ * [P1 "Paper vs. code": SEQ formula alpha*(round(Clip(w/alpha)*k/2 - 0.5)
+ *  + 0.5)/k*2, per-row scale of shape (rows, 1), cast of the quantized
+ *  weight to the activation dtype; P1 "Finding 3": level sets.]
+ *
+ *   q            quantizer
+ *   rows, cols   matrix shape (>= 0)
+ *   w            fp32 [rows*cols], row-major
+ *   alpha        fp32 [rows]
+ *   wq_bf16_out  bf16 bit patterns [rows*cols]: bf16_rn(fl(level*alpha))
+ *   packed_out   nullable; uint8 [rows * cols * bits / 8] with bits =
+ *                pq_code_bits(q): two's-complement codes, 8/bits per byte,
+ *                column k*(8/bits)+i of a row in bits [bits*i+bits-1 :
+ *                bits*i] of byte k, rows back to back. Needs
+ *                cols % (8/bits) == 0, else PQ_ERR_INVALID_ARG.
+ *                [P4: ternary stored as 2-bit signed integers]
+ *   stream       cudaStream_t
+ * Algorithmic traffic: 4 B read + 2 B write per weight (+ bits/8 B packed).
+ */
+PQ_API pq_status_t pq_fakequant_fwd(pq_quant_t q, int64_t rows, int64_t cols,
+                             const float* w, const float* alpha,
+                             uint16_t* wq_bf16_out, uint8_t* packed_out,
+                             void* stream);
+
+/* Straight-through-estimator backward with the per-row scale gradient.
+ * [P1 "QAT versus PTQ": gradient passed straight through inside the
+ *  clipping range; P1 "The 2-bit recipe, in full": exactly zero outside,
+ *  while alpha keeps a boundary-value gradient from the clipped weights;
+ *  P1 "Paper vs. code": LSQ gradient for alpha with 1/sqrt(n*Qp) scaling,
+ *  gradients in FP32 against the shadow weights.]
+ *
+ *   g_bf16       bf16 bit patterns [rows*cols], the upstream dWq
+ *   dw_out       fp32 [rows*cols]: inside ? float(g) : +0.0f, where
+ *                inside = (lo <= x <= hi) on the unclipped x (closed range)
+ *   dalpha_out   fp32 [rows]: grad_scale * sum_j g_j*(level_j - inside_j*x_j),
+ *                accumulated in fp64 in a fixed order, rounded once to fp32
+ *   grad_scale   multiplies each row sum once; pq_default_grad_scale gives
+ *                the LSQ rule 1/sqrt(cols*Qp)
+ * Algorithmic traffic: 4 B + 2 B read, 4 B written per weight.
+ */
+PQ_API pq_status_t pq_fakequant_bwd(pq_quant_t q, int64_t rows, int64_t cols,
+                             const float* w, const float* alpha,
+                             const uint16_t* g_bf16, float* dw_out,
+                             float* dalpha_out, float grad_scale,
+                             void* stream);
+
+/* Packed code export only (the forward's packed_out without the bf16
+ * weights). Same layout and shape rule as packed_out above.
+ * Algorithmic traffic: 4 B read + bits/8 B written per weight. */
+PQ_API pq_status_t pq_pack_codes(pq_quant_t q, int64_t rows, int64_t cols,
+                          const float* w, const float* alpha,
+                          uint8_t* packed_out, void* stream);
+
+/* Storage width in bits of one packed code: 2 (binary, ternary, SEQ2,
+ * SEQ2_B, LSQ2) or 4 (LSQ3, LSQ4); 0 for an unknown quantizer. */
+PQ_API int pq_code_bits(pq_quant_t q);
+
+/* LSQ gradient scale 1/sqrt(cols*Qp) with n = cols weights per scale;
+ * Qp = 1 (binary, ternary, LSQ2), 1.5 (SEQ2, SEQ2_B), 3 (LSQ3), 7 (LSQ4).
+ * [P1 "Paper vs. code"]. Returns 0 for cols <= 0 or an unknown quantizer. */
+PQ_API float pq_default_grad_scale(pq_quant_t q, int64_t cols);
+
+/* Static description of a status code. */
+PQ_API const char* pq_status_string(pq_status_t s);
+
+/* cudaError_t of the calling thread's last PQ_ERR_CUDA (0 if none). */
+PQ_API int pq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PQ_H_ */
