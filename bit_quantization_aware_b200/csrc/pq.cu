@@ -362,9 +362,9 @@ static pq_status_t fwd_common(int q, int64_t rows, int64_t cols, const float* w,
                               void* stream) {
     const int bits = code_bits_of(q);
     if (bits == 0 || rows < 0 || cols < 0) return PQ_ERR_INVALID_ARG;
-    if (!wq && !packed) return PQ_ERR_INVALID_ARG;
     if (packed && (cols % (8 / bits)) != 0) return PQ_ERR_INVALID_ARG;
     if (rows == 0 || cols == 0) return PQ_OK;
+    if (!wq && !packed) return PQ_ERR_INVALID_ARG;
     if (!w || !alpha) return PQ_ERR_INVALID_ARG;
 
     const bool vec = (cols % 8 == 0) && aligned(w, 16) && (!wq || aligned(wq, 16)) &&
@@ -417,13 +417,13 @@ extern "C" {
 pq_status_t pq_fakequant_fwd(pq_quant_t q, int64_t rows, int64_t cols, const float* w,
                              const float* alpha, uint16_t* wq_bf16_out, uint8_t* packed_out,
                              void* stream) {
-    if (!wq_bf16_out) return PQ_ERR_INVALID_ARG;
+    if (!wq_bf16_out && rows > 0 && cols > 0) return PQ_ERR_INVALID_ARG;
     return fwd_common(q, rows, cols, w, alpha, wq_bf16_out, packed_out, stream);
 }
 
 pq_status_t pq_pack_codes(pq_quant_t q, int64_t rows, int64_t cols, const float* w,
                           const float* alpha, uint8_t* packed_out, void* stream) {
-    if (!packed_out) return PQ_ERR_INVALID_ARG;
+    if (!packed_out && rows > 0 && cols > 0) return PQ_ERR_INVALID_ARG;
     return fwd_common(q, rows, cols, w, alpha, nullptr, packed_out, stream);
 }
 

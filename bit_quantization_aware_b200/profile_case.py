@@ -1,0 +1,58 @@
+"""Run one weight matrix through the quantizer a few times (for profilers).
+
+    python -m bit_quantization_aware_b200.profile_case --rows 14336 --cols 4096 \
+        --quant seq2 --iters 3 [--pack]
+
+Draws seeded synthetic inputs on the device (N(0, 0.02) weights, alpha =
+max|w_row| or the quantizer's init, bf16 N(0, 1e-3) upstream gradient),
+then runs forward and backward ``iters`` times on the current stream and
+prints the per-iteration CUDA-event times. Sized by the caller; a
+14336x4096 matrix moves about 0.9 GB per iteration, more than L2.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import inputs as I
+from . import pq
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("--rows", type=int, default=14336)
+    p.add_argument("--cols", type=int, default=4096)
+    p.add_argument("--quant", default="seq2", choices=sorted(pq.QUANTIZERS))
+    p.add_argument("--iters", type=int, default=3)
+    p.add_argument("--pack", action="store_true")
+    a = p.parse_args()
+    q = pq.QUANTIZERS[a.quant]
+    dev = torch.device("cuda")
+    w = I.normal_weights(a.rows, a.cols, seed=0, stream=0, device=dev)
+    alpha = I.alpha_init(w, q)
+    g = I.grad_bf16(a.rows, a.cols, seed=0, stream=64, device=dev)
+    wq = torch.empty((a.rows, a.cols), dtype=torch.bfloat16, device=dev)
+    packed = (torch.empty((a.rows, a.cols * pq.pq_code_bits(q) // 8),
+                          dtype=torch.uint8, device=dev) if a.pack else None)
+    dw = torch.empty((a.rows, a.cols), dtype=torch.float32, device=dev)
+    da = torch.empty((a.rows,), dtype=torch.float32, device=dev)
+    gs = pq.pq_default_grad_scale(q, a.cols)
+    torch.cuda.synchronize()
+    for i in range(a.iters):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        pq.pq_fakequant_fwd(q, w, alpha, wq, packed)
+        e[1].record()
+        pq.pq_fakequant_bwd(q, w, alpha, g, dw, da, gs)
+        e[2].record()
+        torch.cuda.synchronize()
+        n = a.rows * a.cols
+        tf, tb = e[0].elapsed_time(e[1]) * 1e-3, e[1].elapsed_time(e[2]) * 1e-3
+        fb = 6 + (pq.pq_code_bits(q) / 8 if a.pack else 0)
+        print(f"iter {i}: fwd {tf * 1e6:.1f} us ({n * fb / tf / 1e9:.0f} GB/s), "
+              f"bwd {tb * 1e6:.1f} us ({n * 10 / tb / 1e9:.0f} GB/s)")
+
+
+if __name__ == "__main__":
+    main()

@@ -18,8 +18,9 @@
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and the call returns after the launch. Outputs are
  *     ready when the stream reaches that point.
- *   - rows == 0 or cols == 0 is valid and launches nothing, except that the
- *     backward writes d(alpha) = 0 for rows > 0, cols == 0.
+ *   - rows == 0 or cols == 0 is valid and launches nothing (array pointers
+ *     may then be NULL), except that the backward writes d(alpha) = 0 for
+ *     rows > 0, cols == 0 (dalpha_out must then be valid).
  *   - Any alignment is accepted. The fast path needs cols % 8 == 0, 16-byte
  *     aligned fp32/bf16 arrays and a packed buffer aligned to 2 bytes
  *     (2-bit codes) or 4 bytes (4-bit codes); otherwise a slower element

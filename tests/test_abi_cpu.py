@@ -88,6 +88,11 @@ def test_argument_errors_launch_nothing(L):
     assert f(pq.PQ_SEQ2, 4, 0, None, None, fake, None, None) == pq.PQ_OK
     assert k(pq.PQ_LSQ3, 0, 0, None, None, fake, None) == pq.PQ_OK
     assert b(pq.PQ_SEQ2, 0, 8, None, None, None, None, None, 1.0, None) == pq.PQ_OK
+    # empty shapes accept NULL arrays
+    assert f(pq.PQ_SEQ2, 0, 8, None, None, None, None, None) == pq.PQ_OK
+    assert k(pq.PQ_SEQ2, 3, 0, None, None, None, None) == pq.PQ_OK
+    # but the backward of rows > 0, cols == 0 must write d(alpha)
+    assert b(pq.PQ_SEQ2, 3, 0, None, None, None, None, None, 1.0, None) == E
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
