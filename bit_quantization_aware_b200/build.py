@@ -20,7 +20,7 @@ LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libpq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-fmad=false",
+NVCC_FLAGS = ["-O3", "-std=c++20", "-lineinfo", "-fmad=false",
               "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
               "-Xptxas", "-warn-spills", "--expt-relaxed-constexpr"]
 

@@ -1,17 +1,25 @@
 // Kernels and C ABI of the ParetoQ-style weight fake-quantizer (sm_100a).
 //
 // The path is HBM-bound elementwise work (about 10 fp32 operations per 16
-// bytes moved), so it uses no tensor cores: 16-byte vector loads and
-// stores, one row group per thread group, and a fixed-order per-row
-// reduction for the scale gradient.
+// bytes moved), so it uses no tensor cores. Design:
 //
-// Layout of the work: a CTA of 256 threads is split into row groups of TPR
-// threads (TPR a power of two, 1..256); a row group owns one row at a time
-// and walks it in chunks of 8 consecutive weights (two 16-byte loads of W,
-// one 16-byte store of bf16 Wq, one 2- or 4-byte store of packed codes).
-// The forward may also split a row across CTAs (blockIdx.x); the backward
-// keeps a row inside one row group so that the scale gradient is reduced
-// in registers, warp shuffles and shared memory, in a fixed order.
+// * Work unit = (matrix, block of rows[, column segment]). A launch covers
+//   a whole batch of matrices (up to 256 descriptors passed as kernel
+//   parameters), so a training step's many small and large matrices cost
+//   one launch per phase, with no per-matrix ramp-up and tail.
+// * A CTA of 256 threads splits into row groups of TPR threads (a power of
+//   two, 1..256, chosen per matrix so that each thread owns about eight
+//   chunks of 8 weights of its row). Each thread issues the 16-byte loads of
+//   several chunks (4 in the forward, 2 in the backward) before computing
+//   any of them.
+// * A persistent grid (the occupancy limit; the backward's registers are
+//   capped for 4 CTAs per SM) walks the units in order, so concurrent CTAs
+//   stream neighbouring rows. An optional bulk L2 prefetch of each CTA's
+//   next unit (cp.async.bulk.prefetch.L2) measured slower and is off.
+// * The backward reduces the scale gradient per row in a fixed order: fp64
+//   partial sums per thread, warp shuffles, then (TPR > 32) one shared-memory
+//   slot per warp summed by the group's first thread after a barrier of the
+//   group only.
 //
 // Sources: "ParetoQ, the strongest low-bit QAT I could find", sections
 // "Finding 3", "Paper vs. code", "QAT versus PTQ", "The 2-bit recipe, in
@@ -24,10 +32,43 @@
 #include "pq.h"
 #include "pq_quant.cuh"
 
+// Tuning knobs (compile-time; the defaults are the measured choice):
+//   PQ_PREFETCH      1: bulk L2 prefetch of each CTA's next unit
+//   PQ_CTAS_PER_SM   persistent CTAs per SM (0: the occupancy limit)
+//   PQ_CHUNKS_PER_THREAD  target chunks of 8 weights per thread and row
+//   PQ_FWD_UNROLL, PQ_BWD_UNROLL  chunks whose loads a thread issues
+//                    before computing any of them
+//   PQ_LD_HINT, PQ_ST_HINT  cache hints of the streaming loads and stores
+//   PQ_BWD_MIN_CTAS  resident CTAs per SM the backward's registers must allow
+#ifndef PQ_PREFETCH
+#define PQ_PREFETCH 0
+#endif
+#ifndef PQ_CTAS_PER_SM
+#define PQ_CTAS_PER_SM 0
+#endif
+#ifndef PQ_CHUNKS_PER_THREAD
+#define PQ_CHUNKS_PER_THREAD 8
+#endif
+#ifndef PQ_FWD_UNROLL
+#define PQ_FWD_UNROLL 4
+#endif
+#ifndef PQ_BWD_UNROLL
+#define PQ_BWD_UNROLL 2
+#endif
+#ifndef PQ_LD_HINT
+#define PQ_LD_HINT 0
+#endif
+#ifndef PQ_BWD_MIN_CTAS
+#define PQ_BWD_MIN_CTAS 4
+#endif
+#ifndef PQ_ST_HINT
+#define PQ_ST_HINT 0
+#endif
+
 namespace pq {
 
 constexpr int kThreads = 256;
-constexpr int kBlocksPerSm = 8;  // 8 x 256 = 2048 resident threads per SM
+constexpr int kMaxBatch = 256;  // descriptors per launch
 
 // ------------------------------------------------------------ memory helpers
 // Number of valid weights in chunk `ch` (8 except in a ragged last chunk).
@@ -36,9 +77,30 @@ __device__ __forceinline__ int tail_n(int64_t cols, int64_t ch) {
     return r < 8 ? static_cast<int>(r) : 8;
 }
 
+// Streaming load/store flavours (PQ_LD_HINT: 0 evict-first, 1 read-only
+// path, 2 default; PQ_ST_HINT: 0 evict-first, 1 default).
+template <typename T>
+__device__ __forceinline__ T ld_stream(const T* p) {
+#if PQ_LD_HINT == 0
+    return __ldcs(p);
+#elif PQ_LD_HINT == 1
+    return __ldg(p);
+#else
+    return *p;
+#endif
+}
+template <typename T>
+__device__ __forceinline__ void st_stream(T* p, T v) {
+#if PQ_ST_HINT == 0
+    __stcs(p, v);
+#else
+    *p = v;
+#endif
+}
+
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    const float4 a = ld_stream(reinterpret_cast<const float4*>(p));
+    const float4 b = ld_stream(reinterpret_cast<const float4*>(p) + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
@@ -49,8 +111,28 @@ __device__ __forceinline__ void load8_tail(const float* p, int n, float (&v)[8])
 }
 
 __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+    st_stream(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+    st_stream(reinterpret_cast<float4*>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+}
+
+__device__ __forceinline__ void store8_tail(float* p, int n, const float (&v)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i < n) p[i] = v[i];
+}
+
+__device__ __forceinline__ void load_g8(const uint16_t* p, uint32_t (&gw)[4]) {
+    const uint4 u = ld_stream(reinterpret_cast<const uint4*>(p));
+    gw[0] = u.x; gw[1] = u.y; gw[2] = u.z; gw[3] = u.w;
+}
+
+__device__ __forceinline__ void load_g8_tail(const uint16_t* p, int n, uint32_t (&gw)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = (2 * k < n) ? p[2 * k] : 0u;
+        const uint32_t hi = (2 * k + 1 < n) ? p[2 * k + 1] : 0u;
+        gw[k] = lo | (hi << 16);
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -58,24 +140,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
-// ------------------------------------------------------------------ forward
-// One chunk of 8 weights: bf16 outputs as 4 words, packed codes as one word
-// (bits*8 significant bits).
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes) {
+    const char* c = static_cast<const char*>(p);
+    while (bytes > 0) {
+        const uint32_t n = bytes > (1 << 20) ? (1u << 20) : static_cast<uint32_t>(bytes);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c), "r"(n) : "memory");
+        c += n;
+        bytes -= n;
+    }
+}
+
+// Barrier over the `count` threads of one row group (ids 1..8; id 0 is
+// __syncthreads). All threads of the group reach it equally often.
+__device__ __forceinline__ void group_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// ------------------------------------------------------------- chunk math
+// Forward of one chunk of 8 weights: bf16 outputs as 4 words, packed codes
+// as one word (bits*8 significant bits).
 template <int Q, bool WQ, bool PACK>
-__device__ __forceinline__ void fwd_chunk(const float (&v)[8], float a,
+__device__ __forceinline__ void fwd_chunk(const float (&v)[8], const RowScale& s,
                                           uint32_t (&h)[4], uint32_t& pk) {
     constexpr int B = Traits<Q>::bits;
+    float x[8];
+    divide8(v, s, x);
     pk = 0;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-        const Elem e0 = quantize<Q>(v[i], a);
-        const Elem e1 = quantize<Q>(v[i + 1], a);
+        const Elem e0 = quantize_x<Q>(x[i]);
+        const Elem e1 = quantize_x<Q>(x[i + 1]);
         if constexpr (WQ) {
-            h[i / 2] = pack_bf16x2(__fmul_rn(e0.level, a), __fmul_rn(e1.level, a));
+            h[i / 2] = pack_bf16x2(__fmul_rn(e0.level, s.a), __fmul_rn(e1.level, s.a));
         }
         if constexpr (PACK) {
-            pk |= code_field<Q>(e0.r) << (B * i);
-            pk |= code_field<Q>(e1.r) << (B * (i + 1));
+            pk |= code_field<Q>(e0) << (B * i);
+            pk |= code_field<Q>(e1) << (B * (i + 1));
         }
     }
 }
@@ -88,14 +189,14 @@ __device__ __forceinline__ void fwd_store(uint16_t* __restrict__ qrow,
     constexpr int B = Traits<Q>::bits;
     if constexpr (VEC) {
         if constexpr (WQ)
-            __stcs(reinterpret_cast<uint4*>(qrow + ch * 8),
-                   make_uint4(h[0], h[1], h[2], h[3]));
+            st_stream(reinterpret_cast<uint4*>(qrow + ch * 8),
+                      make_uint4(h[0], h[1], h[2], h[3]));
         if constexpr (PACK) {
             if constexpr (B == 2)
-                __stcs(reinterpret_cast<unsigned short*>(prow + ch * 2),
-                       static_cast<unsigned short>(pk));
+                st_stream(reinterpret_cast<unsigned short*>(prow + ch * 2),
+                          static_cast<unsigned short>(pk));
             else
-                __stcs(reinterpret_cast<unsigned int*>(prow + ch * 4), pk);
+                st_stream(reinterpret_cast<unsigned int*>(prow + ch * 4), pk);
         }
     } else {
         if constexpr (WQ) {
@@ -112,189 +213,231 @@ __device__ __forceinline__ void fwd_store(uint16_t* __restrict__ qrow,
     }
 }
 
+// Backward of one chunk: dW for 8 weights and their contribution to the
+// row's sum_j g_j * (level_j - inside_j * x_j), accumulated in fp64.
+template <int Q>
+__device__ __forceinline__ double bwd_chunk(const float (&v)[8], const uint32_t (&gw)[4],
+                                            const RowScale& s, float (&d)[8], double acc) {
+    float x[8];
+    divide8(v, s, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const Elem e = quantize_x<Q>(x[i]);
+        const uint32_t word = gw[i / 2];
+        const float g = (i & 1) ? __uint_as_float(word & 0xFFFF0000u)
+                                : __uint_as_float(word << 16);
+        d[i] = e.inside ? g : 0.0f;
+        const float xm = e.inside ? x[i] : 0.0f;
+        // level - xm is exact in fp64; the product and the sum round once
+        acc = __fma_rn(static_cast<double>(g),
+                       __dsub_rn(static_cast<double>(e.level), static_cast<double>(xm)), acc);
+    }
+    return acc;
+}
+
+// ------------------------------------------------------------ batches
+// Device-side descriptor of one matrix of a batch (kernel parameter space).
+struct MatDesc {
+    const float* w;
+    const float* alpha;
+    uint16_t* wq;          // forward bf16 output (nullable)
+    uint8_t* packed;       // forward packed codes (nullable)
+    const uint16_t* g;     // backward upstream gradient
+    float* dw;             // backward dW
+    float* dalpha;         // backward d(alpha)
+    int64_t rows;
+    int64_t cols;
+    int64_t unit_begin;    // first unit of this matrix in the batch
+    float grad_scale;
+    int32_t tpr_log2;      // threads per row = 1 << tpr_log2
+    int32_t col_splits;    // forward: column segments per row block
+    int32_t pad_;
+};
+
+struct Batch {
+    int32_t n;
+    int32_t pad_;
+    int64_t total_units;
+    MatDesc m[kMaxBatch];
+};
+
+// Moves `mi` forward to the matrix that owns unit u (units increase).
+__device__ __forceinline__ int find_matrix(const Batch& p, int mi, int64_t u) {
+    while (mi + 1 < p.n && p.m[mi + 1].unit_begin <= u) ++mi;
+    return mi;
+}
+
+// Bulk L2 prefetch of the inputs of unit u (vector layout only).
+template <bool BWD>
+__device__ __forceinline__ void prefetch_unit(const Batch& p, int mi, int64_t u) {
+    if (u >= p.total_units) return;
+    mi = find_matrix(p, mi, u);
+    const MatDesc& m = p.m[mi];
+    if (m.col_splits != 1) return;
+    const int64_t rpb = kThreads >> m.tpr_log2;
+    const int64_t r0 = (u - m.unit_begin) * rpb;
+    const int64_t nr = (m.rows - r0) < rpb ? (m.rows - r0) : rpb;
+    prefetch_l2(m.w + r0 * m.cols, nr * m.cols * 4);
+    if constexpr (BWD) prefetch_l2(m.g + r0 * m.cols, nr * m.cols * 2);
+}
+
+// ------------------------------------------------------------------ forward
 template <int Q, bool VEC, bool WQ, bool PACK>
 __global__ void __launch_bounds__(kThreads)
-fwd_kernel(const float* __restrict__ w, const float* __restrict__ alpha,
-           uint16_t* __restrict__ wq, uint8_t* __restrict__ packed,
-           int64_t rows, int64_t cols, int tpr_log2) {
-    const int tpr = 1 << tpr_log2;
-    const int lane = threadIdx.x & (tpr - 1);
-    const int rsub = threadIdx.x >> tpr_log2;
-    const int rpb = kThreads >> tpr_log2;
-    const int64_t nch = (cols + 7) >> 3;
-    const int64_t prow_bytes = cols * Traits<Q>::bits / 8;
-    const int64_t cstride = static_cast<int64_t>(gridDim.x) * tpr;
-
-    for (int64_t row = static_cast<int64_t>(blockIdx.y) * rpb + rsub; row < rows;
-         row += static_cast<int64_t>(gridDim.y) * rpb) {
-        const float a = __ldg(alpha + row);
-        const float* wr = w + row * cols;
-        uint16_t* qr = WQ ? wq + row * cols : nullptr;
-        uint8_t* pr = PACK ? packed + row * prow_bytes : nullptr;
-        int64_t ch = static_cast<int64_t>(blockIdx.x) * tpr + lane;
-        // two chunks per step: four 16-byte loads in flight per thread
-        for (; ch + cstride < nch; ch += 2 * cstride) {
-            const int64_t ch1 = ch + cstride;
-            float v0[8], v1[8];
-            if constexpr (VEC) {
-                load8(wr + ch * 8, v0);
-                load8(wr + ch1 * 8, v1);
-            } else {
-                load8_tail(wr + ch * 8, tail_n(cols, ch), v0);
-                load8_tail(wr + ch1 * 8, tail_n(cols, ch1), v1);
+fwd_units_kernel(const __grid_constant__ Batch p) {
+    int mi = 0;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+        mi = find_matrix(p, mi, u);
+        const MatDesc& m = p.m[mi];
+        if (VEC && PQ_PREFETCH && threadIdx.x == 0) prefetch_unit<false>(p, mi, u + gridDim.x);
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rpb = kThreads >> tl;
+        const int64_t lu = u - m.unit_begin;
+        const int64_t row = (lu / m.col_splits) * rpb + (threadIdx.x >> tl);
+        if (row >= m.rows) continue;
+        const int64_t nch = (m.cols + 7) >> 3;
+        // chunk range of this unit's column segment
+        const int64_t seg = (nch + m.col_splits - 1) / m.col_splits;
+        const int64_t c_begin = (lu % m.col_splits) * seg;
+        const int64_t c_end = (c_begin + seg) < nch ? (c_begin + seg) : nch;
+        const RowScale a = row_scale(__ldg(m.alpha + row));
+        const float* wr = m.w + row * m.cols;
+        uint16_t* qr = WQ ? m.wq + row * m.cols : nullptr;
+        uint8_t* pr = PACK ? m.packed + row * (m.cols * Traits<Q>::bits / 8) : nullptr;
+        constexpr int U = PQ_FWD_UNROLL;
+        for (int64_t ch = c_begin + lane; ch < c_end; ch += U * tpr) {
+            float v[U][8];
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int64_t c = ch + k * tpr;
+                if (c < c_end) {
+                    if constexpr (VEC) load8(wr + c * 8, v[k]);
+                    else load8_tail(wr + c * 8, tail_n(m.cols, c), v[k]);
+                }
             }
-            uint32_t h0[4], h1[4], p0, p1;
-            fwd_chunk<Q, WQ, PACK>(v0, a, h0, p0);
-            fwd_chunk<Q, WQ, PACK>(v1, a, h1, p1);
-            fwd_store<Q, VEC, WQ, PACK>(qr, pr, ch, tail_n(cols, ch), h0, p0);
-            fwd_store<Q, VEC, WQ, PACK>(qr, pr, ch1, tail_n(cols, ch1), h1, p1);
-        }
-        if (ch < nch) {
-            const int n = tail_n(cols, ch);
-            float v0[8];
-            if constexpr (VEC) load8(wr + ch * 8, v0);
-            else load8_tail(wr + ch * 8, n, v0);
-            uint32_t h0[4], p0;
-            fwd_chunk<Q, WQ, PACK>(v0, a, h0, p0);
-            fwd_store<Q, VEC, WQ, PACK>(qr, pr, ch, n, h0, p0);
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int64_t c = ch + k * tpr;
+                if (c < c_end) {
+                    uint32_t h[4], pk;
+                    fwd_chunk<Q, WQ, PACK>(v[k], a, h, pk);
+                    fwd_store<Q, VEC, WQ, PACK>(qr, pr, c, tail_n(m.cols, c), h, pk);
+                }
+            }
         }
     }
 }
 
 // ----------------------------------------------------------------- backward
-// One chunk: dW for 8 weights and their contribution to the row's
-// sum_j g_j * (level_j - inside_j * x_j), in fp64 with separate roundings.
-template <int Q>
-__device__ __forceinline__ double bwd_chunk(const float (&v)[8], const uint32_t (&gw)[4],
-                                            float a, float (&d)[8], double acc) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const Elem e = quantize<Q>(v[i], a);
-        const uint32_t word = gw[i / 2];
-        const float g = (i & 1) ? __uint_as_float(word & 0xFFFF0000u)
-                                : __uint_as_float(word << 16);
-        d[i] = e.inside ? g : 0.0f;
-        const double xm = e.inside ? static_cast<double>(e.x) : 0.0;
-        acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(g),
-                                       __dsub_rn(static_cast<double>(e.level), xm)));
-    }
-    return acc;
-}
-
-__device__ __forceinline__ void load_g8(const uint16_t* p, uint32_t (&gw)[4]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    gw[0] = u.x; gw[1] = u.y; gw[2] = u.z; gw[3] = u.w;
-}
-
-__device__ __forceinline__ void load_g8_tail(const uint16_t* p, int n, uint32_t (&gw)[4]) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = (2 * k < n) ? p[2 * k] : 0u;
-        const uint32_t hi = (2 * k + 1 < n) ? p[2 * k + 1] : 0u;
-        gw[k] = lo | (hi << 16);
-    }
-}
-
-__device__ __forceinline__ void store8_tail(float* p, int n, const float (&v)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (i < n) p[i] = v[i];
-}
-
 template <int Q, bool VEC>
-__global__ void __launch_bounds__(kThreads)
-bwd_kernel(const float* __restrict__ w, const float* __restrict__ alpha,
-           const uint16_t* __restrict__ g, float* __restrict__ dw,
-           float* __restrict__ dalpha, float grad_scale, int64_t rows,
-           int64_t cols, int tpr_log2) {
-    __shared__ double warp_sum[kThreads / 32];
-    const int tpr = 1 << tpr_log2;
-    const int lane = threadIdx.x & (tpr - 1);
-    const int rsub = threadIdx.x >> tpr_log2;
-    const int rpb = kThreads >> tpr_log2;
-    const int64_t nch = (cols + 7) >> 3;
-    const int seg = tpr < 32 ? tpr : 32;
-
+__global__ void __launch_bounds__(kThreads, PQ_BWD_MIN_CTAS)
+bwd_units_kernel(const __grid_constant__ Batch p) {
+    __shared__ double warp_sum[2][kThreads / 32];
+    int mi = 0, prev_mi = 0, parity = 0;
     // block-uniform trip count: every thread reaches every barrier
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpb; base < rows;
-         base += static_cast<int64_t>(gridDim.x) * rpb) {
-        const int64_t row = base + rsub;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x, parity ^= 1) {
+        mi = find_matrix(p, mi, u);
+        // a new matrix may regroup the threads: let every group finish
+        // reading the previous slots first
+        if (mi != prev_mi) __syncthreads();
+        prev_mi = mi;
+        const MatDesc& m = p.m[mi];
+        if (VEC && PQ_PREFETCH && threadIdx.x == 0) prefetch_unit<true>(p, mi, u + gridDim.x);
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rsub = threadIdx.x >> tl;
+        const int rpb = kThreads >> tl;
+        const int64_t row = (u - m.unit_begin) * rpb + rsub;
+        const int64_t nch = (m.cols + 7) >> 3;
         double acc = 0.0;
-        if (row < rows) {
-            const float a = __ldg(alpha + row);
-            const float* wr = w + row * cols;
-            const uint16_t* gr = g + row * cols;
-            float* dr = dw + row * cols;
-            int64_t ch = lane;
-            for (; ch + tpr < nch; ch += 2 * tpr) {
-                const int64_t ch1 = ch + tpr;
-                float v0[8], v1[8], d0[8], d1[8];
-                uint32_t g0[4], g1[4];
-                if constexpr (VEC) {
-                    load8(wr + ch * 8, v0);
-                    load_g8(gr + ch * 8, g0);
-                    load8(wr + ch1 * 8, v1);
-                    load_g8(gr + ch1 * 8, g1);
-                } else {
-                    const int n0 = tail_n(cols, ch);
-                    const int n1 = tail_n(cols, ch1);
-                    load8_tail(wr + ch * 8, n0, v0);
-                    load_g8_tail(gr + ch * 8, n0, g0);
-                    load8_tail(wr + ch1 * 8, n1, v1);
-                    load_g8_tail(gr + ch1 * 8, n1, g1);
+        if (row < m.rows) {
+            const RowScale a = row_scale(__ldg(m.alpha + row));
+            const float* wr = m.w + row * m.cols;
+            const uint16_t* gr = m.g + row * m.cols;
+            float* dr = m.dw + row * m.cols;
+            constexpr int U = PQ_BWD_UNROLL;
+            for (int64_t ch = lane; ch < nch; ch += U * tpr) {
+                float v[U][8];
+                uint32_t gw[U][4];
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t c = ch + k * tpr;
+                    if (c < nch) {
+                        if constexpr (VEC) {
+                            load8(wr + c * 8, v[k]);
+                            load_g8(gr + c * 8, gw[k]);
+                        } else {
+                            const int n = tail_n(m.cols, c);
+                            load8_tail(wr + c * 8, n, v[k]);
+                            load_g8_tail(gr + c * 8, n, gw[k]);
+                        }
+                    }
                 }
-                acc = bwd_chunk<Q>(v0, g0, a, d0, acc);
-                acc = bwd_chunk<Q>(v1, g1, a, d1, acc);
-                if constexpr (VEC) {
-                    store8(dr + ch * 8, d0);
-                    store8(dr + ch1 * 8, d1);
-                } else {
-                    store8_tail(dr + ch * 8, tail_n(cols, ch), d0);
-                    store8_tail(dr + ch1 * 8, tail_n(cols, ch1), d1);
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t c = ch + k * tpr;
+                    if (c < nch) {
+                        float d[8];
+                        acc = bwd_chunk<Q>(v[k], gw[k], a, d, acc);
+                        if constexpr (VEC) store8(dr + c * 8, d);
+                        else store8_tail(dr + c * 8, tail_n(m.cols, c), d);
+                    }
                 }
-            }
-            if (ch < nch) {
-                const int n = tail_n(cols, ch);
-                float v0[8], d0[8];
-                uint32_t g0[4];
-                if constexpr (VEC) {
-                    load8(wr + ch * 8, v0);
-                    load_g8(gr + ch * 8, g0);
-                } else {
-                    load8_tail(wr + ch * 8, n, v0);
-                    load_g8_tail(gr + ch * 8, n, g0);
-                }
-                acc = bwd_chunk<Q>(v0, g0, a, d0, acc);
-                if constexpr (VEC) store8(dr + ch * 8, d0);
-                else store8_tail(dr + ch * 8, n, d0);
             }
         }
         // reduce the row group's partial sums in a fixed order
+        const int seg = tpr < 32 ? tpr : 32;
         for (int off = seg >> 1; off > 0; off >>= 1)
             acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off, seg));
         if (tpr > 32) {
-            if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = acc;
-            __syncthreads();
+            if ((threadIdx.x & 31) == 0) warp_sum[parity][threadIdx.x >> 5] = acc;
+            group_barrier(1 + rsub, tpr);
             if (lane == 0) {
                 const int w0 = threadIdx.x >> 5;
-                double t = warp_sum[w0];
-                for (int k = 1; k < (tpr >> 5); ++k) t = __dadd_rn(t, warp_sum[w0 + k]);
+                double t = warp_sum[parity][w0];
+                for (int k = 1; k < (tpr >> 5); ++k) t = __dadd_rn(t, warp_sum[parity][w0 + k]);
                 acc = t;
             }
-            __syncthreads();
         }
-        if (lane == 0 && row < rows)
-            dalpha[row] = static_cast<float>(__dmul_rn(acc, static_cast<double>(grad_scale)));
+        if (lane == 0 && row < m.rows)
+            m.dalpha[row] = static_cast<float>(__dmul_rn(acc, static_cast<double>(m.grad_scale)));
+    }
+}
+
+// ------------------------------------------------------- scaled weights
+// x = RN(w / alpha_row) with the division routine of the quantizer kernels.
+__global__ void __launch_bounds__(kThreads)
+scaled_weights_kernel(const float* __restrict__ w, const float* __restrict__ alpha,
+                      float* __restrict__ x, int64_t rows, int64_t cols) {
+    const int64_t nch = (cols + 7) >> 3;
+    for (int64_t row = blockIdx.y; row < rows; row += gridDim.y) {
+        const RowScale s = row_scale(__ldg(alpha + row));
+        for (int64_t ch = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; ch < nch;
+             ch += static_cast<int64_t>(gridDim.x) * kThreads) {
+            const int n = tail_n(cols, ch);
+            float v[8], q[8];
+            load8_tail(w + row * cols + ch * 8, n, v);
+            divide8(v, s, q);
+            store8_tail(x + row * cols + ch * 8, n, q);
+        }
     }
 }
 
 // --------------------------------------------------------------- host side
 static thread_local int g_last_cuda_error = 0;
 
+static int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    return dev;
+}
+
 static int sm_count() {
     static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    const int dev = current_device();
     if (cached[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
@@ -314,16 +457,15 @@ static inline int ilog2_ceil(int64_t v) {
     return l;
 }
 
-// Threads per row: about two chunks of 8 per thread, 1..256.
-static inline int choose_tpr_log2(int64_t nch) {
-    int l = ilog2_ceil((nch + 1) / 2);
-    if (l > 8) l = 8;
-    if (l < 0) l = 0;
-    return l;
+// Threads per row: a power of two, 1..256, giving each thread about
+// PQ_CHUNKS_PER_THREAD chunks of 8 weights of its row.
+static inline int choose_tpr_log2(int64_t cols) {
+    const int64_t nch = (cols + 7) / 8;
+    const int l = ilog2_ceil((nch + PQ_CHUNKS_PER_THREAD - 1) / PQ_CHUNKS_PER_THREAD);
+    return l > 8 ? 8 : l;
 }
 
-static pq_status_t finish_launch() {
-    const cudaError_t e = cudaGetLastError();
+static pq_status_t cuda_status(cudaError_t e) {
     if (e != cudaSuccess) {
         g_last_cuda_error = static_cast<int>(e);
         return PQ_ERR_CUDA;
@@ -339,73 +481,207 @@ static int code_bits_of(int q) {
     }
 }
 
-template <int Q, bool VEC>
-static void launch_fwd_q(dim3 grid, cudaStream_t s, const float* w, const float* alpha,
-                         uint16_t* wq, uint8_t* packed, int64_t rows, int64_t cols, int tl) {
-    if (wq && packed)
-        fwd_kernel<Q, VEC, true, true><<<grid, kThreads, 0, s>>>(w, alpha, wq, packed, rows, cols, tl);
-    else if (wq)
-        fwd_kernel<Q, VEC, true, false><<<grid, kThreads, 0, s>>>(w, alpha, wq, packed, rows, cols, tl);
-    else
-        fwd_kernel<Q, VEC, false, true><<<grid, kThreads, 0, s>>>(w, alpha, wq, packed, rows, cols, tl);
-}
-
-template <int Q>
-static void launch_fwd_v(bool vec, dim3 grid, cudaStream_t s, const float* w, const float* alpha,
-                         uint16_t* wq, uint8_t* packed, int64_t rows, int64_t cols, int tl) {
-    if (vec) launch_fwd_q<Q, true>(grid, s, w, alpha, wq, packed, rows, cols, tl);
-    else launch_fwd_q<Q, false>(grid, s, w, alpha, wq, packed, rows, cols, tl);
-}
-
-static pq_status_t fwd_common(int q, int64_t rows, int64_t cols, const float* w,
-                              const float* alpha, uint16_t* wq, uint8_t* packed,
-                              void* stream) {
-    const int bits = code_bits_of(q);
-    if (bits == 0 || rows < 0 || cols < 0) return PQ_ERR_INVALID_ARG;
-    if (packed && (cols % (8 / bits)) != 0) return PQ_ERR_INVALID_ARG;
-    if (rows == 0 || cols == 0) return PQ_OK;
-    if (!wq && !packed) return PQ_ERR_INVALID_ARG;
-    if (!w || !alpha) return PQ_ERR_INVALID_ARG;
-
-    const bool vec = (cols % 8 == 0) && aligned(w, 16) && (!wq || aligned(wq, 16)) &&
-                     (!packed || aligned(packed, bits == 2 ? 2 : 4));
-    const int64_t nch = (cols + 7) / 8;
-    const int tl = choose_tpr_log2(nch);
-    const int64_t tpr = int64_t{1} << tl;
-    const int64_t rpb = kThreads / tpr;
-    const int64_t row_groups = (rows + rpb - 1) / rpb;
-    const int64_t target = static_cast<int64_t>(sm_count()) * kBlocksPerSm;
-    int64_t gy = row_groups < 65535 ? row_groups : 65535;
-    int64_t gx = 1;
-    if (row_groups < target) {  // few rows: split each row across CTAs too
-        const int64_t max_gx = (nch + 2 * tpr - 1) / (2 * tpr);
-        gx = (target + row_groups - 1) / row_groups;
-        if (gx > max_gx) gx = max_gx;
-        if (gx < 1) gx = 1;
-    }
-    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+// Calls f.template operator()<Q>() for the runtime quantizer q.
+template <typename F>
+static bool dispatch_q(int q, F&& f) {
     switch (q) {
-        case PQ_BINARY: launch_fwd_v<PQ_BINARY>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_TERNARY: launch_fwd_v<PQ_TERNARY>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_SEQ2: launch_fwd_v<PQ_SEQ2>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_SEQ2_B: launch_fwd_v<PQ_SEQ2_B>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_LSQ2: launch_fwd_v<PQ_LSQ2>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_LSQ3: launch_fwd_v<PQ_LSQ3>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        case PQ_LSQ4: launch_fwd_v<PQ_LSQ4>(vec, grid, s, w, alpha, wq, packed, rows, cols, tl); break;
-        default: return PQ_ERR_INVALID_ARG;
+        case PQ_BINARY: f.template operator()<PQ_BINARY>(); return true;
+        case PQ_TERNARY: f.template operator()<PQ_TERNARY>(); return true;
+        case PQ_SEQ2: f.template operator()<PQ_SEQ2>(); return true;
+        case PQ_SEQ2_B: f.template operator()<PQ_SEQ2_B>(); return true;
+        case PQ_LSQ2: f.template operator()<PQ_LSQ2>(); return true;
+        case PQ_LSQ3: f.template operator()<PQ_LSQ3>(); return true;
+        case PQ_LSQ4: f.template operator()<PQ_LSQ4>(); return true;
+        default: return false;
     }
-    return finish_launch();
 }
 
-template <int Q>
-static void launch_bwd_v(bool vec, unsigned grid, cudaStream_t s, const float* w,
-                         const float* alpha, const uint16_t* g, float* dw, float* dalpha,
-                         float gs, int64_t rows, int64_t cols, int tl) {
-    if (vec)
-        bwd_kernel<Q, true><<<grid, kThreads, 0, s>>>(w, alpha, g, dw, dalpha, gs, rows, cols, tl);
-    else
-        bwd_kernel<Q, false><<<grid, kThreads, 0, s>>>(w, alpha, g, dw, dalpha, gs, rows, cols, tl);
+// Persistent grid size of one kernel, from its occupancy (once per device).
+template <typename K>
+static int64_t persistent_ctas(K kernel, int* cache) {
+    const int dev = current_device();
+    if (cache[dev] == 0) {
+        int per_sm = PQ_CTAS_PER_SM;
+        if (per_sm <= 0 &&
+            (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
+                 cudaSuccess || per_sm <= 0))
+            per_sm = 4;
+        cache[dev] = per_sm * sm_count();
+    }
+    return cache[dev];
+}
+
+template <int Q, bool VEC, bool WQ, bool PACK>
+static void launch_fwd(const Batch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    auto k = fwd_units_kernel<Q, VEC, WQ, PACK>;
+    const int64_t ctas = persistent_ctas(k, cache);
+    const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
+    k<<<grid, kThreads, 0, s>>>(b);
+}
+
+template <int Q, bool VEC>
+static void launch_bwd(const Batch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    auto k = bwd_units_kernel<Q, VEC>;
+    const int64_t ctas = persistent_ctas(k, cache);
+    const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
+    k<<<grid, kThreads, 0, s>>>(b);
+}
+
+// ------------------------------------------------------- validation
+static bool fwd_vec_ok(const pq_matrix_t& m, int bits) {
+    return m.cols % 8 == 0 && aligned(m.w, 16) &&
+           (!m.wq_bf16_out || aligned(m.wq_bf16_out, 16)) &&
+           (!m.packed_out || aligned(m.packed_out, bits == 2 ? 2 : 4));
+}
+
+static bool bwd_vec_ok(const pq_matrix_t& m) {
+    return m.cols % 8 == 0 && aligned(m.w, 16) && aligned(m.g_bf16, 16) && aligned(m.dw_out, 16);
+}
+
+static pq_status_t check_fwd(int bits, const pq_matrix_t& m) {
+    if (m.rows < 0 || m.cols < 0) return PQ_ERR_INVALID_ARG;
+    if (m.packed_out && (m.cols % (8 / bits)) != 0) return PQ_ERR_INVALID_ARG;
+    if (m.rows == 0 || m.cols == 0) return PQ_OK;
+    if (!m.wq_bf16_out && !m.packed_out) return PQ_ERR_INVALID_ARG;
+    if (!m.w || !m.alpha) return PQ_ERR_INVALID_ARG;
+    return PQ_OK;
+}
+
+static pq_status_t check_bwd(const pq_matrix_t& m) {
+    if (m.rows < 0 || m.cols < 0) return PQ_ERR_INVALID_ARG;
+    if (m.rows == 0) return PQ_OK;
+    if (!m.dalpha_out) return PQ_ERR_INVALID_ARG;
+    if (m.cols == 0) return PQ_OK;
+    if (!m.w || !m.alpha || !m.g_bf16 || !m.dw_out) return PQ_ERR_INVALID_ARG;
+    return PQ_OK;
+}
+
+static void batch_reset(Batch& b) {
+    b.n = 0;
+    b.pad_ = 0;
+    b.total_units = 0;
+}
+
+// Appends one matrix; col_splits > 1 splits each row block's columns into
+// that many units (forward only).
+static void batch_add(Batch& b, const pq_matrix_t& m, int tl, int col_splits) {
+    MatDesc& d = b.m[b.n++];
+    d.w = m.w;
+    d.alpha = m.alpha;
+    d.wq = m.wq_bf16_out;
+    d.packed = m.packed_out;
+    d.g = m.g_bf16;
+    d.dw = m.dw_out;
+    d.dalpha = m.dalpha_out;
+    d.rows = m.rows;
+    d.cols = m.cols;
+    d.unit_begin = b.total_units;
+    d.grad_scale = m.grad_scale;
+    d.tpr_log2 = tl;
+    d.col_splits = col_splits;
+    d.pad_ = 0;
+    const int64_t rpb = kThreads >> tl;
+    b.total_units += (m.rows + rpb - 1) / rpb * col_splits;
+}
+
+// Forward over n matrices. Matrices are grouped by output kind (bf16 and
+// packed, bf16 only, packed only) and by layout (vector or element path);
+// each group goes out in launches of up to kMaxBatch descriptors.
+static pq_status_t fwd_batch_impl(int q, int32_t n, const pq_matrix_t* mats, cudaStream_t s) {
+    const int bits = code_bits_of(q);
+    if (bits == 0 || n < 0 || (n > 0 && !mats)) return PQ_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        const pq_status_t st = check_fwd(bits, mats[i]);
+        if (st != PQ_OK) return st;
+    }
+    static thread_local Batch b;
+    bool launched = false;
+    const int64_t fill = 2 * static_cast<int64_t>(sm_count());
+    for (int cls = 0; cls < 6; ++cls) {
+        const int kind = cls >> 1;   // 0: wq+packed, 1: wq only, 2: packed only
+        const bool vec = (cls & 1) == 0;
+        batch_reset(b);
+        auto flush = [&]() {
+            if (b.n == 0) return;
+            launched = true;
+            dispatch_q(q, [&]<int Q>() {
+                if (vec) {
+                    if (kind == 0) launch_fwd<Q, true, true, true>(b, s);
+                    else if (kind == 1) launch_fwd<Q, true, true, false>(b, s);
+                    else launch_fwd<Q, true, false, true>(b, s);
+                } else {
+                    if (kind == 0) launch_fwd<Q, false, true, true>(b, s);
+                    else if (kind == 1) launch_fwd<Q, false, true, false>(b, s);
+                    else launch_fwd<Q, false, false, true>(b, s);
+                }
+            });
+            batch_reset(b);
+        };
+        for (int32_t i = 0; i < n; ++i) {
+            const pq_matrix_t& m = mats[i];
+            if (m.rows == 0 || m.cols == 0) continue;
+            const int k = (m.wq_bf16_out && m.packed_out) ? 0 : (m.wq_bf16_out ? 1 : 2);
+            if (k != kind || fwd_vec_ok(m, bits) != vec) continue;
+            const int tl = choose_tpr_log2(m.cols);
+            const int64_t tpr = int64_t{1} << tl;
+            const int64_t rpb = kThreads >> tl;
+            const int64_t row_blocks = (m.rows + rpb - 1) / rpb;
+            int64_t splits = 1;
+            if (row_blocks < fill) {  // few rows: split the columns too
+                const int64_t nch = (m.cols + 7) / 8;
+                const int64_t max_splits = (nch + 2 * tpr - 1) / (2 * tpr);
+                splits = (fill + row_blocks - 1) / row_blocks;
+                if (splits > max_splits) splits = max_splits;
+                if (splits < 1) splits = 1;
+            }
+            if (b.n == kMaxBatch) flush();
+            batch_add(b, m, tl, static_cast<int>(splits));
+        }
+        flush();
+    }
+    return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
+}
+
+static pq_status_t bwd_batch_impl(int q, int32_t n, const pq_matrix_t* mats, cudaStream_t s) {
+    if (code_bits_of(q) == 0 || n < 0 || (n > 0 && !mats)) return PQ_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        const pq_status_t st = check_bwd(mats[i]);
+        if (st != PQ_OK) return st;
+    }
+    static thread_local Batch b;
+    bool launched = false;
+    for (int32_t i = 0; i < n; ++i) {  // rows without columns: d(alpha) = 0
+        const pq_matrix_t& m = mats[i];
+        if (m.rows > 0 && m.cols == 0) {
+            launched = true;
+            const pq_status_t st = cuda_status(cudaMemsetAsync(
+                m.dalpha_out, 0, static_cast<size_t>(m.rows) * sizeof(float), s));
+            if (st != PQ_OK) return st;
+        }
+    }
+    for (int cls = 0; cls < 2; ++cls) {
+        const bool vec = cls == 0;
+        batch_reset(b);
+        auto flush = [&]() {
+            if (b.n == 0) return;
+            launched = true;
+            dispatch_q(q, [&]<int Q>() {
+                if (vec) launch_bwd<Q, true>(b, s);
+                else launch_bwd<Q, false>(b, s);
+            });
+            batch_reset(b);
+        };
+        for (int32_t i = 0; i < n; ++i) {
+            const pq_matrix_t& m = mats[i];
+            if (m.rows == 0 || m.cols == 0 || bwd_vec_ok(m) != vec) continue;
+            if (b.n == kMaxBatch) flush();
+            batch_add(b, m, choose_tpr_log2(m.cols), 1);
+        }
+        flush();
+    }
+    return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
 }
 
 }  // namespace pq
@@ -418,46 +694,65 @@ pq_status_t pq_fakequant_fwd(pq_quant_t q, int64_t rows, int64_t cols, const flo
                              const float* alpha, uint16_t* wq_bf16_out, uint8_t* packed_out,
                              void* stream) {
     if (!wq_bf16_out && rows > 0 && cols > 0) return PQ_ERR_INVALID_ARG;
-    return fwd_common(q, rows, cols, w, alpha, wq_bf16_out, packed_out, stream);
+    pq_matrix_t m = {};
+    m.rows = rows;
+    m.cols = cols;
+    m.w = w;
+    m.alpha = alpha;
+    m.wq_bf16_out = wq_bf16_out;
+    m.packed_out = packed_out;
+    return fwd_batch_impl(q, 1, &m, static_cast<cudaStream_t>(stream));
 }
 
 pq_status_t pq_pack_codes(pq_quant_t q, int64_t rows, int64_t cols, const float* w,
                           const float* alpha, uint8_t* packed_out, void* stream) {
     if (!packed_out && rows > 0 && cols > 0) return PQ_ERR_INVALID_ARG;
-    return fwd_common(q, rows, cols, w, alpha, nullptr, packed_out, stream);
+    pq_matrix_t m = {};
+    m.rows = rows;
+    m.cols = cols;
+    m.w = w;
+    m.alpha = alpha;
+    m.packed_out = packed_out;
+    return fwd_batch_impl(q, 1, &m, static_cast<cudaStream_t>(stream));
 }
 
 pq_status_t pq_fakequant_bwd(pq_quant_t q, int64_t rows, int64_t cols, const float* w,
                              const float* alpha, const uint16_t* g_bf16, float* dw_out,
                              float* dalpha_out, float grad_scale, void* stream) {
-    if (code_bits_of(q) == 0 || rows < 0 || cols < 0) return PQ_ERR_INVALID_ARG;
-    if (rows == 0) return PQ_OK;
-    if (!dalpha_out) return PQ_ERR_INVALID_ARG;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cols == 0) {
-        if (cudaMemsetAsync(dalpha_out, 0, static_cast<size_t>(rows) * sizeof(float), s) != cudaSuccess)
-            return finish_launch();
-        return PQ_OK;
-    }
-    if (!w || !alpha || !g_bf16 || !dw_out) return PQ_ERR_INVALID_ARG;
-    const bool vec = (cols % 8 == 0) && aligned(w, 16) && aligned(g_bf16, 16) && aligned(dw_out, 16);
+    pq_matrix_t m = {};
+    m.rows = rows;
+    m.cols = cols;
+    m.w = w;
+    m.alpha = alpha;
+    m.g_bf16 = g_bf16;
+    m.dw_out = dw_out;
+    m.dalpha_out = dalpha_out;
+    m.grad_scale = grad_scale;
+    return bwd_batch_impl(q, 1, &m, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w, const float* alpha,
+                              float* x_out, void* stream) {
+    if (rows < 0 || cols < 0) return PQ_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return PQ_OK;
+    if (!w || !alpha || !x_out) return PQ_ERR_INVALID_ARG;
     const int64_t nch = (cols + 7) / 8;
-    const int tl = choose_tpr_log2(nch);
-    const int64_t rpb = kThreads >> tl;
-    const int64_t row_groups = (rows + rpb - 1) / rpb;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * kBlocksPerSm * 4;
-    const unsigned grid = static_cast<unsigned>(row_groups < cap ? row_groups : cap);
-    switch (q) {
-        case PQ_BINARY: launch_bwd_v<PQ_BINARY>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_TERNARY: launch_bwd_v<PQ_TERNARY>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_SEQ2: launch_bwd_v<PQ_SEQ2>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_SEQ2_B: launch_bwd_v<PQ_SEQ2_B>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_LSQ2: launch_bwd_v<PQ_LSQ2>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_LSQ3: launch_bwd_v<PQ_LSQ3>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        case PQ_LSQ4: launch_bwd_v<PQ_LSQ4>(vec, grid, s, w, alpha, g_bf16, dw_out, dalpha_out, grad_scale, rows, cols, tl); break;
-        default: return PQ_ERR_INVALID_ARG;
-    }
-    return finish_launch();
+    int64_t gx = (nch + kThreads - 1) / kThreads;
+    if (gx > 1024) gx = 1024;
+    const int64_t gy = rows < 65535 ? rows : 65535;
+    scaled_weights_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kThreads,
+                            0, static_cast<cudaStream_t>(stream)>>>(w, alpha, x_out, rows, cols);
+    return cuda_status(cudaGetLastError());
+}
+
+pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,
+                                   void* stream) {
+    return fwd_batch_impl(q, n, mats, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_fakequant_bwd_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,
+                                   void* stream) {
+    return bwd_batch_impl(q, n, mats, static_cast<cudaStream_t>(stream));
 }
 
 int pq_code_bits(pq_quant_t q) { return code_bits_of(q); }

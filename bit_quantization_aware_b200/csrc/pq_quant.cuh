@@ -63,36 +63,111 @@ struct Traits<PQ_LSQ4> {
 // reference in the parity tests), so no division is needed for the levels.
 constexpr float kTwoThirds = 2.0f / 3.0f;
 
+// ------------------------------------------------------------ x = w / alpha
+// Per-row scale: alpha, its correctly rounded reciprocal, and whether the
+// reciprocal-based quotient may be used for this row.
+struct RowScale {
+    float a;
+    float y;    // RN(1 / alpha)
+    bool fast;  // alpha in [2^-60, 2^60]
+};
+
+__device__ __forceinline__ RowScale row_scale(float a) {
+    RowScale s;
+    s.a = a;
+    s.y = __frcp_rn(a);
+    s.fast = (a >= 0x1p-60f) && (a <= 0x1p60f);
+    return s;
+}
+
+// RN(w / alpha) from y = RN(1 / alpha) with fused multiply-adds only:
+// q0 = RN(w*y) is within two ulps of the quotient, one remainder step
+// brings q1 within one ulp, and then, with the exact remainder
+// r1 = w - alpha*q1, RN(q1 + r1*y) is the correctly rounded quotient
+// (Markstein's theorem on the final correction of a quotient). The
+// magnitude guards keep every intermediate a normal number, which the
+// theorem needs; outside them the IEEE division runs instead.
+__device__ __forceinline__ float div_fast(float w, const RowScale& s) {
+    const float q0 = __fmul_rn(w, s.y);
+    const float r0 = __fmaf_rn(-s.a, q0, w);
+    const float q1 = __fmaf_rn(r0, s.y, q0);
+    const float r1 = __fmaf_rn(-s.a, q1, w);
+    return __fmaf_rn(r1, s.y, q1);
+}
+
+__device__ __forceinline__ bool div_fast_ok(float w) {
+    const float m = fabsf(w);
+    return m >= 0x1p-60f && m <= 0x1p60f;
+}
+
+// x[i] = RN(v[i] / alpha) for one chunk of 8 weights.
+__device__ __forceinline__ void divide8(const float (&v)[8], const RowScale& s,
+                                        float (&x)[8]) {
+    bool all = s.fast;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[i] = div_fast(v[i], s);
+        all = all && div_fast_ok(v[i]);
+    }
+    if (!all) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (!s.fast || !div_fast_ok(v[i])) x[i] = __fdiv_rn(v[i], s.a);
+    }
+}
+
+// ---------------------------------------------------------- x -> level
+// Round half to even for |t| < 2^22: t + 1.5*2^23 lies in [2^23, 2^24),
+// where floats are spaced by 1, so the addition rounds t to an integer
+// with ties to even (1.5*2^23 is even); subtracting the constant again is
+// exact. The low bits of the sum's encoding hold that integer in two's
+// complement, since the constant's low 22 mantissa bits are zero.
+constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23
+
 struct Elem {
-    float x;      // fl(w / alpha)
-    float r;      // integer-valued rounded code (may be -0.0)
-    float level;  // level in alpha units
-    bool inside;  // lo <= x <= hi (STE gate, closed range)
+    float level;    // level in alpha units (a zero level keeps the sign of t)
+    bool inside;    // lo <= x <= hi (STE gate, closed range)
+    uint32_t code;  // two's-complement code in the low Traits<Q>::bits bits
 };
 
 template <int Q>
-__device__ __forceinline__ Elem quantize(float w, float alpha) {
+__device__ __forceinline__ Elem quantize_x(float x) {
     using T = Traits<Q>;
     Elem e;
-    e.x = __fdiv_rn(w, alpha);
-    e.inside = (e.x >= T::lo) && (e.x <= T::hi);
-    if constexpr (Q == PQ_BINARY) {
-        e.r = (e.x >= 0.0f) ? 1.0f : -1.0f;
-        e.level = e.r;
+    if constexpr (T::lo == -T::hi) {
+        e.inside = fabsf(x) <= T::hi;  // same as lo <= x <= hi
     } else {
-        const float xc = fminf(fmaxf(e.x, T::lo), T::hi);
+        e.inside = (x >= T::lo) && (x <= T::hi);
+    }
+    if constexpr (Q == PQ_BINARY) {
+        const bool pos = x >= 0.0f;  // sign(+-0) = +1
+        e.level = pos ? 1.0f : -1.0f;
+        e.code = pos ? 1u : 3u;
+    } else {
+        const float xc = fminf(fmaxf(x, T::lo), T::hi);
+        float t;
         if constexpr (Q == PQ_SEQ2) {
-            e.r = rintf(__fsub_rn(__fmul_rn(xc, 2.0f), 0.5f));
-            e.level = __fmul_rn(__fadd_rn(e.r, 0.5f), 0.5f);
+            t = __fmaf_rn(xc, 2.0f, -0.5f);  // 2*xc is exact: one rounding
         } else if constexpr (Q == PQ_SEQ2_B) {
-            e.r = rintf(__fsub_rn(__fmul_rn(xc, 1.5f), 0.5f));
-            e.level = __fmul_rn(__fadd_rn(e.r, 0.5f), kTwoThirds);
+            t = __fsub_rn(__fmul_rn(xc, 1.5f), 0.5f);  // two roundings
         } else if constexpr (Q == PQ_TERNARY) {
-            e.r = rintf(__fmul_rn(xc, 1.5f));
-            e.level = __fmul_rn(e.r, kTwoThirds);
+            t = __fmul_rn(xc, 1.5f);
         } else {  // LSQ integer grid
-            e.r = rintf(xc);
-            e.level = e.r;
+            t = xc;
+        }
+        const float tm = __fadd_rn(t, kRoundShift);
+        float r = __fsub_rn(tm, kRoundShift);
+        e.code = __float_as_uint(tm);
+        if constexpr (Q == PQ_SEQ2) {
+            e.level = __fmaf_rn(r, 0.5f, 0.25f);  // (r + 0.5)/2, exact
+        } else if constexpr (Q == PQ_SEQ2_B) {
+            // (r + 0.5) * fl(2/3) rounded once, as r*c + 0.5*c fused
+            e.level = __fmaf_rn(r, kTwoThirds, 0.5f * kTwoThirds);
+        } else if constexpr (Q == PQ_TERNARY) {
+            r = copysignf(r, t);  // round(-0.3) is -0.0
+            e.level = __fmul_rn(r, kTwoThirds);
+        } else {
+            e.level = copysignf(r, t);
         }
     }
     return e;
@@ -100,9 +175,9 @@ __device__ __forceinline__ Elem quantize(float w, float alpha) {
 
 // Two's-complement code field of width Traits<Q>::bits.
 template <int Q>
-__device__ __forceinline__ uint32_t code_field(float r) {
+__device__ __forceinline__ uint32_t code_field(const Elem& e) {
     constexpr uint32_t mask = (1u << Traits<Q>::bits) - 1u;
-    return static_cast<uint32_t>(__float2int_rz(r)) & mask;
+    return e.code & mask;
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) {

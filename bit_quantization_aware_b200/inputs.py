@@ -88,6 +88,8 @@ def alpha_init(w: torch.Tensor, q: int, *, lsq_rule: str = "lsq") -> torch.Tenso
     paper's 2*mean|w_row|/sqrt(Qp) (``lsq_rule="lsq"``) or max|w_row|/Qp
     (``lsq_rule="max"``).
     """
+    if w.shape[1] == 0:  # empty rows: any positive scale
+        return torch.ones(w.shape[0], dtype=torch.float32, device=w.device)
     a = w.abs()
     if q in (SEQ2, SEQ2_B, TERNARY):
         out = a.amax(dim=1)

@@ -41,8 +41,23 @@ class PQError(RuntimeError):
         self.status = status
 
 
+class PQMatrix(ctypes.Structure):
+    """``pq_matrix_t``: one weight matrix of a batched call (device pointers)."""
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("w", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("wq_bf16_out", ctypes.c_void_p), ("packed_out", ctypes.c_void_p),
+                ("g_bf16", ctypes.c_void_p), ("dw_out", ctypes.c_void_p),
+                ("dalpha_out", ctypes.c_void_p), ("grad_scale", ctypes.c_float)]
+
+
 def _declare(L):
     i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.pq_fakequant_fwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
+    L.pq_fakequant_fwd_batch.restype = i32
+    L.pq_fakequant_bwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
+    L.pq_fakequant_bwd_batch.restype = i32
+    L.pq_scaled_weights.argtypes = [i64, i64, p, p, p, p]
+    L.pq_scaled_weights.restype = i32
     L.pq_fakequant_fwd.argtypes = [i32, i64, i64, p, p, p, p, p]
     L.pq_fakequant_fwd.restype = i32
     L.pq_fakequant_bwd.argtypes = [i32, i64, i64, p, p, p, p, p, f32, p]
@@ -131,6 +146,41 @@ def pq_pack_codes(q, w, alpha, packed_out, stream=None, rows=None, cols=None):
     _check("pq_pack_codes", lib().pq_pack_codes(
         q, rows, cols, _ptr(w), _ptr(alpha), _ptr(packed_out),
         _stream(stream)))
+
+
+def pq_scaled_weights(w, alpha, x_out, stream=None, rows=None, cols=None):
+    """x = fl(w / alpha_row) (fp32 [rows, cols])."""
+    rows, cols = _shape(w, rows, cols)
+    _check("pq_scaled_weights", lib().pq_scaled_weights(
+        rows, cols, _ptr(w), _ptr(alpha), _ptr(x_out), _stream(stream)))
+
+
+def matrix_array(descs):
+    """Build a ``pq_matrix_t[]`` from dicts with keys rows, cols, w, alpha,
+    wq, packed, g, dw, dalpha, grad_scale (tensors or raw pointers; missing
+    keys are NULL / 0)."""
+    arr = (PQMatrix * len(descs))()
+    for i, d in enumerate(descs):
+        m = arr[i]
+        m.rows, m.cols = int(d["rows"]), int(d["cols"])
+        m.w, m.alpha = _ptr(d.get("w")), _ptr(d.get("alpha"))
+        m.wq_bf16_out, m.packed_out = _ptr(d.get("wq")), _ptr(d.get("packed"))
+        m.g_bf16, m.dw_out = _ptr(d.get("g")), _ptr(d.get("dw"))
+        m.dalpha_out = _ptr(d.get("dalpha"))
+        m.grad_scale = float(d.get("grad_scale", 0.0))
+    return arr
+
+
+def pq_fakequant_fwd_batch(q, mats, stream=None):
+    """Forward over a ``pq_matrix_t[]`` (see ``matrix_array``)."""
+    _check("pq_fakequant_fwd_batch", lib().pq_fakequant_fwd_batch(
+        q, len(mats), mats, _stream(stream)))
+
+
+def pq_fakequant_bwd_batch(q, mats, stream=None):
+    """Backward over a ``pq_matrix_t[]`` (see ``matrix_array``)."""
+    _check("pq_fakequant_bwd_batch", lib().pq_fakequant_bwd_batch(
+        q, len(mats), mats, _stream(stream)))
 
 
 def pq_code_bits(q) -> int:

@@ -40,7 +40,8 @@ class QuantStep:
     """Buffers and launches for one quantizer over a list of matrices."""
 
     def __init__(self, mats, q: int, device="cuda", pack: bool = False,
-                 alloc_outputs: bool = True):
+                 alloc_outputs: bool = True, batched: bool = True):
+        self.batched = batched
         self.mats = list(mats)
         self.q = q
         self.pack = pack
@@ -80,6 +81,14 @@ class QuantStep:
                     m.rows, m.cols * bits // 8) if pack else None),
                 grad_scale=pq.pq_default_grad_scale(q, m.cols)))
 
+        self._fwd_descs = pq.matrix_array([
+            dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, wq=b.wq,
+                 packed=b.packed) for b in self.bufs])
+        self._bwd_descs = pq.matrix_array([
+            dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
+                 dw=b.dw, dalpha=b.dalpha, grad_scale=b.grad_scale)
+            for b in self.bufs])
+
     @property
     def weights(self) -> int:
         return sum(m.numel for m in self.mats)
@@ -106,10 +115,18 @@ class QuantStep:
                         device=self.device, out=b.g)
 
     def fwd_all(self, stream=None):
+        """Forward of every matrix: one batched call (or one call each)."""
+        if self.batched:
+            pq.pq_fakequant_fwd_batch(self.q, self._fwd_descs, stream)
+            return
         for b in self.bufs:
             pq.pq_fakequant_fwd(self.q, b.w, b.alpha, b.wq, b.packed, stream)
 
     def bwd_all(self, stream=None):
+        """Backward of every matrix: one batched call (or one call each)."""
+        if self.batched:
+            pq.pq_fakequant_bwd_batch(self.q, self._bwd_descs, stream)
+            return
         for b in self.bufs:
             pq.pq_fakequant_bwd(self.q, b.w, b.alpha, b.g, b.dw, b.dalpha,
                                 b.grad_scale, stream)
@@ -120,4 +137,8 @@ class QuantStep:
 
     @property
     def launches_per_step(self) -> int:
+        """Kernel launches of one step (all matrices use the vector layout:
+        one launch per 256 matrices per phase when batched)."""
+        if self.batched:
+            return 2 * ((len(self.mats) + 255) // 256)
         return 2 * len(self.mats)

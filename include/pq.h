@@ -145,6 +145,49 @@ PQ_API pq_status_t pq_pack_codes(pq_quant_t q, int64_t rows, int64_t cols,
                           const float* w, const float* alpha,
                           uint8_t* packed_out, void* stream);
 
+/* One weight matrix of a batched call. The forward reads rows, cols, w,
+ * alpha and writes wq_bf16_out and/or packed_out (at least one non-NULL when
+ * the matrix is not empty); the backward reads rows, cols, w, alpha, g_bf16,
+ * grad_scale and writes dw_out and dalpha_out. Fields a call does not use
+ * are ignored. Layouts and rules are those of the single-matrix calls. */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    const float* w;
+    const float* alpha;
+    uint16_t* wq_bf16_out;
+    uint8_t* packed_out;
+    const uint16_t* g_bf16;
+    float* dw_out;
+    float* dalpha_out;
+    float grad_scale;
+} pq_matrix_t;
+
+/* Forward over n matrices in as few launches as possible (one per 256
+ * matrices of the vector layout and output kind; the element path runs per
+ * matrix). `mats` is a HOST array read during the call only; descriptors
+ * travel as kernel parameters, so nothing is allocated. Equivalent to n
+ * calls of pq_fakequant_fwd (or pq_pack_codes when wq_bf16_out is NULL)
+ * on the same stream. All descriptors are validated before any launch. */
+PQ_API pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n,
+                                          const pq_matrix_t* mats, void* stream);
+
+/* Backward over n matrices, batched like pq_fakequant_fwd_batch; equivalent
+ * to n calls of pq_fakequant_bwd on the same stream. */
+PQ_API pq_status_t pq_fakequant_bwd_batch(pq_quant_t q, int32_t n,
+                                          const pq_matrix_t* mats, void* stream);
+
+/* Scaled weights x = fl(w / alpha_row): the first step of every quantizer,
+ * computed by the same device routine as the forward and backward kernels
+ * (the correctly rounded fp32 quotient; [P1 "Paper vs. code": the
+ * quantizer clips and rounds w/alpha]). Useful to inspect a layer's
+ * distribution in alpha units and to check the division on its own.
+ *   w      fp32 [rows*cols] (any alignment), alpha fp32 [rows]
+ *   x_out  fp32 [rows*cols], overwritten
+ * Traffic: 4 B read + 4 B written per weight. */
+PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
+                                     const float* alpha, float* x_out, void* stream);
+
 /* Storage width in bits of one packed code: 2 (binary, ternary, SEQ2,
  * SEQ2_B, LSQ2) or 4 (LSQ3, LSQ4); 0 for an unknown quantizer. */
 PQ_API int pq_code_bits(pq_quant_t q);

@@ -29,6 +29,8 @@ def declared():
 def test_header_declares_entry_points():
     names = declared()
     for n in ("pq_fakequant_fwd", "pq_fakequant_bwd", "pq_pack_codes",
+              "pq_fakequant_fwd_batch", "pq_fakequant_bwd_batch",
+              "pq_scaled_weights",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
               "pq_last_cuda_error"):
         assert n in names
@@ -88,6 +90,11 @@ def test_argument_errors_launch_nothing(L):
     assert f(pq.PQ_SEQ2, 4, 0, None, None, fake, None, None) == pq.PQ_OK
     assert k(pq.PQ_LSQ3, 0, 0, None, None, fake, None) == pq.PQ_OK
     assert b(pq.PQ_SEQ2, 0, 8, None, None, None, None, None, 1.0, None) == pq.PQ_OK
+    sw = L.pq_scaled_weights
+    assert sw(-1, 8, fake, fake, fake, None) == E
+    assert sw(4, 8, None, fake, fake, None) == E
+    assert sw(4, 8, fake, fake, None, None) == E
+    assert sw(0, 8, None, None, None, None) == pq.PQ_OK
     # empty shapes accept NULL arrays
     assert f(pq.PQ_SEQ2, 0, 8, None, None, None, None, None) == pq.PQ_OK
     assert k(pq.PQ_SEQ2, 3, 0, None, None, None, None) == pq.PQ_OK
@@ -104,3 +111,30 @@ def test_binding_fails_loudly_without_library(tmp_path):
             pq.lib(os.path.join(tmp_path, "missing.so"))
     finally:
         pq._lib = saved
+
+
+def test_batch_argument_errors_launch_nothing(L):
+    from bit_quantization_aware_b200 import pq
+    E = pq.PQ_ERR_INVALID_ARG
+    fake = 0x10000
+    good = dict(rows=4, cols=8, w=fake, alpha=fake, wq=fake, g=fake, dw=fake,
+                dalpha=fake, grad_scale=1.0)
+    arr = pq.matrix_array([good])
+    assert L.pq_fakequant_fwd_batch(99, 1, arr, None) == E
+    assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, -1, arr, None) == E
+    assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, 1, None, None) == E
+    assert L.pq_fakequant_bwd_batch(pq.PQ_SEQ2, 1, None, None) == E
+    # one bad descriptor anywhere rejects the whole call before any launch
+    for bad in (dict(good, rows=-1), dict(good, w=None), dict(good, wq=None),
+                dict(good, cols=6, packed=fake)):
+        arr = pq.matrix_array([dict(good, rows=0)] * 3 + [bad])
+        assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, 4, arr, None) == E
+    for bad in (dict(good, dalpha=None), dict(good, g=None), dict(good, cols=-2)):
+        arr = pq.matrix_array([dict(good, rows=0), bad])
+        assert L.pq_fakequant_bwd_batch(pq.PQ_SEQ2, 2, arr, None) == E
+    # empty batches and empty matrices launch nothing
+    assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, 0, None, None) == pq.PQ_OK
+    arr = pq.matrix_array([dict(rows=0, cols=8), dict(rows=3, cols=0)])
+    assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, 2, arr, None) == pq.PQ_OK
+    arr = pq.matrix_array([dict(rows=0, cols=8)])
+    assert L.pq_fakequant_bwd_batch(pq.PQ_SEQ2, 1, arr, None) == pq.PQ_OK

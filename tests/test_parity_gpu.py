@@ -262,3 +262,168 @@ def test_idempotence_on_gpu(q):
     w2 = wq.float().cpu()
     wq2, *_ = run_gpu(q, w2, a, g, False)
     assert torch.equal(wq.view(torch.int16), wq2.view(torch.int16))
+
+
+def _batch_case(q, shapes, seed, pack):
+    """Inputs, outputs and descriptors for a batch of matrices; every other
+    matrix is offset by one element (misaligned: element path)."""
+    bits = pq.pq_code_bits(q)
+    items, fwd_d, bwd_d = [], [], []
+    for i, (rows, cols) in enumerate(shapes):
+        off = 1 if i % 3 == 2 else 0
+        w, a, g = make_case(rows, cols, q, seed=seed + i, special=rows * cols >= 8)
+        n = rows * cols
+        wbuf = torch.empty(n + off + 8, dtype=torch.float32, device=DEV)
+        gbuf = torch.empty(n + off + 8, dtype=torch.bfloat16, device=DEV)
+        qbuf = torch.empty(n + off + 8, dtype=torch.bfloat16, device=DEV)
+        dbuf = torch.empty(n + off + 8, dtype=torch.float32, device=DEV)
+        wd, gd = wbuf[off:off + n], gbuf[off:off + n]
+        wd.copy_(w.reshape(-1)); gd.copy_(g.reshape(-1))
+        ad = a.to(DEV)
+        can_pack = pack and cols % (8 // bits) == 0
+        pk = (torch.zeros(n * bits // 8 + 8, dtype=torch.uint8, device=DEV)[:n * bits // 8]
+              if can_pack else None)
+        da = torch.full((rows,), float("nan"), device=DEV)
+        gs = pq.pq_default_grad_scale(q, cols)
+        items.append((w, a, g, qbuf[off:off + n], pk, dbuf[off:off + n], da, gs, rows, cols))
+        fwd_d.append(dict(rows=rows, cols=cols, w=wd, alpha=ad, wq=qbuf[off:off + n], packed=pk))
+        bwd_d.append(dict(rows=rows, cols=cols, w=wd, alpha=ad, g=gd, dw=dbuf[off:off + n],
+                          dalpha=da, grad_scale=gs))
+    return items, pq.matrix_array(fwd_d), pq.matrix_array(bwd_d)
+
+
+@pytest.mark.parametrize("q", ALLQ)
+def test_batched_calls_match_oracle(q):
+    """One batched forward and one batched backward over matrices of mixed
+    shapes, alignments and empty ones; each compared with the oracle."""
+    shapes = [(256, 1024), (1, 8), (3, 24), (5, 12), (64, 4096), (0, 8),
+              (7, 1000), (9, 1001), (33, 1032), (2, 70000), (300, 264), (4, 0)]
+    items, fd, bd = _batch_case(q, shapes, seed=20, pack=True)
+    pq.pq_fakequant_fwd_batch(q, fd)
+    pq.pq_fakequant_bwd_batch(q, bd)
+    torch.cuda.synchronize()
+    for w, a, g, wq, pk, dw, da, gs, rows, cols in items:
+        if rows == 0:
+            continue
+        if cols == 0:
+            assert torch.all(da == 0)
+            continue
+        wn, an, gn = np_inputs(w, a, g)
+        check_fwd(q, wn, an, wq.view(rows, cols),
+                  pk.view(rows, -1) if pk is not None else None)
+        check_bwd(q, wn, an, gn, gs, dw.view(rows, cols), da)
+
+
+def test_batch_of_more_than_256_matrices():
+    """300 matrices in one call: the library splits the launches."""
+    q = pq.PQ_SEQ2
+    shapes = [(3 + i % 5, 8 * (1 + i % 7)) for i in range(300)]
+    items, fd, bd = _batch_case(q, shapes, seed=40, pack=True)
+    pq.pq_fakequant_fwd_batch(q, fd)
+    pq.pq_fakequant_bwd_batch(q, bd)
+    torch.cuda.synchronize()
+    for w, a, g, wq, pk, dw, da, gs, rows, cols in items:
+        wn, an, gn = np_inputs(w, a, g)
+        check_fwd(q, wn, an, wq.view(rows, cols), pk.view(rows, -1))
+        check_bwd(q, wn, an, gn, gs, dw.view(rows, cols), da)
+
+
+def test_batched_step_equals_per_matrix_calls():
+    """The 1B stack: batched calls give the same bits as one call per
+    matrix."""
+    mats = I.llama_1b_stack()[:14]
+    s1 = QuantStep(mats, pq.PQ_SEQ2, device=DEV, pack=True, batched=True)
+    s1.generate(seed=9)
+    s2 = QuantStep(mats, pq.PQ_SEQ2, device=DEV, pack=True, batched=False)
+    s2.w_all.copy_(s1.w_all); s2.g_all.copy_(s1.g_all); s2.alpha_all.copy_(s1.alpha_all)
+    s1.run(); s2.run()
+    torch.cuda.synchronize()
+    for x, y in ((s1.wq_all, s2.wq_all), (s1.packed_all, s2.packed_all),
+                 (s1.dw_all, s2.dw_all), (s1.dalpha_all, s2.dalpha_all)):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def _special_alphas():
+    # 1, 1-2^-24, 2-2^-23, mantissa all ones, 0.02, 2, 0.5+ulp, 2^-60 and
+    # its neighbours, 2^60 and its neighbours, smallest normal, a
+    # subnormal, 2^126, 0.05
+    bits = [0x3F800000, 0x3F7FFFFF, 0x3FFFFFFF, 0x3C7FFFFF, 0x3CA3D70A,
+            0x40000000, 0x3F000001, 0x21800000, 0x217FFFFF, 0x21800001,
+            0x5D800000, 0x5D7FFFFF, 0x5D800001, 0x00800000, 0x00000400,
+            0x7E800000, 0x3D4CCCCD]
+    rng = np.random.default_rng(31)
+    rnd = np.exp(rng.uniform(np.log(1e-30), np.log(1e30), 49)).astype(np.float32)
+    return np.concatenate([np.array(bits, np.uint32).view(np.float32), rnd])
+
+
+def test_scaled_weights_match_ieee_division():
+    """x = fl(w/alpha) from the library's division routine equals numpy's
+    IEEE fp32 division, bit for bit, over a strided sweep of all finite
+    fp32 bit patterns of w (both signs, every exponent) for 64 scales,
+    among them mantissas of all ones, powers of two, the edges of the
+    reciprocal path's range (2^-60, 2^60), a subnormal and a huge one."""
+    alphas = _special_alphas()
+    stride = 2053  # odd: every residue of the low mantissa bits appears
+    pos = np.arange(0, 0x7F800000, stride, dtype=np.uint32)
+    pats = np.concatenate([pos, pos | np.uint32(0x80000000)]).view(np.float32)
+    cols = len(pats) // 8 * 8
+    pats = pats[:cols]
+    w = torch.from_numpy(np.ascontiguousarray(pats)).to(DEV)
+    x = torch.empty(cols, dtype=torch.float32, device=DEV)
+    for a in alphas:
+        ad = torch.tensor([a], dtype=torch.float32, device=DEV)
+        pq.pq_scaled_weights(w, ad, x, rows=1, cols=cols)
+        torch.cuda.synchronize()
+        with np.errstate(over="ignore", under="ignore", divide="ignore"):
+            want = (pats / np.float32(a)).astype(np.float32)
+        got = x.cpu().numpy()
+        bad = np.flatnonzero(got.view(np.uint32) != want.view(np.uint32))
+        assert bad.size == 0, (f"alpha={a!r}: {bad.size} mismatches, e.g. "
+                               f"w={pats[bad[0]]!r} gpu={got[bad[0]]!r} "
+                               f"ieee={want[bad[0]]!r}")
+
+
+def _threshold_targets(q):
+    third = float(np.float32(1.0) / np.float32(3.0))
+    base = [-0.99, 0.99, -0.5, 0.0, 0.5, -third, third, -1.0, 1.0, -0.25, 0.25]
+    if q in (pq.PQ_LSQ2, pq.PQ_LSQ3, pq.PQ_LSQ4):
+        b = {pq.PQ_LSQ2: 2, pq.PQ_LSQ3: 3, pq.PQ_LSQ4: 4}[q]
+        lo, hi = -(2 ** (b - 1)), 2 ** (b - 1) - 1
+        base += [k + 0.5 for k in range(lo - 1, hi + 1)] + [float(lo), float(hi)]
+    return np.array(base, np.float32)
+
+
+@pytest.mark.parametrize("q", ALLQ)
+def test_weights_on_code_and_clip_boundaries(q):
+    """For 512 scales, weights within 6 ulps of w = target*alpha for every
+    rounding tie and clip bound of the quantizer: the places where a
+    one-ulp error in w/alpha would flip a code or the STE mask."""
+    rng = np.random.default_rng(37 + q)
+    alphas = np.concatenate([_special_alphas()[:17],
+                             np.exp(rng.uniform(np.log(1e-3), np.log(10.0), 500))]
+                            ).astype(np.float32)
+    tg = _threshold_targets(q)
+    ks = np.arange(-6, 7)
+    rows = []
+    for a in alphas:
+        w0 = (tg.astype(np.float32) * a).astype(np.float32)
+        cand = w0[:, None].view(np.int32).astype(np.int64) + np.sign(w0[:, None] + 0).astype(
+            np.int64) * ks[None, :]
+        tiny = np.where(ks >= 0, ks, 0x80000000 | -ks).astype(np.int64)
+        cand = np.where(w0[:, None] == 0, tiny[None, :], cand)
+        row = (cand & 0xFFFFFFFF).astype(np.uint32).view(np.float32).ravel()
+        row = row[np.isfinite(row)]
+        rows.append(row)
+    cols = max(len(r) for r in rows)
+    cols = (cols + 7) // 8 * 8
+    W = np.zeros((len(rows), cols), np.float32)
+    for i, r in enumerate(rows):
+        W[i, :len(r)] = r
+    w = torch.from_numpy(W)
+    a = torch.from_numpy(alphas)
+    g = I.grad_bf16(len(rows), cols, seed=7, stream=77 + q, device="cpu")
+    wq, pk, pk2, dw, da, gs = run_gpu(q, w, a, g, True)
+    wn, an, gn = np_inputs(w, a, g)
+    check_fwd(q, wn, an, wq, pk)
+    check_fwd(q, wn, an, None, pk2)
+    check_bwd(q, wn, an, gn, gs, dw, da)
