@@ -92,6 +92,23 @@ def recorded_traffic():
     return d
 
 
+# ------------------------------------------------------------- rank logic
+def reduce_max(values, device, world):
+    """Element-wise max over ranks (timings: the slowest rank decides)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def step_throughput(weights_per_rank, world, ms_per_step):
+    """Whole-job Gweights/s: the weights every rank processed in one step
+    over the (max-over-ranks) step time."""
+    return weights_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of SM clocks and throttle reasons during the timed
@@ -269,7 +286,7 @@ def run_ours(args):
         step.run()
     torch.cuda.synchronize()
 
-    n_b = len(step.bufs)
+    n_b = step.launches_per_step // 2  # backward launches per step
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
     bwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -300,14 +317,12 @@ def run_ours(args):
 
     ms_total = ev_start.elapsed_time(ev_end)
     bwd_ms = sum(a.elapsed_time(b) for a, b in bwd_ev)
-    t = torch.tensor([ms_total, bwd_ms], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, bwd_ms = float(t[0]), float(t[1])
+    ms_total, bwd_ms = reduce_max([ms_total, bwd_ms], f"cuda:{local}", world)
     ms_step = ms_total / args.steps
-    value = weights * world / (ms_step * 1e-3) / 1e9
+    value = step_throughput(weights, world, ms_step)
 
-    # roofline of the dominant kernel (the backward: 10 of 16 bytes/weight)
+    # roofline of the dominant kernel (the backward: 10 of 16 bytes/weight;
+    # one batched launch covers all matrices of the step)
     peak, peak_kind = measured_peaks()
     bwd_bytes_step = step.bytes_bwd()
     bwd_s_step = bwd_ms * 1e-3 / args.steps
@@ -316,7 +331,7 @@ def run_ours(args):
     traffic = None
     if tr is not None:
         traffic = tr["dram_bytes_per_weight"] * weights / n_b
-    roofline = {"bound": "hbm", "kernel": "pq::bwd_kernel<SEQ2, vec>",
+    roofline = {"bound": "hbm", "kernel": "pq::bwd_units_kernel<SEQ2, vector layout>",
                 "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peak_kind} hbm_gbs (STREAM-style copy)",
@@ -353,17 +368,40 @@ def run_ours(args):
     return 0
 
 
+def bind_to_gpu_numa_node(device_index):
+    """Pin this process to the CPUs next to the GPU (sysfs local_cpulist), so
+    that pinned host buffers are first touched on the GPU's NUMA node."""
+    try:
+        import torch
+        p = torch.cuda.get_device_properties(device_index)
+        bus = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        with open(f"/sys/bus/pci/devices/{bus}/local_cpulist") as f:
+            spec = f.read().strip()
+        cpus = set()
+        for part in spec.split(","):
+            a, _, b = part.partition("-")
+            cpus.update(range(int(a), int(b or a) + 1))
+        if cpus:
+            os.sched_setaffinity(0, cpus)
+            return spec
+    except Exception:
+        return None
+    return None
+
+
 def run_e2e(step, args, local, world):
     """Same metric through the public API from host buffers: every step
-    copies each layer's W and dWq from pinned host memory, runs the forward
-    and backward calls, and copies Wq, dW and d(alpha) back to pinned host
-    memory. Copies in and out run on their own streams and overlap compute
-    across layers."""
+    copies each layer's W and dWq from pinned host memory, runs the batched
+    forward and backward calls for the layer's matrices, and copies Wq, dW
+    and d(alpha) back to pinned host memory. Copies in, compute and copies
+    out run on three streams, so layer l's outputs travel while layer l+1's
+    inputs arrive."""
     import torch
     import torch.distributed as dist
 
     from bit_quantization_aware_b200 import pq
 
+    numa = bind_to_gpu_numa_node(local)
     layers = sorted({b.m.layer for b in step.bufs})
     by_layer = {l: [b for b in step.bufs if b.m.layer == l] for l in layers}
     n_layer = sum(b.m.numel for b in by_layer[layers[0]])
@@ -374,16 +412,21 @@ def run_e2e(step, args, local, world):
     h_wq = torch.empty(n_layer, dtype=torch.bfloat16, **pin)
     h_dw = torch.empty(n_layer, dtype=torch.float32, **pin)
     h_da = torch.empty(rows_layer, dtype=torch.float32, **pin)
-    # start from the device data so that host inputs are realistic
+    # host inputs: the device data of layer 0 (realistic values)
     o = 0
     for b in by_layer[layers[0]]:
         h_w[o:o + b.m.numel].copy_(b.w.reshape(-1))
         h_g[o:o + b.m.numel].copy_(b.g.reshape(-1))
         o += b.m.numel
+    fwd_d = {l: pq.matrix_array([dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha,
+                                      wq=b.wq) for b in by_layer[l]]) for l in layers}
+    bwd_d = {l: pq.matrix_array([dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha,
+                                      g=b.g, dw=b.dw, dalpha=b.dalpha,
+                                      grad_scale=b.grad_scale) for b in by_layer[l]])
+             for l in layers}
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
     def one_step():
-        done_in, done_cmp = {}, {}
         for l in layers:
             with torch.cuda.stream(s_in):
                 o = 0
@@ -391,22 +434,11 @@ def run_e2e(step, args, local, world):
                     b.w.view(-1).copy_(h_w[o:o + b.m.numel], non_blocking=True)
                     b.g.view(-1).copy_(h_g[o:o + b.m.numel], non_blocking=True)
                     o += b.m.numel
-                e = torch.cuda.Event()
-                e.record(s_in)
-                done_in[l] = e
-        for l in layers:
-            s_cmp.wait_event(done_in[l])
-            for b in by_layer[l]:
-                pq.pq_fakequant_fwd(step.q, b.w, b.alpha, b.wq, None, s_cmp)
-            for b in by_layer[l]:
-                pq.pq_fakequant_bwd(step.q, b.w, b.alpha, b.g, b.dw, b.dalpha,
-                                    b.grad_scale, s_cmp)
-            e = torch.cuda.Event()
-            e.record(s_cmp)
-            done_cmp[l] = e
-        with torch.cuda.stream(s_out):
-            for l in layers:
-                s_out.wait_event(done_cmp[l])
+            s_cmp.wait_stream(s_in)
+            pq.pq_fakequant_fwd_batch(step.q, fwd_d[l], s_cmp)
+            pq.pq_fakequant_bwd_batch(step.q, bwd_d[l], s_cmp)
+            s_out.wait_stream(s_cmp)
+            with torch.cuda.stream(s_out):
                 o, ro = 0, 0
                 for b in by_layer[l]:
                     h_wq[o:o + b.m.numel].copy_(b.wq.view(-1), non_blocking=True)
@@ -420,9 +452,9 @@ def run_e2e(step, args, local, world):
     k = max(1, args.e2e_steps)
     if world > 1:
         dist.barrier()
-    t0 = time.perf_counter()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     start.record(s_in)
     for _ in range(k):
         one_step()
@@ -430,19 +462,16 @@ def run_e2e(step, args, local, world):
         s_in.wait_stream(s_out)
     end.record(s_in)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
     wall = (time.perf_counter() - t0) * 1e3
-    t = torch.tensor([max(ms, 0.0)], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t[0])
+    ms = reduce_max([start.elapsed_time(end)], f"cuda:{local}", world)[0]
     ms_step = ms / k
     bi = sum(b.m.numel * 6 for b in step.bufs)
     bo = sum(b.m.numel * 6 + b.m.rows * 4 for b in step.bufs)
-    return {"value": step.weights * world / (ms_step * 1e-3) / 1e9, "unit": UNIT,
+    return {"value": step_throughput(step.weights, world, ms_step), "unit": UNIT,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
             "ms_per_step": ms_step, "steps": k, "wall_ms_per_step": wall / k,
-            "how": "pinned host W, dWq -> device; pq_fakequant_fwd/bwd per matrix; "
+            "pcie_GBs": (bi + bo) / (ms_step * 1e-3) / 1e9, "numa_cpus": numa,
+            "how": "pinned host W, dWq -> device; pq_fakequant_fwd_batch/bwd_batch per layer; "
                    "Wq, dW, dalpha -> pinned host; three streams, layer-pipelined"}
 
 
