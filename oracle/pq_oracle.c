@@ -257,6 +257,42 @@ int pqo_bwd(int q, int64_t rows, int64_t cols, const float* w,
     return 0;
 }
 
+/* Level of an integer code c in alpha units, by the same formulas as the
+ * forward: SEQ (c + shift)/kh, ternary c/1.5, LSQ and binary c. */
+static float pqo_level_of_code(const pqo_params* p, int c) {
+    if (p->is_binary) return (float)c;
+    if (p->shift != 0.0f) {
+        volatile float num = (float)c + p->shift;
+        return num / p->kh;
+    }
+    if (p->kh != 1.0f) return (float)c / p->kh;
+    return (float)c;
+}
+
+/* Dequantize packed codes: read each field (two's complement, `bits` wide,
+ * first column in the lowest bits), sign-extend it to the code c, and
+ * write bf16_rne(fl(level(c) * alpha)). A zero level gives +0.0: the
+ * stored code does not keep the sign of a rounded-to-zero argument.
+ * Needs cols % (8/bits) == 0. Returns 0 on success, -1 on a bad argument. */
+int pqo_dequant(int q, int64_t rows, int64_t cols, const uint8_t* packed,
+                const float* alpha, uint16_t* wq_bf16) {
+    pqo_params p;
+    if (pqo_get_params(q, &p) || rows < 0 || cols < 0) return -1;
+    const int64_t per_byte = 8 / p.bits;
+    const unsigned mask = (1u << p.bits) - 1u;
+    if (cols % per_byte != 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < cols; ++j) {
+            unsigned byte = packed[r * (cols / per_byte) + j / per_byte];
+            unsigned f = (byte >> (p.bits * (int)(j % per_byte))) & mask;
+            int c = (f & (1u << (p.bits - 1))) ? (int)f - (1 << p.bits) : (int)f;
+            volatile float prod = pqo_level_of_code(&p, c) * alpha[r];
+            wq_bf16[r * cols + j] = pqo_bf16_rne(prod);
+        }
+    }
+    return 0;
+}
+
 /* Standalone code export: packed codes only. */
 int pqo_pack(int q, int64_t rows, int64_t cols, const float* w,
              const float* alpha, uint8_t* packed) {

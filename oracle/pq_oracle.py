@@ -65,6 +65,8 @@ class Oracle:
         L.pqo_bwd.restype = ctypes.c_int
         L.pqo_pack.argtypes = [ctypes.c_int, i64, i64, p, p, p]
         L.pqo_pack.restype = ctypes.c_int
+        L.pqo_dequant.argtypes = [ctypes.c_int, i64, i64, p, p, p]
+        L.pqo_dequant.restype = ctypes.c_int
         L.pqo_default_grad_scale.argtypes = [ctypes.c_int, i64]
         L.pqo_default_grad_scale.restype = ctypes.c_float
         L.pqo_code_bits.argtypes = [ctypes.c_int]
@@ -128,6 +130,17 @@ class Oracle:
             raise ValueError(f"oracle pack rejected q={q} shape={w.shape}")
         return out
 
+    def dequant(self, q: int, packed, alpha, cols: int):
+        """bf16 bits [R, cols] from packed codes [R, cols*bits/8]."""
+        packed = np.ascontiguousarray(packed, np.uint8)
+        rows = packed.shape[0]
+        alpha = np.ascontiguousarray(alpha, np.float32).reshape(rows)
+        out = np.empty((rows, cols), np.uint16)
+        rc = self.lib.pqo_dequant(q, rows, cols, _ptr(packed), _ptr(alpha), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle dequant rejected q={q} cols={cols}")
+        return out
+
     def quantize_scalar(self, q: int, w: float, alpha: float,
                         clip_hi: float = 0.0):
         """One element: dict(code, level, wq32, inside, x). ``clip_hi`` > 0
@@ -175,6 +188,10 @@ def pack(q, w, alpha):
 
 def quantize_scalar(q, w, alpha, clip_hi=0.0):
     return default().quantize_scalar(q, w, alpha, clip_hi)
+
+
+def dequant(q, packed, alpha, cols):
+    return default().dequant(q, packed, alpha, cols)
 
 
 def bf16_rne(f):

@@ -384,9 +384,36 @@ def check_pack_roundtrip(O):
         assert np.array_equal(un.astype(np.int8), codes), q
 
 
+def check_dequant_golden(O):
+    """Stored codes decode to the printed levels (golden rows, alpha = 1)."""
+    for row in golden("pack_rows.json")["rows"]:
+        q = NAMES[row["q"]]
+        packed = np.array(row["bytes"], np.uint8).reshape(1, -1)
+        got = (O.dequant(q, packed, np.ones(1, np.float32), len(row["codes"]))
+               .astype(np.uint32) << 16).view(np.float32).ravel()
+        want = [frac_f32(v) if isinstance(v, list) else float(v) for v in row["levels"]]
+        want = torch.tensor(want, dtype=torch.float32).to(torch.bfloat16).float().numpy()
+        assert np.array_equal(np.abs(got), np.abs(want)) and np.array_equal(got, want), (row["q"], got)
+
+
+def check_dequant_inverts_pack(O):
+    """Decoding the packed codes reproduces the forward's bf16 weights, up
+    to the sign of a zero (codes do not store it)."""
+    rng = np.random.default_rng(29)
+    for q in ALL_QUANTIZERS:
+        w = rng.normal(0, 0.02, (6, 64)).astype(np.float32)
+        alpha = (np.abs(w).max(axis=1) * rng.uniform(0.3, 1.0, 6)).astype(np.float32)
+        wq, _, packed = O.fwd(q, w, alpha, pack=True)
+        dq = O.dequant(q, packed, alpha, 64)
+        zero = (wq & 0x7FFF) == 0
+        assert np.array_equal(dq[~zero], wq[~zero]), q
+        assert np.all(dq[zero] == 0), q
+
+
 ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_nearest_level, check_binary_sign, check_lsq_textbook,
               check_overflow_example, check_ties_half_even, check_idempotence,
               check_bf16_rne, check_ste, check_dalpha_fd,
               check_dalpha_all_clipped, check_grad_scale, check_pack_golden,
-              check_pack_roundtrip]
+              check_pack_roundtrip, check_dequant_golden,
+              check_dequant_inverts_pack]

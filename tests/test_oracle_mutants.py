@@ -51,6 +51,12 @@ MUTANTS = {
     "zero_sign_dropped": ("c = (int)r;\n    }", "c = (int)r;\n        lev = (lev == 0.0f) ? 0.0f : lev;\n    }"),
     "grad_scale_missing": ("dalpha[r] = (float)(acc * (double)grad_scale);",
                            "dalpha[r] = (float)(acc);"),
+    "dequant_no_sign_extend": ("int c = (f & (1u << (p.bits - 1))) ? (int)f - (1 << p.bits) : (int)f;",
+                               "int c = (int)f;"),
+    "dequant_field_order": ("unsigned f = (byte >> (p.bits * (int)(j % per_byte))) & mask;",
+                            "unsigned f = (byte >> (p.bits * (int)(per_byte - 1 - j % per_byte))) & mask;"),
+    "dequant_no_alpha": ("volatile float prod = pqo_level_of_code(&p, c) * alpha[r];",
+                         "volatile float prod = pqo_level_of_code(&p, c);"),
 }
 
 
