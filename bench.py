@@ -39,6 +39,9 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--op", choices=["quantizer", "dequant"], default="quantizer",
+                   help="quantizer: the forward+backward step (the headline); "
+                        "dequant: packed codes -> bf16 over the same layer set")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -475,10 +478,67 @@ def run_e2e(step, args, local, world):
                    "Wq, dW, dalpha -> pinned host; three streams, layer-pipelined"}
 
 
+def run_dequant(args):
+    """Packed 2-bit codes + alpha -> bf16 weights for every matrix of the
+    Llama-3-8B-shaped set (the export path's consumer), one batched call,
+    1 GPU. Prints one JSON line with its own roofline (2.25 B/weight)."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.step import QuantStep
+
+    torch.cuda.set_device(0)
+    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device="cuda:0", pack=True)
+    step.generate(seed=3)
+    step.fwd_all()
+    torch.cuda.synchronize()
+    out = torch.empty_like(step.wq_all)
+    descs, o = [], 0
+    for b in step.bufs:
+        n = b.m.numel
+        descs.append(dict(rows=b.m.rows, cols=b.m.cols, alpha=b.alpha, packed=b.packed,
+                          wq=out[o:o + n]))
+        o += (n + 63) // 64 * 64
+    mats = pq.matrix_array(descs)
+
+    def go():
+        pq.pq_dequant_codes_batch(step.q, mats)
+
+    for _ in range(max(args.warmup, 1)):
+        go()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        go()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    bytes_step = sum(b.m.numel * 2 + b.m.numel // 4 + b.m.rows * 4 for b in step.bufs)
+    peak, kind = measured_peaks()
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "packed-code dequantization Gweights/s", "op": "dequant",
+        "value": step.weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "u8->bf16", "data": "synthetic",
+        "config": {"workload": "llama3_8b_linear_set_seq2_dequant",
+                   "weights": step.weights, "launches_per_step": 1},
+        "roofline": {"bound": "hbm", "kernel": "pq::dequant_units_kernel<SEQ2, vector layout>",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{kind} hbm_gbs",
+                     "algorithmic_bytes_per_step": bytes_step}}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "dequant":
+        return run_dequant(args)
     return run_ours(args)
 
 

@@ -306,7 +306,7 @@ fwd_units_kernel(const __grid_constant__ Batch p) {
         const float* wr = m.w + row * m.cols;
         uint16_t* qr = WQ ? m.wq + row * m.cols : nullptr;
         uint8_t* pr = PACK ? m.packed + row * (m.cols * Traits<Q>::bits / 8) : nullptr;
-        constexpr int U = PQ_FWD_UNROLL;
+        constexpr int U = VEC ? PQ_FWD_UNROLL : 2;  // element path: fewer registers
         for (int64_t ch = c_begin + lane; ch < c_end; ch += U * tpr) {
             float v[U][8];
 #pragma unroll
@@ -426,6 +426,118 @@ scaled_weights_kernel(const float* __restrict__ w, const float* __restrict__ alp
     }
 }
 
+// ----------------------------------------------------------- dequantize
+// Packed codes -> bf16(fl(level * alpha)), over a batch of matrices in the
+// same (matrix, row block) units as the forward. In a batch descriptor,
+// `packed` is the input (codes a forward wrote) and `wq` the output.
+//
+// Vector layout (cols % 8 == 0, aligned): lane l of a row group decodes
+// chunks of 8 codes l, l + TPR, ..., four loads in flight, so each warp
+// store writes 512 contiguous bytes. 2-bit codes: the row's four possible
+// outputs form a table held byte-planar in two registers (lo = low bytes of
+// entries 0..3, hi = high bytes), so one byte permute (PRMT) decodes two
+// weights; its selectors come from spreading a byte's four 2-bit fields to
+// byte positions with two overlap-free multiplies (even fields by 1 + 2^12,
+// odd ones by 2^6 + 2^18). 4-bit codes and the element path decode each
+// field arithmetically.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    return __byte_perm(a, b, sel);
+}
+
+// Fields of byte b (4 codes of 2 bits) moved to bits 0, 8, 16, 24.
+__device__ __forceinline__ uint32_t spread2(uint32_t b) {
+    return ((b & 0x33u) * 0x1001u | (b & 0xCCu) * 0x40040u) & 0x03030303u;
+}
+
+template <int Q, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+dequant_units_kernel(const __grid_constant__ Batch p) {
+    constexpr int B = Traits<Q>::bits;
+    constexpr uint32_t mask = (1u << B) - 1u;
+    int mi = 0;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+        mi = find_matrix(p, mi, u);
+        const MatDesc& m = p.m[mi];
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rpb = kThreads >> tl;
+        const int64_t row = (u - m.unit_begin) * rpb + (threadIdx.x >> tl);
+        if (row >= m.rows) continue;
+        const float a = __ldg(m.alpha + row);
+        const uint8_t* src = m.packed + row * (m.cols * B / 8);
+        uint16_t* dst = m.wq + row * m.cols;
+        if constexpr (VEC) {
+            // lane l decodes chunks l, l + tpr, ... of 8 codes: each warp
+            // store writes 512 contiguous bytes
+            uint32_t lo = 0, hi = 0;
+            if constexpr (B == 2) {  // table of the 4 outputs, byte-planar
+                const uint32_t e01 = pack_bf16x2(__fmul_rn(level_of_field<Q>(0), a),
+                                                 __fmul_rn(level_of_field<Q>(1), a));
+                const uint32_t e23 = pack_bf16x2(__fmul_rn(level_of_field<Q>(2), a),
+                                                 __fmul_rn(level_of_field<Q>(3), a));
+                lo = prmt(e01, e23, 0x6420);
+                hi = prmt(e01, e23, 0x7531);
+            }
+            constexpr int U = 4;
+            const int64_t nch = m.cols >> 3;
+            for (int64_t ch = lane; ch < nch; ch += U * tpr) {
+                uint32_t pk[U];
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t c = ch + k * tpr;
+                    if (c < nch) {
+                        if constexpr (B == 2)
+                            pk[k] = ld_stream(reinterpret_cast<const unsigned short*>(src + c * 2));
+                        else
+                            pk[k] = ld_stream(reinterpret_cast<const unsigned int*>(src + c * 4));
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t c = ch + k * tpr;
+                    if (c < nch) {
+                        uint32_t o[4];
+                        if constexpr (B == 2) {
+                            const uint32_t t0 = spread2(pk[k] & 0xFFu);
+                            const uint32_t t1 = spread2(pk[k] >> 8);
+                            o[0] = prmt(lo, hi, t0 * 0x11u + 0x4040u);
+                            o[1] = prmt(lo, hi, (t0 >> 16) * 0x11u + 0x4040u);
+                            o[2] = prmt(lo, hi, t1 * 0x11u + 0x4040u);
+                            o[3] = prmt(lo, hi, (t1 >> 16) * 0x11u + 0x4040u);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                o[j] = pack_bf16x2(
+                                    __fmul_rn(level_of_field<Q>((pk[k] >> (8 * j)) & mask), a),
+                                    __fmul_rn(level_of_field<Q>((pk[k] >> (8 * j + 4)) & mask), a));
+                        }
+                        st_stream(reinterpret_cast<uint4*>(dst + c * 8),
+                                  make_uint4(o[0], o[1], o[2], o[3]));
+                    }
+                }
+            }
+        } else {  // element path: groups of 8 codes
+            const int64_t nch = (m.cols + 7) >> 3;
+            for (int64_t ch = lane; ch < nch; ch += tpr) {
+                const int n = tail_n(m.cols, ch);
+                uint32_t pk = 0;
+#pragma unroll
+                for (int k = 0; k < B; ++k)  // B bytes hold 8 codes
+                    if (k * (8 / B) < n) pk |= static_cast<uint32_t>(src[ch * B + k]) << (8 * k);
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const uint32_t hw = pack_bf16x2(
+                        __fmul_rn(level_of_field<Q>((pk >> (B * i)) & mask), a),
+                        __fmul_rn(level_of_field<Q>((pk >> (B * (i + 1))) & mask), a));
+                    if (i < n) dst[ch * 8 + i] = static_cast<uint16_t>(hw);
+                    if (i + 1 < n) dst[ch * 8 + i + 1] = static_cast<uint16_t>(hw >> 16);
+                }
+            }
+        }
+    }
+}
+
 // --------------------------------------------------------------- host side
 static thread_local int g_last_cuda_error = 0;
 
@@ -524,6 +636,15 @@ template <int Q, bool VEC>
 static void launch_bwd(const Batch& b, cudaStream_t s) {
     static int cache[64] = {0};
     auto k = bwd_units_kernel<Q, VEC>;
+    const int64_t ctas = persistent_ctas(k, cache);
+    const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
+    k<<<grid, kThreads, 0, s>>>(b);
+}
+
+template <int Q, bool VEC>
+static void launch_dequant(const Batch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    auto k = dequant_units_kernel<Q, VEC>;
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
@@ -684,6 +805,44 @@ static pq_status_t bwd_batch_impl(int q, int32_t n, const pq_matrix_t* mats, cud
     return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
 }
 
+// Dequantization over n matrices (packed_out is read, wq_bf16_out written).
+static pq_status_t dequant_batch_impl(int q, int32_t n, const pq_matrix_t* mats, cudaStream_t s) {
+    const int bits = code_bits_of(q);
+    if (bits == 0 || n < 0 || (n > 0 && !mats)) return PQ_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        const pq_matrix_t& m = mats[i];
+        if (m.rows < 0 || m.cols < 0 || m.cols % (8 / bits) != 0) return PQ_ERR_INVALID_ARG;
+        if (m.rows > 0 && m.cols > 0 && (!m.packed_out || !m.alpha || !m.wq_bf16_out))
+            return PQ_ERR_INVALID_ARG;
+    }
+    static thread_local Batch b;
+    bool launched = false;
+    for (int cls = 0; cls < 2; ++cls) {
+        const bool vec = cls == 0;
+        batch_reset(b);
+        auto flush = [&]() {
+            if (b.n == 0) return;
+            launched = true;
+            dispatch_q(q, [&]<int Q>() {
+                if (vec) launch_dequant<Q, true>(b, s);
+                else launch_dequant<Q, false>(b, s);
+            });
+            batch_reset(b);
+        };
+        for (int32_t i = 0; i < n; ++i) {
+            const pq_matrix_t& m = mats[i];
+            if (m.rows == 0 || m.cols == 0) continue;
+            const bool v = m.cols % 8 == 0 && aligned(m.packed_out, bits == 2 ? 2 : 4) &&
+                           aligned(m.wq_bf16_out, 16);
+            if (v != vec) continue;
+            if (b.n == kMaxBatch) flush();
+            batch_add(b, m, choose_tpr_log2(m.cols), 1);
+        }
+        flush();
+    }
+    return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
+}
+
 }  // namespace pq
 
 using namespace pq;
@@ -743,6 +902,22 @@ pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w, const 
     scaled_weights_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kThreads,
                             0, static_cast<cudaStream_t>(stream)>>>(w, alpha, x_out, rows, cols);
     return cuda_status(cudaGetLastError());
+}
+
+pq_status_t pq_dequant_codes(pq_quant_t q, int64_t rows, int64_t cols, const uint8_t* packed,
+                             const float* alpha, uint16_t* wq_bf16_out, void* stream) {
+    pq_matrix_t m = {};
+    m.rows = rows;
+    m.cols = cols;
+    m.alpha = alpha;
+    m.packed_out = const_cast<uint8_t*>(packed);
+    m.wq_bf16_out = wq_bf16_out;
+    return dequant_batch_impl(q, 1, &m, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_dequant_codes_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,
+                                   void* stream) {
+    return dequant_batch_impl(q, n, mats, static_cast<cudaStream_t>(stream));
 }
 
 pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,

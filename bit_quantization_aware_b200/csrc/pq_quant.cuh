@@ -173,6 +173,26 @@ __device__ __forceinline__ Elem quantize_x(float x) {
     return e;
 }
 
+// Level (alpha units) of a stored code field f: sign-extend it to the code
+// c, turn c into a float without the conversion unit (the add/subtract
+// constant in reverse: the encoding of 1.5*2^23 + c, minus 1.5*2^23), and
+// apply the forward's level formula. A zero level is +0.0.
+template <int Q>
+__device__ __forceinline__ float level_of_field(uint32_t f) {
+    constexpr int B = Traits<Q>::bits;
+    const int c = static_cast<int>(f << (32 - B)) >> (32 - B);
+    const float cf = __fsub_rn(__int_as_float(0x4B400000 + c), kRoundShift);
+    if constexpr (Q == PQ_SEQ2) {
+        return __fmaf_rn(cf, 0.5f, 0.25f);
+    } else if constexpr (Q == PQ_SEQ2_B) {
+        return __fmaf_rn(cf, kTwoThirds, 0.5f * kTwoThirds);
+    } else if constexpr (Q == PQ_TERNARY) {
+        return __fmul_rn(cf, kTwoThirds);
+    } else {  // LSQ grid and binary: the code is the level
+        return cf;
+    }
+}
+
 // Two's-complement code field of width Traits<Q>::bits.
 template <int Q>
 __device__ __forceinline__ uint32_t code_field(const Elem& e) {

@@ -56,6 +56,10 @@ def _declare(L):
     L.pq_fakequant_fwd_batch.restype = i32
     L.pq_fakequant_bwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_fakequant_bwd_batch.restype = i32
+    L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
+    L.pq_dequant_codes_batch.restype = i32
+    L.pq_dequant_codes.argtypes = [i32, i64, i64, p, p, p, p]
+    L.pq_dequant_codes.restype = i32
     L.pq_scaled_weights.argtypes = [i64, i64, p, p, p, p]
     L.pq_scaled_weights.restype = i32
     L.pq_fakequant_fwd.argtypes = [i32, i64, i64, p, p, p, p, p]
@@ -146,6 +150,21 @@ def pq_pack_codes(q, w, alpha, packed_out, stream=None, rows=None, cols=None):
     _check("pq_pack_codes", lib().pq_pack_codes(
         q, rows, cols, _ptr(w), _ptr(alpha), _ptr(packed_out),
         _stream(stream)))
+
+
+def pq_dequant_codes(q, packed, alpha, wq_out, stream=None, rows=None, cols=None):
+    """bf16 weights [rows, cols] from packed codes [rows, cols*bits/8]."""
+    if rows is None or cols is None:
+        rows, cols = wq_out.shape
+    _check("pq_dequant_codes", lib().pq_dequant_codes(
+        q, int(rows), int(cols), _ptr(packed), _ptr(alpha), _ptr(wq_out),
+        _stream(stream)))
+
+
+def pq_dequant_codes_batch(q, mats, stream=None):
+    """Dequantization over a ``pq_matrix_t[]`` (packed read, wq written)."""
+    _check("pq_dequant_codes_batch", lib().pq_dequant_codes_batch(
+        q, len(mats), mats, _stream(stream)))
 
 
 def pq_scaled_weights(w, alpha, x_out, stream=None, rows=None, cols=None):

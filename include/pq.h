@@ -177,6 +177,30 @@ PQ_API pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n,
 PQ_API pq_status_t pq_fakequant_bwd_batch(pq_quant_t q, int32_t n,
                                           const pq_matrix_t* mats, void* stream);
 
+/* Dequantize packed codes back to bf16 weights: each stored code c (layout
+ * of packed_out above) becomes bf16_rn(fl(level(c) * alpha_row)) with the
+ * forward's level formulas, so the result equals the forward's
+ * wq_bf16_out except that a zero level is +0.0 (the code does not keep the
+ * sign of a rounded-to-zero weight). This is the consumer of exported
+ * low-bit weights [P4: 2-bit kernels read packed weights; P1 "Paper vs.
+ * code": the training code has no packed path].
+ *   packed       uint8 [rows * cols * bits / 8], cols % (8/bits) == 0
+ *   alpha        fp32 [rows]
+ *   wq_bf16_out  bf16 bit patterns [rows*cols], overwritten
+ * Fast path: cols % 8 == 0, packed aligned to 2 (2-bit) or 4 (4-bit)
+ * bytes, wq_bf16_out to 16 bytes; any other layout takes an element path
+ * with the same results. Traffic: bits/8 B read + 2 B written per weight. */
+PQ_API pq_status_t pq_dequant_codes(pq_quant_t q, int64_t rows, int64_t cols,
+                                    const uint8_t* packed, const float* alpha,
+                                    uint16_t* wq_bf16_out, void* stream);
+
+/* Dequantization over n matrices in as few launches as possible: for each
+ * descriptor, packed_out is READ (the codes a forward wrote), alpha read,
+ * wq_bf16_out written; other fields are ignored. Equivalent to n calls of
+ * pq_dequant_codes on the same stream. */
+PQ_API pq_status_t pq_dequant_codes_batch(pq_quant_t q, int32_t n,
+                                          const pq_matrix_t* mats, void* stream);
+
 /* Scaled weights x = fl(w / alpha_row): the first step of every quantizer,
  * computed by the same device routine as the forward and backward kernels
  * (the correctly rounded fp32 quotient; [P1 "Paper vs. code": the

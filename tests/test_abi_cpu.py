@@ -30,7 +30,7 @@ def test_header_declares_entry_points():
     names = declared()
     for n in ("pq_fakequant_fwd", "pq_fakequant_bwd", "pq_pack_codes",
               "pq_fakequant_fwd_batch", "pq_fakequant_bwd_batch",
-              "pq_scaled_weights",
+              "pq_scaled_weights", "pq_dequant_codes", "pq_dequant_codes_batch",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
               "pq_last_cuda_error"):
         assert n in names
@@ -90,6 +90,13 @@ def test_argument_errors_launch_nothing(L):
     assert f(pq.PQ_SEQ2, 4, 0, None, None, fake, None, None) == pq.PQ_OK
     assert k(pq.PQ_LSQ3, 0, 0, None, None, fake, None) == pq.PQ_OK
     assert b(pq.PQ_SEQ2, 0, 8, None, None, None, None, None, 1.0, None) == pq.PQ_OK
+    dq = L.pq_dequant_codes
+    assert dq(99, 4, 8, fake, fake, fake, None) == E
+    assert dq(pq.PQ_SEQ2, 4, 6, fake, fake, fake, None) == E      # cols % 4
+    assert dq(pq.PQ_LSQ4, 4, 7, fake, fake, fake, None) == E      # cols % 2
+    assert dq(pq.PQ_SEQ2, 4, 8, None, fake, fake, None) == E
+    assert dq(pq.PQ_SEQ2, 4, 8, fake, fake, None, None) == E
+    assert dq(pq.PQ_SEQ2, 0, 8, None, None, None, None) == pq.PQ_OK
     sw = L.pq_scaled_weights
     assert sw(-1, 8, fake, fake, fake, None) == E
     assert sw(4, 8, None, fake, fake, None) == E

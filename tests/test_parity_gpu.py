@@ -427,3 +427,73 @@ def test_weights_on_code_and_clip_boundaries(q):
     check_fwd(q, wn, an, wq, pk)
     check_fwd(q, wn, an, None, pk2)
     check_bwd(q, wn, an, gn, gs, dw, da)
+
+
+def _dequant_gpu(q, packed_np, alpha_np, cols, offset=0):
+    rows = packed_np.shape[0]
+    nb = packed_np.size
+    pbuf = torch.zeros(nb + offset + 16, dtype=torch.uint8, device=DEV)
+    pk = pbuf[offset:offset + nb]
+    pk.copy_(torch.from_numpy(packed_np.ravel()))
+    qbuf = torch.empty(rows * cols + offset + 8, dtype=torch.bfloat16, device=DEV)
+    out = qbuf[offset:offset + rows * cols].view(rows, cols)
+    pq.pq_dequant_codes(q, pk, torch.from_numpy(alpha_np).to(DEV), out, rows=rows, cols=cols)
+    torch.cuda.synchronize()
+    return bits16(out)
+
+
+@pytest.mark.parametrize("q", ALLQ)
+@pytest.mark.parametrize("shape,offset", [((1, 32), 0), ((3, 96), 0), ((5, 12), 0),
+                                          ((7, 1000), 0), ((33, 1032), 0), ((64, 4096), 0),
+                                          ((9, 4096), 1), ((2, 70000), 0)])
+def test_dequant_matches_oracle(q, shape, offset):
+    """Packed codes -> bf16: every element equals the oracle's decoding
+    (random bytes, so every code value of the format appears)."""
+    rows, cols = shape
+    bits = pq.pq_code_bits(q)
+    if cols % (8 // bits):
+        pytest.skip("shape not packable")
+    rng = np.random.default_rng(rows * 7 + cols)
+    packed = rng.integers(0, 256, (rows, cols * bits // 8), dtype=np.uint8)
+    alpha = np.exp(rng.uniform(-6, 1, rows)).astype(np.float32)
+    got = _dequant_gpu(q, packed, alpha, cols, offset)
+    want = pq_oracle.dequant(q, packed, alpha, cols)
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, f"{len(bad)} mismatches, first {bad[0].tolist()}"
+
+
+@pytest.mark.parametrize("q", ALLQ)
+def test_dequant_inverts_forward_codes(q):
+    """On 2048x8192: decoding the forward's packed codes gives the forward's
+    bf16 weights, except that zero levels decode to +0."""
+    w = I.normal_weights(2048, 8192, seed=11, stream=0, device=DEV)
+    a = I.alpha_init(w, q)
+    wq, pk = pq.fakequant_fwd(q, w, a, pack=True)
+    out = torch.empty_like(wq)
+    pq.pq_dequant_codes(q, pk, a, out)
+    torch.cuda.synchronize()
+    zero = (wq.view(torch.int16) & 0x7FFF) == 0
+    assert torch.equal(out.view(torch.int16)[~zero], wq.view(torch.int16)[~zero])
+    assert torch.all(out.view(torch.int16)[zero] == 0)
+
+
+def test_dequant_batch_equals_single_calls():
+    """A batch of mixed shapes and alignments decodes like single calls."""
+    q = pq.PQ_SEQ2
+    rng = np.random.default_rng(41)
+    shapes = [(64, 4096), (3, 96), (5, 12), (33, 1032), (0, 8), (7, 1000)]
+    descs, singles = [], []
+    for rows, cols in shapes:
+        packed = torch.from_numpy(rng.integers(0, 256, (rows, cols // 4), dtype=np.uint8)).to(DEV)
+        alpha = torch.from_numpy(np.exp(rng.uniform(-5, 0, rows)).astype(np.float32)).to(DEV)
+        o1 = torch.empty((rows, cols), dtype=torch.bfloat16, device=DEV)
+        o2 = torch.empty((rows, cols), dtype=torch.bfloat16, device=DEV)
+        descs.append(dict(rows=rows, cols=cols, packed=packed if rows else None,
+                          alpha=alpha if rows else None, wq=o1 if rows else None))
+        if rows:
+            pq.pq_dequant_codes(q, packed, alpha, o2)
+        singles.append((o1, o2))
+    pq.pq_dequant_codes_batch(q, pq.matrix_array(descs))
+    torch.cuda.synchronize()
+    for o1, o2 in singles:
+        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
