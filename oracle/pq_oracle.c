@@ -293,6 +293,105 @@ int pqo_dequant(int q, int64_t rows, int64_t cols, const uint8_t* packed,
     return 0;
 }
 
+/* One AdamW step (decoupled weight decay) on one fp32 parameter, in this
+ * fixed fp32 order, each step rounded on its own:
+ *   p  = (wd != 0) ? p * decay : p
+ *   m  = b1*m + c1*g
+ *   v  = b2*v + c2*(g*g)
+ *   den = sqrt(v) * inv_sbc2 + eps
+ *   p  = p - step * (m / den)
+ * with the scalar factors formed once in double from the hyperparameters
+ * and rounded to fp32: decay = 1 - lr*wd, b1 = beta1, c1 = 1 - beta1,
+ * b2 = beta2, c2 = 1 - beta2, inv_sbc2 = 1/sqrt(1 - beta2^t),
+ * step = lr/(1 - beta1^t), eps. */
+typedef struct {
+    double lr, beta1, beta2, eps, weight_decay;
+    int64_t step;  /* t >= 1 */
+} pqo_adamw;
+
+typedef struct {
+    float decay, b1, c1, b2, c2, inv_sbc2, step, eps;
+    int has_decay;
+} pqo_adamw_k;
+
+static pqo_adamw_k pqo_adamw_consts(const pqo_adamw* h) {
+    pqo_adamw_k k;
+    const double t = (double)h->step;
+    k.decay = (float)(1.0 - h->lr * h->weight_decay);
+    k.has_decay = h->weight_decay != 0.0;
+    k.b1 = (float)h->beta1;
+    k.c1 = (float)(1.0 - h->beta1);
+    k.b2 = (float)h->beta2;
+    k.c2 = (float)(1.0 - h->beta2);
+    k.inv_sbc2 = (float)(1.0 / sqrt(1.0 - pow(h->beta2, t)));
+    k.step = (float)(h->lr / (1.0 - pow(h->beta1, t)));
+    k.eps = (float)h->eps;
+    return k;
+}
+
+static float pqo_adamw_update(const pqo_adamw_k* k, float p, float g, float* m, float* v) {
+    if (k->has_decay) {
+        volatile float pd = p * k->decay;
+        p = pd;
+    }
+    volatile float a1 = k->b1 * *m;
+    volatile float a2 = k->c1 * g;
+    *m = a1 + a2;
+    volatile float gg = g * g;
+    volatile float b1 = k->b2 * *v;
+    volatile float b2 = k->c2 * gg;
+    *v = b1 + b2;
+    volatile float sq = sqrtf(*v);
+    volatile float sc = sq * k->inv_sbc2;
+    volatile float den = sc + k->eps;
+    volatile float ratio = *m / den;
+    volatile float upd = k->step * ratio;
+    return p - upd;
+}
+
+/* Backward fused with AdamW: computes dW and d(alpha) from the current w
+ * and alpha exactly as pqo_bwd, then applies one AdamW step to every
+ * weight (gradient dW, states m_w, v_w) and to every row's alpha
+ * (gradient: the fp32 d(alpha), states m_a, v_a). w, alpha and the four
+ * state arrays are updated in place; dalpha (nullable) receives the fp32
+ * d(alpha). hw and ha are the hyperparameters of weights and scales. */
+int pqo_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alpha,
+                  const uint16_t* g_bf16, float* m_w, float* v_w, float* m_a,
+                  float* v_a, float grad_scale, const pqo_adamw* hw,
+                  const pqo_adamw* ha, float* dalpha) {
+    pqo_params p;
+    if (pqo_get_params(q, &p) || rows < 0 || cols < 0 || !hw || !ha) return -1;
+    const pqo_adamw_k kw = pqo_adamw_consts(hw), ka = pqo_adamw_consts(ha);
+    for (int64_t r = 0; r < rows; ++r) {
+        float da;
+        if (pqo_bwd(q, 1, cols, w + r * cols, alpha + r, g_bf16 + r * cols, NULL, &da,
+                    grad_scale, NULL))
+            return -1;
+        for (int64_t j = 0; j < cols; ++j) {
+            int inside;
+            pqo_quantize_scalar(q, w[r * cols + j], alpha[r], 0.0f, NULL, NULL, NULL,
+                                &inside, NULL);
+            float g = pqo_bf16_to_float(g_bf16[r * cols + j]);
+            float dw = inside ? g : 0.0f;
+            w[r * cols + j] = pqo_adamw_update(&kw, w[r * cols + j], dw,
+                                               &m_w[r * cols + j], &v_w[r * cols + j]);
+        }
+        alpha[r] = pqo_adamw_update(&ka, alpha[r], da, &m_a[r], &v_a[r]);
+        if (dalpha) dalpha[r] = da;
+    }
+    return 0;
+}
+
+/* One AdamW step over n parameters with given gradients (for pinning the
+ * update rule against a library optimizer). */
+int pqo_adamw_step(int64_t n, float* p, const float* g, float* m, float* v,
+                   const pqo_adamw* h) {
+    if (n < 0 || !h) return -1;
+    const pqo_adamw_k k = pqo_adamw_consts(h);
+    for (int64_t i = 0; i < n; ++i) p[i] = pqo_adamw_update(&k, p[i], g[i], &m[i], &v[i]);
+    return 0;
+}
+
 /* Standalone code export: packed codes only. */
 int pqo_pack(int q, int64_t rows, int64_t cols, const float* w,
              const float* alpha, uint8_t* packed) {

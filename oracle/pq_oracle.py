@@ -52,6 +52,17 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+class AdamW(ctypes.Structure):
+    """Hyperparameters of one AdamW step (t >= 1 is the step count)."""
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
+                ("weight_decay", ctypes.c_double), ("step", ctypes.c_int64)]
+
+    @classmethod
+    def at_step(cls, t, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+        return cls(lr, beta1, beta2, eps, weight_decay, t)
+
+
 class Oracle:
     """One loaded copy of the oracle library."""
 
@@ -67,6 +78,12 @@ class Oracle:
         L.pqo_pack.restype = ctypes.c_int
         L.pqo_dequant.argtypes = [ctypes.c_int, i64, i64, p, p, p]
         L.pqo_dequant.restype = ctypes.c_int
+        L.pqo_bwd_adamw.argtypes = [ctypes.c_int, i64, i64, p, p, p, p, p, p, p,
+                                    ctypes.c_float, ctypes.POINTER(AdamW),
+                                    ctypes.POINTER(AdamW), p]
+        L.pqo_bwd_adamw.restype = ctypes.c_int
+        L.pqo_adamw_step.argtypes = [i64, p, p, p, p, ctypes.POINTER(AdamW)]
+        L.pqo_adamw_step.restype = ctypes.c_int
         L.pqo_default_grad_scale.argtypes = [ctypes.c_int, i64]
         L.pqo_default_grad_scale.restype = ctypes.c_float
         L.pqo_code_bits.argtypes = [ctypes.c_int]
@@ -140,6 +157,39 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle dequant rejected q={q} cols={cols}")
         return out
+
+    def bwd_adamw(self, q, w, alpha, g_bf16, m_w, v_w, m_a, v_a, grad_scale,
+                  hw, ha):
+        """Fused backward + AdamW on copies; returns (w, alpha, m_w, v_w, m_a,
+        v_a, dalpha), all fp32."""
+        w = np.array(w, np.float32, order="C", copy=True)
+        rows, cols = w.shape
+        alpha = np.array(alpha, np.float32, copy=True).reshape(rows)
+        g = np.ascontiguousarray(g_bf16).view(np.uint16)
+        m_w = np.array(m_w, np.float32, order="C", copy=True)
+        v_w = np.array(v_w, np.float32, order="C", copy=True)
+        m_a = np.array(m_a, np.float32, copy=True).reshape(rows)
+        v_a = np.array(v_a, np.float32, copy=True).reshape(rows)
+        da = np.empty(rows, np.float32)
+        rc = self.lib.pqo_bwd_adamw(q, rows, cols, _ptr(w), _ptr(alpha), _ptr(g),
+                                    _ptr(m_w), _ptr(v_w), _ptr(m_a), _ptr(v_a),
+                                    ctypes.c_float(grad_scale), ctypes.byref(hw),
+                                    ctypes.byref(ha), _ptr(da))
+        if rc != 0:
+            raise ValueError("oracle bwd_adamw rejected its arguments")
+        return w, alpha, m_w, v_w, m_a, v_a, da
+
+    def adamw_step(self, p, g, m, v, h):
+        """One AdamW step on copies of fp32 arrays; returns (p, m, v)."""
+        p = np.array(p, np.float32, copy=True).ravel()
+        g = np.ascontiguousarray(g, np.float32).ravel()
+        m = np.array(m, np.float32, copy=True).ravel()
+        v = np.array(v, np.float32, copy=True).ravel()
+        rc = self.lib.pqo_adamw_step(len(p), _ptr(p), _ptr(g), _ptr(m), _ptr(v),
+                                     ctypes.byref(h))
+        if rc != 0:
+            raise ValueError("oracle adamw rejected its arguments")
+        return p, m, v
 
     def quantize_scalar(self, q: int, w: float, alpha: float,
                         clip_hi: float = 0.0):

@@ -410,10 +410,73 @@ def check_dequant_inverts_pack(O):
         assert np.all(dq[zero] == 0), q
 
 
+def check_adamw_vs_torch(O):
+    """One AdamW step matches torch.optim.AdamW (fp32, CPU) over five steps,
+    with and without decoupled weight decay, to within fp32 rounding."""
+    from oracle.pq_oracle import AdamW
+    rng = np.random.default_rng(43)
+    for wd in (0.0, 0.05):
+        p0 = rng.normal(0, 0.02, 4096).astype(np.float32)
+        t_p = torch.nn.Parameter(torch.from_numpy(p0.copy()))
+        opt = torch.optim.AdamW([t_p], lr=2e-3, betas=(0.9, 0.999), eps=1e-8,
+                                weight_decay=wd, foreach=False, fused=False)
+        p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+        for t in range(1, 6):
+            g = rng.normal(0, 1e-3, 4096).astype(np.float32)
+            t_p.grad = torch.from_numpy(g.copy())
+            opt.step()
+            prev = p
+            p, m, v = O.adamw_step(p, g, m, v, AdamW.at_step(t, 2e-3, weight_decay=wd))
+            st = opt.state[t_p]
+            # tolerances against the scale of the quantity (torch forms the
+            # first moment as a lerp: same value up to a few ulps)
+            gs = float(np.abs(g).max())
+            assert np.allclose(m, st["exp_avg"].numpy(), rtol=1e-5, atol=1e-6 * gs), (wd, t)
+            assert np.allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-5, atol=1e-6 * gs * gs), (wd, t)
+            upd, t_upd = p - prev, t_p.detach().numpy() - prev
+            assert np.allclose(upd, t_upd, rtol=1e-4, atol=1e-5 * 2e-3), (wd, t)
+            p = t_p.detach().numpy().copy()  # stay on torch's trajectory
+
+
+def check_adamw_first_step(O):
+    """Closed form of Adam's first step from zero moments: the bias-corrected
+    moments are g and g^2, so the update is lr * g / (|g| + eps)."""
+    from oracle.pq_oracle import AdamW
+    g = np.array([1e-3, -2e-2, 5e-1, -7.0, 1e-6], np.float32)
+    p0 = np.zeros_like(g)
+    p, m, v = O.adamw_step(p0, g, np.zeros_like(g), np.zeros_like(g),
+                           AdamW.at_step(1, 1e-2))
+    want = -1e-2 * g.astype(np.float64) / (np.abs(g.astype(np.float64)) + 1e-8)
+    assert np.allclose(p, want, rtol=1e-5), (p, want)
+    assert np.allclose(m, 0.1 * g, rtol=1e-6) and np.allclose(v, 0.001 * g * g, rtol=1e-5)
+
+
+def check_bwd_adamw_composes(O):
+    """The fused backward + AdamW equals the backward followed by AdamW
+    steps on W (gradient dW) and alpha (gradient d(alpha)), bit for bit."""
+    from oracle.pq_oracle import AdamW
+    rng = np.random.default_rng(47)
+    for q in ALL_QUANTIZERS:
+        w = rng.normal(0, 0.02, (5, 48)).astype(np.float32)
+        a = (np.abs(w).max(axis=1) * 0.8).astype(np.float32)
+        gb = torch.randn(5, 48).mul(1e-3).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        mw, vw = rng.normal(0, 1e-4, (5, 48)).astype(np.float32), np.abs(rng.normal(0, 1e-7, (5, 48))).astype(np.float32)
+        ma, va = rng.normal(0, 1e-4, 5).astype(np.float32), np.abs(rng.normal(0, 1e-7, 5)).astype(np.float32)
+        hw, ha = AdamW.at_step(3, 2e-5, weight_decay=0.01), AdamW.at_step(3, 1e-4)
+        fw, fa, fmw, fvw, fma, fva, fda = O.bwd_adamw(q, w, a, gb, mw, vw, ma, va, 0.5, hw, ha)
+        dw, da, _ = O.bwd(q, w, a, gb, 0.5)
+        pw, pmw, pvw = O.adamw_step(w, dw, mw, vw, hw)
+        pa, pma, pva = O.adamw_step(a, da, ma, va, ha)
+        for x, y in ((fw.ravel(), pw), (fmw.ravel(), pmw), (fvw.ravel(), pvw),
+                     (fa, pa), (fma, pma), (fva, pva), (fda, da)):
+            assert np.array_equal(x.view(np.uint32), y.view(np.uint32)), q
+
+
 ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_nearest_level, check_binary_sign, check_lsq_textbook,
               check_overflow_example, check_ties_half_even, check_idempotence,
               check_bf16_rne, check_ste, check_dalpha_fd,
               check_dalpha_all_clipped, check_grad_scale, check_pack_golden,
               check_pack_roundtrip, check_dequant_golden,
-              check_dequant_inverts_pack]
+              check_dequant_inverts_pack, check_adamw_vs_torch,
+              check_adamw_first_step, check_bwd_adamw_composes]

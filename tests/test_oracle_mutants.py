@@ -42,6 +42,12 @@ MUTANTS = {
                       "p->lo = -clip_seq; p->hi = clip_seq; p->kh = 1.5f; p->shift = 0.5f;"),
     "grad_scale_no_sqrt": ("(float)(1.0 / sqrt((double)cols * (double)p.qp))",
                            "(float)(1.0 / ((double)cols * (double)p.qp))"),
+    "adamw_no_bias_correction": ("k.step = (float)(h->lr / (1.0 - pow(h->beta1, t)));", "k.step = (float)h->lr;"),
+    "adamw_no_eps": ("volatile float den = sc + k->eps;", "volatile float den = sc;"),
+    "adamw_no_sqrt": ("volatile float sq = sqrtf(*v);", "volatile float sq = *v;"),
+    "adamw_betas_swapped": ("volatile float a1 = k->b1 * *m;", "volatile float a1 = k->b2 * *m;"),
+    "adamw_decay_sign": ("k.decay = (float)(1.0 - h->lr * h->weight_decay);", "k.decay = (float)(1.0 + h->lr * h->weight_decay);"),
+    "adamw_alpha_uses_w_hparams": ("alpha[r] = pqo_adamw_update(&ka,", "alpha[r] = pqo_adamw_update(&kw,"),
     "dequant_no_alpha": ("volatile float prod = lev * alpha;",
                          "volatile float prod = lev;"),
     "binary_sign_zero": ("c = (x >= 0.0f) ? 1 : -1;", "c = (x > 0.0f) ? 1 : -1;"),
@@ -55,6 +61,12 @@ MUTANTS = {
                                "int c = (int)f;"),
     "dequant_field_order": ("unsigned f = (byte >> (p.bits * (int)(j % per_byte))) & mask;",
                             "unsigned f = (byte >> (p.bits * (int)(per_byte - 1 - j % per_byte))) & mask;"),
+    "adamw_no_bias_correction": ("k.step = (float)(h->lr / (1.0 - pow(h->beta1, t)));", "k.step = (float)h->lr;"),
+    "adamw_no_eps": ("volatile float den = sc + k->eps;", "volatile float den = sc;"),
+    "adamw_no_sqrt": ("volatile float sq = sqrtf(*v);", "volatile float sq = *v;"),
+    "adamw_betas_swapped": ("volatile float a1 = k->b1 * *m;", "volatile float a1 = k->b2 * *m;"),
+    "adamw_decay_sign": ("k.decay = (float)(1.0 - h->lr * h->weight_decay);", "k.decay = (float)(1.0 + h->lr * h->weight_decay);"),
+    "adamw_alpha_uses_w_hparams": ("alpha[r] = pqo_adamw_update(&ka,", "alpha[r] = pqo_adamw_update(&kw,"),
     "dequant_no_alpha": ("volatile float prod = pqo_level_of_code(&p, c) * alpha[r];",
                          "volatile float prod = pqo_level_of_code(&p, c);"),
 }
