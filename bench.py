@@ -39,9 +39,10 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--op", choices=["quantizer", "dequant"], default="quantizer",
+    p.add_argument("--op", choices=["quantizer", "dequant", "bwd_adamw"], default="quantizer",
                    help="quantizer: the forward+backward step (the headline); "
-                        "dequant: packed codes -> bf16 over the same layer set")
+                        "dequant: packed codes -> bf16 over the same layer set; "
+                        "bwd_adamw: the backward fused with the AdamW step")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -533,12 +534,112 @@ def run_dequant(args):
     return 0
 
 
+def run_bwd_adamw(args):
+    """The backward fused with one AdamW step over every matrix of the
+    Llama-3-8B-shaped set (one batched launch per step), 1 GPU; beside it,
+    for context, the unfused sequence: the batched backward writing dW, then
+    torch's fused AdamW over the same weights. Prints one JSON line."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.step import QuantStep
+
+    torch.cuda.set_device(0)
+    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device="cuda:0", alloc_outputs=False)
+    step.generate(seed=3)
+    m_w = torch.zeros_like(step.w_all)
+    v_w = torch.zeros_like(step.w_all)
+    m_a = torch.zeros_like(step.alpha_all)
+    v_a = torch.zeros_like(step.alpha_all)
+    descs, o, ro = [], 0, 0
+    for b in step.bufs:
+        n = b.m.numel
+        descs.append(dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
+                          m_w=m_w[o:o + n], v_w=v_w[o:o + n], m_alpha=m_a[ro:ro + b.m.rows],
+                          v_alpha=v_a[ro:ro + b.m.rows], grad_scale=b.grad_scale))
+        o += (n + 63) // 64 * 64
+        ro += (b.m.rows + 63) // 64 * 64
+    arr = pq.adamw_matrix_array(descs)
+    t = [0]
+
+    def fused():
+        t[0] += 1
+        pq.pq_fakequant_bwd_adamw(step.q, arr, pq.adamw(t[0], 2e-5), pq.adamw(t[0], 2e-5))
+
+    for _ in range(max(args.warmup, 1)):
+        fused()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fused()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+
+    # context: backward (dW to memory) + torch fused AdamW on the same data;
+    # our moment buffers make room for torch's
+    del arr, descs, m_w, v_w
+    torch.cuda.empty_cache()
+    dw_all = torch.empty_like(step.w_all)
+    bwd_descs, o = [], 0
+    params = []
+    for b in step.bufs:
+        n = b.m.numel
+        dw = dw_all[o:o + n].view(b.m.rows, b.m.cols)
+        bwd_descs.append(dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
+                              dw=dw, dalpha=b.dalpha, grad_scale=b.grad_scale))
+        prm = torch.nn.Parameter(b.w, requires_grad=True)
+        prm.grad = dw
+        params.append(prm)
+        o += (n + 63) // 64 * 64
+    bwd_arr = pq.matrix_array(bwd_descs)
+    opt = torch.optim.AdamW(params, lr=2e-5, weight_decay=0.0, fused=True)
+
+    def unfused():
+        pq.pq_fakequant_bwd_batch(step.q, bwd_arr)
+        opt.step()
+
+    for _ in range(max(args.warmup, 1)):
+        unfused()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        unfused()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_unfused = e0.elapsed_time(e1) / args.steps
+
+    rows = sum(b.m.rows for b in step.bufs)
+    bytes_step = 26 * step.weights + 24 * rows
+    peak, kind = measured_peaks()
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "backward + AdamW step Gweights/s", "op": "bwd_adamw",
+        "value": step.weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "llama3_8b_linear_set_seq2_bwd_adamw", "weights": step.weights,
+                   "launches_per_step": 1},
+        "roofline": {"bound": "hbm", "kernel": "pq::bwd_adamw_units_kernel<SEQ2, vector layout>",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": f"{kind} hbm_gbs",
+                     "algorithmic_bytes_per_step": bytes_step},
+        "unfused": {"ms_per_step": ms_unfused,
+                    "what": "pq_fakequant_bwd_batch (dW to memory) + torch.optim.AdamW(fused=True)",
+                    "speedup_of_fused": ms_unfused / ms}}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "dequant":
         return run_dequant(args)
+    if args.op == "bwd_adamw":
+        return run_bwd_adamw(args)
     return run_ours(args)
 
 

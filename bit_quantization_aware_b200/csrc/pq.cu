@@ -254,15 +254,18 @@ struct MatDesc {
     int32_t pad_;
 };
 
-struct Batch {
+template <typename D>
+struct BatchT {
     int32_t n;
     int32_t pad_;
     int64_t total_units;
-    MatDesc m[kMaxBatch];
+    D m[kMaxBatch];
 };
+using Batch = BatchT<MatDesc>;
 
 // Moves `mi` forward to the matrix that owns unit u (units increase).
-__device__ __forceinline__ int find_matrix(const Batch& p, int mi, int64_t u) {
+template <typename D>
+__device__ __forceinline__ int find_matrix(const BatchT<D>& p, int mi, int64_t u) {
     while (mi + 1 < p.n && p.m[mi + 1].unit_begin <= u) ++mi;
     return mi;
 }
@@ -534,6 +537,128 @@ dequant_units_kernel(const __grid_constant__ Batch p) {
                     if (i + 1 < n) dst[ch * 8 + i + 1] = static_cast<uint16_t>(hw >> 16);
                 }
             }
+        }
+    }
+}
+
+// ------------------------------------------------ backward fused with AdamW
+// fp32 factors of one AdamW step, formed on the host in double from the
+// hyperparameters and rounded once (see pq_adamw_t in pq.h).
+struct AdamK {
+    float decay, b1, c1, b2, c2, inv_sbc2, step, eps;
+    int32_t has_decay;
+    int32_t pad_;
+};
+
+// AdamW on one parameter: p*decay (if any), m = b1*m + c1*g,
+// v = b2*v + c2*(g*g), p -= step * m / (sqrt(v)*inv_sbc2 + eps); every
+// step rounds on its own (IEEE square root and division).
+__device__ __forceinline__ float adamw_update(const AdamK& k, float p, float g, float& m,
+                                              float& v) {
+    if (k.has_decay) p = __fmul_rn(p, k.decay);
+    m = __fadd_rn(__fmul_rn(k.b1, m), __fmul_rn(k.c1, g));
+    v = __fadd_rn(__fmul_rn(k.b2, v), __fmul_rn(k.c2, __fmul_rn(g, g)));
+    const float den = __fadd_rn(__fmul_rn(__fsqrt_rn(v), k.inv_sbc2), k.eps);
+    return __fsub_rn(p, __fmul_rn(k.step, __fdiv_rn(m, den)));
+}
+
+struct AdamDesc {
+    float* w;              // shadow weights, updated in place
+    float* alpha;          // scales, updated in place
+    const uint16_t* g;     // upstream gradient dWq (bf16)
+    float* m_w;            // first moments of w
+    float* v_w;            // second moments of w
+    float* m_a;            // first moments of alpha
+    float* v_a;            // second moments of alpha
+    float* dalpha;         // d(alpha) out (nullable)
+    int64_t rows;
+    int64_t cols;
+    int64_t unit_begin;
+    float grad_scale;
+    int32_t tpr_log2;
+};
+
+struct AdamBatch {
+    BatchT<AdamDesc> b;
+    AdamK kw;  // weights
+    AdamK ka;  // scales
+};
+
+template <int Q, bool VEC>
+__global__ void __launch_bounds__(kThreads, 3)
+bwd_adamw_units_kernel(const __grid_constant__ AdamBatch P) {
+    const BatchT<AdamDesc>& p = P.b;
+    __shared__ double warp_sum[2][kThreads / 32];
+    int mi = 0, prev_mi = 0, parity = 0;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x, parity ^= 1) {
+        mi = find_matrix(p, mi, u);
+        if (mi != prev_mi) __syncthreads();
+        prev_mi = mi;
+        const AdamDesc& m = p.m[mi];
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rsub = threadIdx.x >> tl;
+        const int64_t row = (u - m.unit_begin) * (kThreads >> tl) + rsub;
+        const int64_t nch = (m.cols + 7) >> 3;
+        double acc = 0.0;
+        if (row < m.rows) {
+            // plain load: alpha is written by this kernel (after every
+            // thread of the row has read it)
+            const RowScale a = row_scale(m.alpha[row]);
+            float* wr = m.w + row * m.cols;
+            const uint16_t* gr = m.g + row * m.cols;
+            float* mr = m.m_w + row * m.cols;
+            float* vr = m.v_w + row * m.cols;
+            for (int64_t ch = lane; ch < nch; ch += tpr) {
+                const int n = VEC ? 8 : tail_n(m.cols, ch);
+                float wv[8], mv[8], vv[8], d[8];
+                uint32_t gw[4];
+                if constexpr (VEC) {
+                    load8(wr + ch * 8, wv);
+                    load_g8(gr + ch * 8, gw);
+                    load8(mr + ch * 8, mv);
+                    load8(vr + ch * 8, vv);
+                } else {
+                    load8_tail(wr + ch * 8, n, wv);
+                    load_g8_tail(gr + ch * 8, n, gw);
+                    load8_tail(mr + ch * 8, n, mv);
+                    load8_tail(vr + ch * 8, n, vv);
+                }
+                acc = bwd_chunk<Q>(wv, gw, a, d, acc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wv[i] = adamw_update(P.kw, wv[i], d[i], mv[i], vv[i]);
+                if constexpr (VEC) {
+                    store8(wr + ch * 8, wv);
+                    store8(mr + ch * 8, mv);
+                    store8(vr + ch * 8, vv);
+                } else {
+                    store8_tail(wr + ch * 8, n, wv);
+                    store8_tail(mr + ch * 8, n, mv);
+                    store8_tail(vr + ch * 8, n, vv);
+                }
+            }
+        }
+        const int seg = tpr < 32 ? tpr : 32;
+        for (int off = seg >> 1; off > 0; off >>= 1)
+            acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off, seg));
+        if (tpr > 32) {
+            if ((threadIdx.x & 31) == 0) warp_sum[parity][threadIdx.x >> 5] = acc;
+            group_barrier(1 + rsub, tpr);
+            if (lane == 0) {
+                const int w0 = threadIdx.x >> 5;
+                double t = warp_sum[parity][w0];
+                for (int k = 1; k < (tpr >> 5); ++k) t = __dadd_rn(t, warp_sum[parity][w0 + k]);
+                acc = t;
+            }
+        }
+        if (lane == 0 && row < m.rows) {
+            const float da = static_cast<float>(__dmul_rn(acc, static_cast<double>(m.grad_scale)));
+            if (m.dalpha) m.dalpha[row] = da;
+            float ma = m.m_a[row], va = m.v_a[row];
+            m.alpha[row] = adamw_update(P.ka, m.alpha[row], da, ma, va);
+            m.m_a[row] = ma;
+            m.v_a[row] = va;
         }
     }
 }
@@ -843,6 +968,96 @@ static pq_status_t dequant_batch_impl(int q, int32_t n, const pq_matrix_t* mats,
     return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
 }
 
+static AdamK adamw_consts(const pq_adamw_t& h) {
+    AdamK k;
+    const double t = static_cast<double>(h.step);
+    k.decay = static_cast<float>(1.0 - h.lr * h.weight_decay);
+    k.has_decay = h.weight_decay != 0.0;
+    k.b1 = static_cast<float>(h.beta1);
+    k.c1 = static_cast<float>(1.0 - h.beta1);
+    k.b2 = static_cast<float>(h.beta2);
+    k.c2 = static_cast<float>(1.0 - h.beta2);
+    k.inv_sbc2 = static_cast<float>(1.0 / sqrt(1.0 - pow(h.beta2, t)));
+    k.step = static_cast<float>(h.lr / (1.0 - pow(h.beta1, t)));
+    k.eps = static_cast<float>(h.eps);
+    k.pad_ = 0;
+    return k;
+}
+
+static bool adamw_ok(const pq_adamw_t* h) {
+    return h && h->step >= 1 && h->beta1 >= 0.0 && h->beta1 < 1.0 && h->beta2 >= 0.0 &&
+           h->beta2 < 1.0 && h->eps > 0.0 && h->lr >= 0.0;
+}
+
+template <int Q, bool VEC>
+static void launch_bwd_adamw(const AdamBatch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    auto k = bwd_adamw_units_kernel<Q, VEC>;
+    const int64_t ctas = persistent_ctas(k, cache);
+    const unsigned grid = static_cast<unsigned>(b.b.total_units < ctas ? b.b.total_units : ctas);
+    k<<<grid, kThreads, 0, s>>>(b);
+}
+
+static pq_status_t bwd_adamw_impl(int q, int32_t n, const pq_adamw_matrix_t* mats,
+                                  const pq_adamw_t* hw, const pq_adamw_t* ha, cudaStream_t s) {
+    if (code_bits_of(q) == 0 || n < 0 || (n > 0 && !mats)) return PQ_ERR_INVALID_ARG;
+    if (!adamw_ok(hw) || !adamw_ok(ha)) return PQ_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        const pq_adamw_matrix_t& m = mats[i];
+        if (m.rows < 0 || m.cols < 0) return PQ_ERR_INVALID_ARG;
+        if (m.rows == 0) continue;
+        if (!m.alpha || !m.m_alpha || !m.v_alpha) return PQ_ERR_INVALID_ARG;
+        if (m.cols > 0 && (!m.w || !m.g_bf16 || !m.m_w || !m.v_w)) return PQ_ERR_INVALID_ARG;
+    }
+    static thread_local AdamBatch b;
+    b.kw = adamw_consts(*hw);
+    b.ka = adamw_consts(*ha);
+    bool launched = false;
+    for (int cls = 0; cls < 2; ++cls) {
+        const bool vec = cls == 0;
+        b.b.n = 0;
+        b.b.pad_ = 0;
+        b.b.total_units = 0;
+        auto flush = [&]() {
+            if (b.b.n == 0) return;
+            launched = true;
+            dispatch_q(q, [&]<int Q>() {
+                if (vec) launch_bwd_adamw<Q, true>(b, s);
+                else launch_bwd_adamw<Q, false>(b, s);
+            });
+            b.b.n = 0;
+            b.b.total_units = 0;
+        };
+        for (int32_t i = 0; i < n; ++i) {
+            const pq_adamw_matrix_t& m = mats[i];
+            if (m.rows == 0) continue;
+            // rows without columns still take an AdamW step on alpha with
+            // d(alpha) = 0: they go through the element path
+            const bool v = m.cols > 0 && m.cols % 8 == 0 && aligned(m.w, 16) &&
+                           aligned(m.g_bf16, 16) && aligned(m.m_w, 16) && aligned(m.v_w, 16);
+            if (v != vec) continue;
+            if (b.b.n == kMaxBatch) flush();
+            AdamDesc& d = b.b.m[b.b.n++];
+            d.w = m.w;
+            d.alpha = m.alpha;
+            d.g = m.g_bf16;
+            d.m_w = m.m_w;
+            d.v_w = m.v_w;
+            d.m_a = m.m_alpha;
+            d.v_a = m.v_alpha;
+            d.dalpha = m.dalpha_out;
+            d.rows = m.rows;
+            d.cols = m.cols;
+            d.unit_begin = b.b.total_units;
+            d.grad_scale = m.grad_scale;
+            d.tpr_log2 = choose_tpr_log2(m.cols);
+            b.b.total_units += (m.rows + (kThreads >> d.tpr_log2) - 1) / (kThreads >> d.tpr_log2);
+        }
+        flush();
+    }
+    return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
+}
+
 }  // namespace pq
 
 using namespace pq;
@@ -918,6 +1133,12 @@ pq_status_t pq_dequant_codes(pq_quant_t q, int64_t rows, int64_t cols, const uin
 pq_status_t pq_dequant_codes_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,
                                    void* stream) {
     return dequant_batch_impl(q, n, mats, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_fakequant_bwd_adamw(pq_quant_t q, int32_t n, const pq_adamw_matrix_t* mats,
+                                   const pq_adamw_t* hp_w, const pq_adamw_t* hp_alpha,
+                                   void* stream) {
+    return bwd_adamw_impl(q, n, mats, hp_w, hp_alpha, static_cast<cudaStream_t>(stream));
 }
 
 pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,

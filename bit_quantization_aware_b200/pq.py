@@ -50,12 +50,32 @@ class PQMatrix(ctypes.Structure):
                 ("dalpha_out", ctypes.c_void_p), ("grad_scale", ctypes.c_float)]
 
 
+class PQAdamW(ctypes.Structure):
+    """``pq_adamw_t``: hyperparameters of one AdamW step (step >= 1)."""
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
+                ("weight_decay", ctypes.c_double), ("step", ctypes.c_int64)]
+
+
+class PQAdamWMatrix(ctypes.Structure):
+    """``pq_adamw_matrix_t``: one matrix of the fused backward + AdamW."""
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("w", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("g_bf16", ctypes.c_void_p), ("m_w", ctypes.c_void_p),
+                ("v_w", ctypes.c_void_p), ("m_alpha", ctypes.c_void_p),
+                ("v_alpha", ctypes.c_void_p), ("dalpha_out", ctypes.c_void_p),
+                ("grad_scale", ctypes.c_float)]
+
+
 def _declare(L):
     i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.pq_fakequant_fwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_fakequant_fwd_batch.restype = i32
     L.pq_fakequant_bwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_fakequant_bwd_batch.restype = i32
+    L.pq_fakequant_bwd_adamw.argtypes = [i32, i32, ctypes.POINTER(PQAdamWMatrix),
+                                         ctypes.POINTER(PQAdamW), ctypes.POINTER(PQAdamW), p]
+    L.pq_fakequant_bwd_adamw.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_dequant_codes_batch.restype = i32
     L.pq_dequant_codes.argtypes = [i32, i64, i64, p, p, p, p]
@@ -200,6 +220,32 @@ def pq_fakequant_bwd_batch(q, mats, stream=None):
     """Backward over a ``pq_matrix_t[]`` (see ``matrix_array``)."""
     _check("pq_fakequant_bwd_batch", lib().pq_fakequant_bwd_batch(
         q, len(mats), mats, _stream(stream)))
+
+
+def adamw_matrix_array(descs):
+    """Build a ``pq_adamw_matrix_t[]`` from dicts with keys rows, cols, w,
+    alpha, g, m_w, v_w, m_alpha, v_alpha, dalpha (optional), grad_scale."""
+    arr = (PQAdamWMatrix * len(descs))()
+    for i, d in enumerate(descs):
+        m = arr[i]
+        m.rows, m.cols = int(d["rows"]), int(d["cols"])
+        m.w, m.alpha, m.g_bf16 = _ptr(d.get("w")), _ptr(d.get("alpha")), _ptr(d.get("g"))
+        m.m_w, m.v_w = _ptr(d.get("m_w")), _ptr(d.get("v_w"))
+        m.m_alpha, m.v_alpha = _ptr(d.get("m_alpha")), _ptr(d.get("v_alpha"))
+        m.dalpha_out = _ptr(d.get("dalpha"))
+        m.grad_scale = float(d.get("grad_scale", 0.0))
+    return arr
+
+
+def adamw(step, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0):
+    return PQAdamW(lr, beta1, beta2, eps, weight_decay, step)
+
+
+def pq_fakequant_bwd_adamw(q, mats, hp_w, hp_alpha, stream=None):
+    """Backward fused with one AdamW step over a ``pq_adamw_matrix_t[]``."""
+    _check("pq_fakequant_bwd_adamw", lib().pq_fakequant_bwd_adamw(
+        q, len(mats), mats, ctypes.byref(hp_w), ctypes.byref(hp_alpha),
+        _stream(stream)))
 
 
 def pq_code_bits(q) -> int:

@@ -177,6 +177,55 @@ PQ_API pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n,
 PQ_API pq_status_t pq_fakequant_bwd_batch(pq_quant_t q, int32_t n,
                                           const pq_matrix_t* mats, void* stream);
 
+/* Hyperparameters of one AdamW step (decoupled weight decay). The library
+ * forms its scalar factors once in double and rounds each to fp32:
+ * decay = 1 - lr*weight_decay, beta1, 1 - beta1, beta2, 1 - beta2,
+ * 1/sqrt(1 - beta2^step), lr/(1 - beta1^step), eps. Requires step >= 1,
+ * 0 <= beta < 1, eps > 0, lr >= 0. [P1 "The 2-bit recipe, in full":
+ * AdamW, weight decay 0; betas and eps are not stated there.] */
+typedef struct {
+    double lr;
+    double beta1;
+    double beta2;
+    double eps;
+    double weight_decay;
+    int64_t step;
+} pq_adamw_t;
+
+/* One weight matrix of pq_fakequant_bwd_adamw (device pointers). */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    float* w;                 /* fp32 [rows*cols], updated in place */
+    float* alpha;             /* fp32 [rows], updated in place */
+    const uint16_t* g_bf16;   /* bf16 [rows*cols], upstream dWq */
+    float* m_w;               /* fp32 [rows*cols], AdamW first moments of w */
+    float* v_w;               /* fp32 [rows*cols], second moments of w */
+    float* m_alpha;           /* fp32 [rows], first moments of alpha */
+    float* v_alpha;           /* fp32 [rows], second moments of alpha */
+    float* dalpha_out;        /* fp32 [rows] or NULL: d(alpha) as computed */
+    float grad_scale;         /* as in pq_fakequant_bwd */
+} pq_adamw_matrix_t;
+
+/* Backward fused with the optimizer step: for every matrix, the STE
+ * gradient dW and d(alpha) of pq_fakequant_bwd are formed from the CURRENT
+ * w and alpha, then one AdamW step updates every weight (gradient dW,
+ * hyperparameters hp_w) and every row's alpha (gradient: the fp32
+ * d(alpha), hyperparameters hp_alpha), in one pass: dW never goes to
+ * memory. Per weight, element by element in fp32 (each step rounded on its
+ * own): p = p*decay (if weight_decay != 0); m = beta1*m + (1-beta1)*g;
+ * v = beta2*v + (1-beta2)*(g*g); p = p - (lr/bc1) * (m / (sqrt(v)/sqrt(bc2) +
+ * eps)), with 1/sqrt(bc2) a precomputed factor. With data-parallel
+ * replicas, all-reduce g_bf16 first: dW and d(alpha) are linear in it and
+ * the STE mask is identical on every replica.
+ * Traffic: 14 B read + 12 B written per weight (38 B for the backward
+ * followed by a separate AdamW). Batched like pq_fakequant_bwd_batch; the
+ * buffers of different matrices must not overlap. */
+PQ_API pq_status_t pq_fakequant_bwd_adamw(pq_quant_t q, int32_t n,
+                                          const pq_adamw_matrix_t* mats,
+                                          const pq_adamw_t* hp_w,
+                                          const pq_adamw_t* hp_alpha, void* stream);
+
 /* Dequantize packed codes back to bf16 weights: each stored code c (layout
  * of packed_out above) becomes bf16_rn(fl(level(c) * alpha_row)) with the
  * forward's level formulas, so the result equals the forward's

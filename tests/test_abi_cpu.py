@@ -31,6 +31,7 @@ def test_header_declares_entry_points():
     for n in ("pq_fakequant_fwd", "pq_fakequant_bwd", "pq_pack_codes",
               "pq_fakequant_fwd_batch", "pq_fakequant_bwd_batch",
               "pq_scaled_weights", "pq_dequant_codes", "pq_dequant_codes_batch",
+              "pq_fakequant_bwd_adamw",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
               "pq_last_cuda_error"):
         assert n in names
@@ -145,3 +146,25 @@ def test_batch_argument_errors_launch_nothing(L):
     assert L.pq_fakequant_fwd_batch(pq.PQ_SEQ2, 2, arr, None) == pq.PQ_OK
     arr = pq.matrix_array([dict(rows=0, cols=8)])
     assert L.pq_fakequant_bwd_batch(pq.PQ_SEQ2, 1, arr, None) == pq.PQ_OK
+
+
+def test_adamw_argument_errors(L):
+    from bit_quantization_aware_b200 import pq
+    E = pq.PQ_ERR_INVALID_ARG
+    fake = 0x10000
+    good = dict(rows=4, cols=8, w=fake, alpha=fake, g=fake, m_w=fake, v_w=fake,
+                m_alpha=fake, v_alpha=fake, grad_scale=1.0)
+    h = pq.adamw(1, 1e-3)
+    f = pq.lib().pq_fakequant_bwd_adamw
+    import ctypes
+    arr = pq.adamw_matrix_array([good])
+    assert f(pq.PQ_SEQ2, 1, arr, ctypes.byref(pq.adamw(0, 1e-3)), ctypes.byref(h), None) == E
+    assert f(pq.PQ_SEQ2, 1, arr, ctypes.byref(h), ctypes.byref(pq.adamw(1, 1e-3, beta1=1.0)), None) == E
+    assert f(pq.PQ_SEQ2, 1, arr, None, ctypes.byref(h), None) == E
+    assert f(99, 1, arr, ctypes.byref(h), ctypes.byref(h), None) == E
+    for bad in (dict(good, m_w=None), dict(good, alpha=None), dict(good, rows=-1),
+                dict(good, v_alpha=None)):
+        arr = pq.adamw_matrix_array([dict(good, rows=0), bad])
+        assert f(pq.PQ_SEQ2, 2, arr, ctypes.byref(h), ctypes.byref(h), None) == E
+    arr = pq.adamw_matrix_array([dict(rows=0, cols=8)])
+    assert f(pq.PQ_SEQ2, 1, arr, ctypes.byref(h), ctypes.byref(h), None) == pq.PQ_OK

@@ -497,3 +497,107 @@ def test_dequant_batch_equals_single_calls():
     torch.cuda.synchronize()
     for o1, o2 in singles:
         assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def _adamw_case(q, rows, cols, seed, offset=0):
+    rng = np.random.default_rng(seed)
+    w, a, g = make_case(rows, cols, q, seed=seed, special=rows * cols >= 8)
+    mw = rng.normal(0, 1e-4, (rows, cols)).astype(np.float32)
+    vw = np.abs(rng.normal(0, 1e-7, (rows, cols))).astype(np.float32)
+    ma = rng.normal(0, 1e-3, rows).astype(np.float32)
+    va = np.abs(rng.normal(0, 1e-6, rows)).astype(np.float32)
+    return w.numpy(), a.numpy(), g.view(torch.int16).numpy().view(np.uint16), mw, vw, ma, va
+
+
+def _adamw_gpu(q, w, a, g, mw, vw, ma, va, gs, hw, ha, offset=0):
+    rows, cols = w.shape
+    n = rows * cols
+
+    def dev(x, dtype):
+        buf = torch.empty(n + offset + 8, dtype=dtype, device=DEV)
+        t = buf[offset:offset + n]
+        t.copy_(torch.from_numpy(np.ascontiguousarray(x).ravel()))
+        return t
+
+    wd = dev(w, torch.float32)
+    gd = dev(g.view(np.int16), torch.int16)
+    mwd, vwd = dev(mw, torch.float32), dev(vw, torch.float32)
+    ad = torch.from_numpy(a.copy()).to(DEV)
+    mad, vad = torch.from_numpy(ma.copy()).to(DEV), torch.from_numpy(va.copy()).to(DEV)
+    da = torch.full((rows,), float("nan"), device=DEV)
+    arr = pq.adamw_matrix_array([dict(rows=rows, cols=cols, w=wd, alpha=ad, g=gd, m_w=mwd,
+                                      v_w=vwd, m_alpha=mad, v_alpha=vad, dalpha=da,
+                                      grad_scale=gs)])
+    pq.pq_fakequant_bwd_adamw(q, arr, hw, ha)
+    torch.cuda.synchronize()
+    f = lambda t: t.cpu().numpy().reshape(-1)
+    return (f(wd).reshape(rows, cols), f(ad), f(mwd).reshape(rows, cols),
+            f(vwd).reshape(rows, cols), f(mad), f(vad), f(da))
+
+
+def _check_adamw(q, w, a, g, mw, vw, ma, va, gs, t, offset=0):
+    from oracle.pq_oracle import AdamW
+    hw_o, ha_o = AdamW.at_step(t, 2e-5, weight_decay=0.01), AdamW.at_step(t, 1e-4)
+    hw, ha = pq.adamw(t, 2e-5, weight_decay=0.01), pq.adamw(t, 1e-4)
+    got = _adamw_gpu(q, w, a, g, mw, vw, ma, va, gs, hw, ha, offset)
+    ref = pq_oracle.default().bwd_adamw(q, w, a, g, mw, vw, ma, va, gs, hw_o, ha_o)
+    for name, x, y in zip(("w", "m_w", "v_w"), (got[0], got[2], got[3]),
+                          (ref[0], ref[2], ref[3])):
+        bad = np.argwhere(x.view(np.uint32) != y.view(np.uint32))
+        assert bad.size == 0, f"q={q} t={t} {name}: {len(bad)} mismatches, first {bad[0].tolist()}"
+    # d(alpha) within the reduction-order tolerance; alpha's own AdamW step
+    # from the GPU's d(alpha) is exact
+    _, ref_da, row_abs = pq_oracle.bwd(q, w, a, g, gs)
+    tol = 1e-4 * np.maximum(np.abs(ref_da), 1e-6 * gs * row_abs)
+    assert np.all(np.abs(got[6].astype(np.float64) - ref_da) <= tol), q
+    pa, pma, pva = pq_oracle.default().adamw_step(a, got[6], ma, va, ha_o)
+    for x, y in ((got[1], pa), (got[4], pma), (got[5], pva)):
+        assert np.array_equal(x.view(np.uint32), y.view(np.uint32)), q
+    return got
+
+
+@pytest.mark.parametrize("q", ALLQ)
+@pytest.mark.parametrize("shape,offset", [((33, 1032), 0), ((7, 1000), 0), ((5, 12), 0),
+                                          ((64, 4096), 0), ((9, 2048), 1), ((3, 0), 0)])
+def test_bwd_adamw_two_steps(q, shape, offset):
+    """Fused backward + AdamW: two consecutive steps (the second from the
+    GPU's state), weights and moments bit-exact against the oracle."""
+    rows, cols = shape
+    w, a, g, mw, vw, ma, va = _adamw_case(q, rows, cols, seed=50 + rows)
+    gs = pq.pq_default_grad_scale(q, cols) if cols else 1.0
+    got = _check_adamw(q, w, a, g, mw, vw, ma, va, gs, 1, offset)
+    w2, a2, mw2, vw2, ma2, va2 = got[0], got[1], got[2], got[3], got[4], got[5]
+    _check_adamw(q, w2, a2, g, mw2, vw2, ma2, va2, gs, 2, offset)
+
+
+def test_bwd_adamw_batch_2048x8192_and_stack():
+    """Batched fused step over mixed matrices (2048x8192 and a 1B-stack
+    layer) equals single-matrix calls bit for bit."""
+    q = pq.PQ_SEQ2
+    mats = [I.Matrix("big", 2048, 8192, 0, 0)] + I.llama_1b_stack()[:7]
+    hw, ha = pq.adamw(5, 2e-5), pq.adamw(5, 1e-4)
+    states = []
+    for i, m in enumerate(mats):
+        w = I.normal_weights(m.rows, m.cols, seed=60 + i, stream=0, device=DEV)
+        a = I.alpha_init(w, q)
+        g = I.grad_bf16(m.rows, m.cols, seed=60 + i, stream=64, device=DEV)
+        mw = torch.randn_like(w) * 1e-4
+        vw = torch.rand_like(w) * 1e-7
+        ma = torch.randn_like(a) * 1e-3
+        va = torch.rand_like(a) * 1e-6
+        states.append([w, a, g, mw, vw, ma, va])
+    clones = [[t.clone() for t in st] for st in states]
+
+    def desc(st, m):
+        w, a, g, mw, vw, ma, va = st
+        return dict(rows=m.rows, cols=m.cols, w=w, alpha=a, g=g, m_w=mw, v_w=vw,
+                    m_alpha=ma, v_alpha=va, grad_scale=pq.pq_default_grad_scale(q, m.cols))
+
+    pq.pq_fakequant_bwd_adamw(q, pq.adamw_matrix_array([desc(st, m) for st, m in zip(states, mats)]), hw, ha)
+    for st, m in zip(clones, mats):
+        pq.pq_fakequant_bwd_adamw(q, pq.adamw_matrix_array([desc(st, m)]), hw, ha)
+    torch.cuda.synchronize()
+    for s1, s2 in zip(states, clones):
+        for x, y in zip(s1, s2):
+            assert torch.equal(x.view(torch.uint8) if x.dtype != torch.bfloat16 else x.view(torch.int16),
+                               y.view(torch.uint8) if y.dtype != torch.bfloat16 else y.view(torch.int16))
