@@ -382,6 +382,44 @@ int pqo_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alpha,
     return 0;
 }
 
+/* Backward + AdamW of one row shard whose upstream gradient is the sum of
+ * n_src bf16 gradients (one per data-parallel replica, for the same rows):
+ * gbar = fl(fl(sum_k g_k) * grad_mult), summed in source order in fp32;
+ * then exactly pqo_bwd_adamw's steps with the fp32 gbar in place of g
+ * (dW = inside ? gbar : 0; the d(alpha) term is gbar*(level - inside*x)). */
+int pqo_reduce_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alpha,
+                         int n_src, const uint16_t* const* g_srcs, float grad_mult,
+                         float* m_w, float* v_w, float* m_a, float* v_a, float grad_scale,
+                         const pqo_adamw* hw, const pqo_adamw* ha, float* dalpha) {
+    pqo_params p;
+    if (pqo_get_params(q, &p) || rows < 0 || cols < 0 || n_src < 1 || !g_srcs || !hw || !ha)
+        return -1;
+    const pqo_adamw_k kw = pqo_adamw_consts(hw), ka = pqo_adamw_consts(ha);
+    for (int64_t r = 0; r < rows; ++r) {
+        const float a = alpha[r];
+        double acc = 0.0;
+        for (int64_t j = 0; j < cols; ++j) {
+            float sum = 0.0f;
+            for (int k = 0; k < n_src; ++k) {
+                volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);
+                sum = t;
+            }
+            volatile float gbar = sum * grad_mult;
+            int inside;
+            float lev, x;
+            pqo_quantize_scalar(q, w[r * cols + j], a, 0.0f, NULL, &lev, NULL, &inside, &x);
+            const float dw = inside ? gbar : 0.0f;
+            acc += (double)gbar * ((double)lev - (inside ? (double)x : 0.0));
+            w[r * cols + j] = pqo_adamw_update(&kw, w[r * cols + j], dw, &m_w[r * cols + j],
+                                               &v_w[r * cols + j]);
+        }
+        const float da = (float)(acc * (double)grad_scale);
+        alpha[r] = pqo_adamw_update(&ka, a, da, &m_a[r], &v_a[r]);
+        if (dalpha) dalpha[r] = da;
+    }
+    return 0;
+}
+
 /* One AdamW step over n parameters with given gradients (for pinning the
  * update rule against a library optimizer). */
 int pqo_adamw_step(int64_t n, float* p, const float* g, float* m, float* v,

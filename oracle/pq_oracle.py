@@ -82,6 +82,10 @@ class Oracle:
                                     ctypes.c_float, ctypes.POINTER(AdamW),
                                     ctypes.POINTER(AdamW), p]
         L.pqo_bwd_adamw.restype = ctypes.c_int
+        L.pqo_reduce_bwd_adamw.argtypes = [ctypes.c_int, i64, i64, p, p, ctypes.c_int, p,
+                                           ctypes.c_float, p, p, p, p, ctypes.c_float,
+                                           ctypes.POINTER(AdamW), ctypes.POINTER(AdamW), p]
+        L.pqo_reduce_bwd_adamw.restype = ctypes.c_int
         L.pqo_adamw_step.argtypes = [i64, p, p, p, p, ctypes.POINTER(AdamW)]
         L.pqo_adamw_step.restype = ctypes.c_int
         L.pqo_default_grad_scale.argtypes = [ctypes.c_int, i64]
@@ -177,6 +181,29 @@ class Oracle:
                                     ctypes.byref(ha), _ptr(da))
         if rc != 0:
             raise ValueError("oracle bwd_adamw rejected its arguments")
+        return w, alpha, m_w, v_w, m_a, v_a, da
+
+    def reduce_bwd_adamw(self, q, w, alpha, g_list, grad_mult, m_w, v_w, m_a, v_a,
+                         grad_scale, hw, ha):
+        """Backward + AdamW with the upstream gradient summed over the bf16
+        arrays of g_list; returns (w, alpha, m_w, v_w, m_a, v_a, dalpha)."""
+        w = np.array(w, np.float32, order="C", copy=True)
+        rows, cols = w.shape
+        alpha = np.array(alpha, np.float32, copy=True).reshape(rows)
+        gs = [np.ascontiguousarray(g).view(np.uint16) for g in g_list]
+        ptrs = (ctypes.c_void_p * len(gs))(*[g.ctypes.data for g in gs])
+        m_w = np.array(m_w, np.float32, order="C", copy=True)
+        v_w = np.array(v_w, np.float32, order="C", copy=True)
+        m_a = np.array(m_a, np.float32, copy=True).reshape(rows)
+        v_a = np.array(v_a, np.float32, copy=True).reshape(rows)
+        da = np.empty(rows, np.float32)
+        rc = self.lib.pqo_reduce_bwd_adamw(q, rows, cols, _ptr(w), _ptr(alpha), len(gs),
+                                           ctypes.cast(ptrs, ctypes.c_void_p),
+                                           ctypes.c_float(grad_mult), _ptr(m_w), _ptr(v_w),
+                                           _ptr(m_a), _ptr(v_a), ctypes.c_float(grad_scale),
+                                           ctypes.byref(hw), ctypes.byref(ha), _ptr(da))
+        if rc != 0:
+            raise ValueError("oracle reduce_bwd_adamw rejected its arguments")
         return w, alpha, m_w, v_w, m_a, v_a, da
 
     def adamw_step(self, p, g, m, v, h):

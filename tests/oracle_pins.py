@@ -472,6 +472,51 @@ def check_bwd_adamw_composes(O):
             assert np.array_equal(x.view(np.uint32), y.view(np.uint32)), q
 
 
+def check_reduce_equals_single_source(O):
+    """The multi-source backward + AdamW reduces to the single-source one:
+    one source with multiplier 1, and n identical sources with multiplier
+    1/n (n a power of two, so the mean is exact), give the same bits."""
+    from oracle.pq_oracle import AdamW
+    rng = np.random.default_rng(53)
+    for q in ALL_QUANTIZERS:
+        w = rng.normal(0, 0.02, (4, 40)).astype(np.float32)
+        a = (np.abs(w).max(axis=1) * 0.7).astype(np.float32)
+        gb = torch.randn(4, 40).mul(1e-3).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        st = [rng.normal(0, 1e-4, (4, 40)).astype(np.float32),
+              np.abs(rng.normal(0, 1e-7, (4, 40))).astype(np.float32),
+              rng.normal(0, 1e-4, 4).astype(np.float32),
+              np.abs(rng.normal(0, 1e-7, 4)).astype(np.float32)]
+        hw, ha = AdamW.at_step(2, 2e-5), AdamW.at_step(2, 1e-4)
+        ref = O.bwd_adamw(q, w, a, gb, *st, 0.5, hw, ha)
+        for n, mult in ((1, 1.0), (2, 0.5), (4, 0.25)):
+            got = O.reduce_bwd_adamw(q, w, a, [gb] * n, mult, *st, 0.5, hw, ha)
+            for x, y in zip(got, ref):
+                assert np.array_equal(np.asarray(x).view(np.uint32),
+                                      np.asarray(y).view(np.uint32)), (q, n)
+
+
+def check_reduce_sums_in_fp32(O):
+    """With two different sources the gradient is their fp32 sum: the
+    weights inside the clip range move as Adam's first step moves them for
+    g = g0 + g1 (computed here with numpy), outside they do not move."""
+    from oracle.pq_oracle import AdamW
+    rng = np.random.default_rng(59)
+    w = rng.normal(0, 0.02, (3, 64)).astype(np.float32)
+    a = (np.abs(w).max(axis=1) * 0.6).astype(np.float32)  # some clipped
+    g0 = torch.randn(3, 64).mul(1e-3).to(torch.bfloat16)
+    g1 = torch.randn(3, 64).mul(1e-3).to(torch.bfloat16)
+    gsum = (g0.float() + g1.float()).numpy()
+    z = np.zeros_like(w)
+    hw = AdamW.at_step(1, 1e-3)
+    nw, *_ = O.reduce_bwd_adamw(SEQ2, w, a, [g0.view(torch.int16).numpy(), g1.view(torch.int16).numpy()],
+                                1.0, z, z, np.zeros(3, np.float32), np.zeros(3, np.float32),
+                                0.5, hw, AdamW.at_step(1, 1e-4))
+    inside = np.abs(w / a[:, None]) <= np.float32(0.99)
+    step = -1e-3 * gsum / (np.abs(gsum) + 1e-8)
+    assert np.allclose((nw - w)[inside], step[inside], rtol=1e-4, atol=1e-9)
+    assert np.array_equal(nw[~inside], w[~inside])
+
+
 ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_nearest_level, check_binary_sign, check_lsq_textbook,
               check_overflow_example, check_ties_half_even, check_idempotence,
@@ -479,4 +524,5 @@ ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_dalpha_all_clipped, check_grad_scale, check_pack_golden,
               check_pack_roundtrip, check_dequant_golden,
               check_dequant_inverts_pack, check_adamw_vs_torch,
-              check_adamw_first_step, check_bwd_adamw_composes]
+              check_adamw_first_step, check_bwd_adamw_composes,
+              check_reduce_equals_single_source, check_reduce_sums_in_fp32]

@@ -48,6 +48,9 @@ MUTANTS = {
     "adamw_betas_swapped": ("volatile float a1 = k->b1 * *m;", "volatile float a1 = k->b2 * *m;"),
     "adamw_decay_sign": ("k.decay = (float)(1.0 - h->lr * h->weight_decay);", "k.decay = (float)(1.0 + h->lr * h->weight_decay);"),
     "adamw_alpha_uses_w_hparams": ("alpha[r] = pqo_adamw_update(&ka,", "alpha[r] = pqo_adamw_update(&kw,"),
+    "reduce_no_multiplier": ("volatile float gbar = sum * grad_mult;", "volatile float gbar = sum;"),
+    "reduce_first_source_only": ("volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);",
+                                 "volatile float t = pqo_bf16_to_float(g_srcs[0][r * cols + j]);"),
     "dequant_no_alpha": ("volatile float prod = lev * alpha;",
                          "volatile float prod = lev;"),
     "binary_sign_zero": ("c = (x >= 0.0f) ? 1 : -1;", "c = (x > 0.0f) ? 1 : -1;"),
@@ -67,6 +70,9 @@ MUTANTS = {
     "adamw_betas_swapped": ("volatile float a1 = k->b1 * *m;", "volatile float a1 = k->b2 * *m;"),
     "adamw_decay_sign": ("k.decay = (float)(1.0 - h->lr * h->weight_decay);", "k.decay = (float)(1.0 + h->lr * h->weight_decay);"),
     "adamw_alpha_uses_w_hparams": ("alpha[r] = pqo_adamw_update(&ka,", "alpha[r] = pqo_adamw_update(&kw,"),
+    "reduce_no_multiplier": ("volatile float gbar = sum * grad_mult;", "volatile float gbar = sum;"),
+    "reduce_first_source_only": ("volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);",
+                                 "volatile float t = pqo_bf16_to_float(g_srcs[0][r * cols + j]);"),
     "dequant_no_alpha": ("volatile float prod = pqo_level_of_code(&p, c) * alpha[r];",
                          "volatile float prod = pqo_level_of_code(&p, c);"),
 }
