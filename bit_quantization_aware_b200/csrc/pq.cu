@@ -235,6 +235,23 @@ __device__ __forceinline__ double bwd_chunk(const float (&v)[8], const uint32_t 
     return acc;
 }
 
+// Backward of one chunk with an fp32 upstream gradient (already reduced).
+template <int Q>
+__device__ __forceinline__ double bwd_chunk_f32(const float (&v)[8], const float (&g)[8],
+                                                const RowScale& s, float (&d)[8], double acc) {
+    float x[8];
+    divide8(v, s, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const Elem e = quantize_x<Q>(x[i]);
+        d[i] = e.inside ? g[i] : 0.0f;
+        const float xm = e.inside ? x[i] : 0.0f;
+        acc = __fma_rn(static_cast<double>(g[i]),
+                       __dsub_rn(static_cast<double>(e.level), static_cast<double>(xm)), acc);
+    }
+    return acc;
+}
+
 // ------------------------------------------------------------ batches
 // Device-side descriptor of one matrix of a batch (kernel parameter space).
 struct MatDesc {
@@ -626,6 +643,126 @@ bwd_adamw_units_kernel(const __grid_constant__ AdamBatch P) {
                     load8_tail(vr + ch * 8, n, vv);
                 }
                 acc = bwd_chunk<Q>(wv, gw, a, d, acc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wv[i] = adamw_update(P.kw, wv[i], d[i], mv[i], vv[i]);
+                if constexpr (VEC) {
+                    store8(wr + ch * 8, wv);
+                    store8(mr + ch * 8, mv);
+                    store8(vr + ch * 8, vv);
+                } else {
+                    store8_tail(wr + ch * 8, n, wv);
+                    store8_tail(mr + ch * 8, n, mv);
+                    store8_tail(vr + ch * 8, n, vv);
+                }
+            }
+        }
+        const int seg = tpr < 32 ? tpr : 32;
+        for (int off = seg >> 1; off > 0; off >>= 1)
+            acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off, seg));
+        if (tpr > 32) {
+            if ((threadIdx.x & 31) == 0) warp_sum[parity][threadIdx.x >> 5] = acc;
+            group_barrier(1 + rsub, tpr);
+            if (lane == 0) {
+                const int w0 = threadIdx.x >> 5;
+                double t = warp_sum[parity][w0];
+                for (int k = 1; k < (tpr >> 5); ++k) t = __dadd_rn(t, warp_sum[parity][w0 + k]);
+                acc = t;
+            }
+        }
+        if (lane == 0 && row < m.rows) {
+            const float da = static_cast<float>(__dmul_rn(acc, static_cast<double>(m.grad_scale)));
+            if (m.dalpha) m.dalpha[row] = da;
+            float ma = m.m_a[row], va = m.v_a[row];
+            m.alpha[row] = adamw_update(P.ka, m.alpha[row], da, ma, va);
+            m.m_a[row] = ma;
+            m.v_a[row] = va;
+        }
+    }
+}
+
+// ------------------------------- reduce-scatter fused with backward + AdamW
+// One rank's row shards: the upstream gradient of each shard row is summed
+// over the n_src replicas' bf16 gradients (buffers of identical layout,
+// local or on peer GPUs), in source order in fp32, times grad_mult; then the
+// backward and AdamW of bwd_adamw_units_kernel.
+constexpr int kMaxSources = 16;
+
+struct ShardDesc {
+    float* w;
+    float* alpha;
+    float* m_w;
+    float* v_w;
+    float* m_a;
+    float* v_a;
+    float* dalpha;
+    int64_t rows;
+    int64_t cols;
+    int64_t g_offset;      // element offset of row 0 in every source buffer
+    int64_t unit_begin;
+    float grad_scale;
+    int32_t tpr_log2;
+};
+
+struct ReduceBatch {
+    BatchT<ShardDesc> b;
+    const uint16_t* src[kMaxSources];
+    int32_t n_src;
+    float grad_mult;
+    AdamK kw;
+    AdamK ka;
+};
+
+template <int Q, bool VEC>
+__global__ void __launch_bounds__(kThreads, 3)
+reduce_bwd_adamw_units_kernel(const __grid_constant__ ReduceBatch P) {
+    const BatchT<ShardDesc>& p = P.b;
+    __shared__ double warp_sum[2][kThreads / 32];
+    int mi = 0, prev_mi = 0, parity = 0;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x, parity ^= 1) {
+        mi = find_matrix(p, mi, u);
+        if (mi != prev_mi) __syncthreads();
+        prev_mi = mi;
+        const ShardDesc& m = p.m[mi];
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rsub = threadIdx.x >> tl;
+        const int64_t row = (u - m.unit_begin) * (kThreads >> tl) + rsub;
+        const int64_t nch = (m.cols + 7) >> 3;
+        double acc = 0.0;
+        if (row < m.rows) {
+            const RowScale a = row_scale(m.alpha[row]);  // plain load: written below
+            float* wr = m.w + row * m.cols;
+            float* mr = m.m_w + row * m.cols;
+            float* vr = m.v_w + row * m.cols;
+            const int64_t goff = m.g_offset + row * m.cols;
+            for (int64_t ch = lane; ch < nch; ch += tpr) {
+                const int n = VEC ? 8 : tail_n(m.cols, ch);
+                float wv[8], mv[8], vv[8], gs[8], d[8];
+                if constexpr (VEC) {
+                    load8(wr + ch * 8, wv);
+                    load8(mr + ch * 8, mv);
+                    load8(vr + ch * 8, vv);
+                } else {
+                    load8_tail(wr + ch * 8, n, wv);
+                    load8_tail(mr + ch * 8, n, mv);
+                    load8_tail(vr + ch * 8, n, vv);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) gs[i] = 0.0f;
+#pragma unroll 4
+                for (int k = 0; k < P.n_src; ++k) {
+                    uint32_t gw[4];
+                    if constexpr (VEC) load_g8(P.src[k] + goff + ch * 8, gw);
+                    else load_g8_tail(P.src[k] + goff + ch * 8, n, gw);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        gs[i] = __fadd_rn(gs[i], (i & 1) ? __uint_as_float(gw[i / 2] & 0xFFFF0000u)
+                                                         : __uint_as_float(gw[i / 2] << 16));
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) gs[i] = __fmul_rn(gs[i], P.grad_mult);
+                acc = bwd_chunk_f32<Q>(wv, gs, a, d, acc);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) wv[i] = adamw_update(P.kw, wv[i], d[i], mv[i], vv[i]);
                 if constexpr (VEC) {
@@ -1058,6 +1195,84 @@ static pq_status_t bwd_adamw_impl(int q, int32_t n, const pq_adamw_matrix_t* mat
     return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
 }
 
+template <int Q, bool VEC>
+static void launch_reduce_bwd_adamw(const ReduceBatch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    auto k = reduce_bwd_adamw_units_kernel<Q, VEC>;
+    const int64_t ctas = persistent_ctas(k, cache);
+    const unsigned grid = static_cast<unsigned>(b.b.total_units < ctas ? b.b.total_units : ctas);
+    k<<<grid, kThreads, 0, s>>>(b);
+}
+
+static pq_status_t reduce_bwd_adamw_impl(int q, int32_t n_src, const uint16_t* const* srcs,
+                                         float grad_mult, int32_t n, const pq_shard_t* sh,
+                                         const pq_adamw_t* hw, const pq_adamw_t* ha,
+                                         cudaStream_t s) {
+    if (code_bits_of(q) == 0 || n < 0 || (n > 0 && !sh)) return PQ_ERR_INVALID_ARG;
+    if (n_src < 1 || n_src > kMaxSources || !srcs) return PQ_ERR_INVALID_ARG;
+    if (!adamw_ok(hw) || !adamw_ok(ha)) return PQ_ERR_INVALID_ARG;
+    bool src_aligned = true;
+    for (int k = 0; k < n_src; ++k) {
+        if (!srcs[k]) return PQ_ERR_INVALID_ARG;
+        src_aligned = src_aligned && aligned(srcs[k], 16);
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        const pq_shard_t& m = sh[i];
+        if (m.rows < 0 || m.cols < 0 || m.g_offset < 0) return PQ_ERR_INVALID_ARG;
+        if (m.rows == 0) continue;
+        if (!m.alpha || !m.m_alpha || !m.v_alpha) return PQ_ERR_INVALID_ARG;
+        if (m.cols > 0 && (!m.w || !m.m_w || !m.v_w)) return PQ_ERR_INVALID_ARG;
+    }
+    static thread_local ReduceBatch b;
+    for (int k = 0; k < kMaxSources; ++k) b.src[k] = k < n_src ? srcs[k] : nullptr;
+    b.n_src = n_src;
+    b.grad_mult = grad_mult;
+    b.kw = adamw_consts(*hw);
+    b.ka = adamw_consts(*ha);
+    bool launched = false;
+    for (int cls = 0; cls < 2; ++cls) {
+        const bool vec = cls == 0;
+        b.b.n = 0;
+        b.b.pad_ = 0;
+        b.b.total_units = 0;
+        auto flush = [&]() {
+            if (b.b.n == 0) return;
+            launched = true;
+            dispatch_q(q, [&]<int Q>() {
+                if (vec) launch_reduce_bwd_adamw<Q, true>(b, s);
+                else launch_reduce_bwd_adamw<Q, false>(b, s);
+            });
+            b.b.n = 0;
+            b.b.total_units = 0;
+        };
+        for (int32_t i = 0; i < n; ++i) {
+            const pq_shard_t& m = sh[i];
+            if (m.rows == 0) continue;
+            const bool v = src_aligned && m.cols > 0 && m.cols % 8 == 0 && m.g_offset % 8 == 0 &&
+                           aligned(m.w, 16) && aligned(m.m_w, 16) && aligned(m.v_w, 16);
+            if (v != vec) continue;
+            if (b.b.n == kMaxBatch) flush();
+            ShardDesc& d = b.b.m[b.b.n++];
+            d.w = m.w;
+            d.alpha = m.alpha;
+            d.m_w = m.m_w;
+            d.v_w = m.v_w;
+            d.m_a = m.m_alpha;
+            d.v_a = m.v_alpha;
+            d.dalpha = m.dalpha_out;
+            d.rows = m.rows;
+            d.cols = m.cols;
+            d.g_offset = m.g_offset;
+            d.unit_begin = b.b.total_units;
+            d.grad_scale = m.grad_scale;
+            d.tpr_log2 = choose_tpr_log2(m.cols);
+            b.b.total_units += (m.rows + (kThreads >> d.tpr_log2) - 1) / (kThreads >> d.tpr_log2);
+        }
+        flush();
+    }
+    return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
+}
+
 }  // namespace pq
 
 using namespace pq;
@@ -1139,6 +1354,13 @@ pq_status_t pq_fakequant_bwd_adamw(pq_quant_t q, int32_t n, const pq_adamw_matri
                                    const pq_adamw_t* hp_w, const pq_adamw_t* hp_alpha,
                                    void* stream) {
     return bwd_adamw_impl(q, n, mats, hp_w, hp_alpha, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_reduce_bwd_adamw(pq_quant_t q, int32_t n_src, const uint16_t* const* g_sources,
+                                float grad_mult, int32_t n, const pq_shard_t* shards,
+                                const pq_adamw_t* hp_w, const pq_adamw_t* hp_alpha, void* stream) {
+    return reduce_bwd_adamw_impl(q, n_src, g_sources, grad_mult, n, shards, hp_w, hp_alpha,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 pq_status_t pq_fakequant_fwd_batch(pq_quant_t q, int32_t n, const pq_matrix_t* mats,

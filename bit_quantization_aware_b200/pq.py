@@ -67,6 +67,16 @@ class PQAdamWMatrix(ctypes.Structure):
                 ("grad_scale", ctypes.c_float)]
 
 
+class PQShard(ctypes.Structure):
+    """``pq_shard_t``: one row shard of a matrix owned by this GPU."""
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("w", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("m_w", ctypes.c_void_p), ("v_w", ctypes.c_void_p),
+                ("m_alpha", ctypes.c_void_p), ("v_alpha", ctypes.c_void_p),
+                ("dalpha_out", ctypes.c_void_p), ("g_offset", ctypes.c_int64),
+                ("grad_scale", ctypes.c_float)]
+
+
 def _declare(L):
     i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.pq_fakequant_fwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
@@ -76,6 +86,10 @@ def _declare(L):
     L.pq_fakequant_bwd_adamw.argtypes = [i32, i32, ctypes.POINTER(PQAdamWMatrix),
                                          ctypes.POINTER(PQAdamW), ctypes.POINTER(PQAdamW), p]
     L.pq_fakequant_bwd_adamw.restype = i32
+    L.pq_reduce_bwd_adamw.argtypes = [i32, i32, ctypes.POINTER(ctypes.c_void_p), f32, i32,
+                                      ctypes.POINTER(PQShard), ctypes.POINTER(PQAdamW),
+                                      ctypes.POINTER(PQAdamW), p]
+    L.pq_reduce_bwd_adamw.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_dequant_codes_batch.restype = i32
     L.pq_dequant_codes.argtypes = [i32, i64, i64, p, p, p, p]
@@ -246,6 +260,31 @@ def pq_fakequant_bwd_adamw(q, mats, hp_w, hp_alpha, stream=None):
     _check("pq_fakequant_bwd_adamw", lib().pq_fakequant_bwd_adamw(
         q, len(mats), mats, ctypes.byref(hp_w), ctypes.byref(hp_alpha),
         _stream(stream)))
+
+
+def shard_array(descs):
+    """Build a ``pq_shard_t[]`` from dicts with keys rows, cols, w, alpha,
+    m_w, v_w, m_alpha, v_alpha, dalpha (optional), g_offset, grad_scale."""
+    arr = (PQShard * len(descs))()
+    for i, d in enumerate(descs):
+        m = arr[i]
+        m.rows, m.cols = int(d["rows"]), int(d["cols"])
+        m.w, m.alpha = _ptr(d.get("w")), _ptr(d.get("alpha"))
+        m.m_w, m.v_w = _ptr(d.get("m_w")), _ptr(d.get("v_w"))
+        m.m_alpha, m.v_alpha = _ptr(d.get("m_alpha")), _ptr(d.get("v_alpha"))
+        m.dalpha_out = _ptr(d.get("dalpha"))
+        m.g_offset = int(d.get("g_offset", 0))
+        m.grad_scale = float(d.get("grad_scale", 0.0))
+    return arr
+
+
+def pq_reduce_bwd_adamw(q, g_sources, grad_mult, shards, hp_w, hp_alpha, stream=None):
+    """Reduce over replicas' bf16 gradients fused with backward + AdamW.
+    ``g_sources``: device pointers (ints) or CUDA tensors, one per replica."""
+    srcs = (ctypes.c_void_p * len(g_sources))(*[_ptr(g) for g in g_sources])
+    _check("pq_reduce_bwd_adamw", lib().pq_reduce_bwd_adamw(
+        q, len(g_sources), srcs, ctypes.c_float(grad_mult), len(shards), shards,
+        ctypes.byref(hp_w), ctypes.byref(hp_alpha), _stream(stream)))
 
 
 def pq_code_bits(q) -> int:

@@ -226,6 +226,43 @@ PQ_API pq_status_t pq_fakequant_bwd_adamw(pq_quant_t q, int32_t n,
                                           const pq_adamw_t* hp_w,
                                           const pq_adamw_t* hp_alpha, void* stream);
 
+/* One row shard of a weight matrix owned by this GPU (row-sharded,
+ * owner-computes training): the shard's rows of w, alpha and the AdamW
+ * moments live here; its upstream gradient rows sit at element offset
+ * g_offset in every replica's gradient buffer (see pq_reduce_bwd_adamw). */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    float* w;
+    float* alpha;
+    float* m_w;
+    float* v_w;
+    float* m_alpha;
+    float* v_alpha;
+    float* dalpha_out;        /* nullable */
+    int64_t g_offset;         /* elements, >= 0 */
+    float grad_scale;
+} pq_shard_t;
+
+/* Reduce-scatter fused with the backward and AdamW: for every shard, the
+ * upstream gradient of each element is the fp32 sum, in source order, of
+ * the bf16 gradients g_sources[0..n_src) (one per data-parallel replica,
+ * all with the same layout; device pointers, local or another GPU's
+ * memory reachable by peer access, e.g. symmetric memory), times
+ * grad_mult (1/n_src for a mean); then the steps of
+ * pq_fakequant_bwd_adamw run with that fp32 gradient. Each GPU calls this
+ * on its own shards after every replica's gradient is complete (the
+ * caller orders the launch after the replicas' writes, e.g. with a
+ * collective or barrier on the stream); no data crosses GPUs except these
+ * reads. 1 <= n_src <= 16. Traffic per weight: 2*n_src B gradient reads
+ * (2*(n_src-1) over NVLink) + 12 B read + 12 B written locally. */
+PQ_API pq_status_t pq_reduce_bwd_adamw(pq_quant_t q, int32_t n_src,
+                                       const uint16_t* const* g_sources,
+                                       float grad_mult, int32_t n,
+                                       const pq_shard_t* shards,
+                                       const pq_adamw_t* hp_w,
+                                       const pq_adamw_t* hp_alpha, void* stream);
+
 /* Dequantize packed codes back to bf16 weights: each stored code c (layout
  * of packed_out above) becomes bf16_rn(fl(level(c) * alpha_row)) with the
  * forward's level formulas, so the result equals the forward's

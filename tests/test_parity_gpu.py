@@ -406,7 +406,8 @@ def test_weights_on_code_and_clip_boundaries(q):
     ks = np.arange(-6, 7)
     rows = []
     for a in alphas:
-        w0 = (tg.astype(np.float32) * a).astype(np.float32)
+        with np.errstate(over="ignore"):
+            w0 = (tg.astype(np.float32) * a).astype(np.float32)
         cand = w0[:, None].view(np.int32).astype(np.int64) + np.sign(w0[:, None] + 0).astype(
             np.int64) * ks[None, :]
         tiny = np.where(ks >= 0, ks, 0x80000000 | -ks).astype(np.int64)
