@@ -420,6 +420,37 @@ int pqo_reduce_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alp
     return 0;
 }
 
+/* Weight-only low-bit matmul: Y[m][n] = sum_k X[m][k] * level(c[n][k]) *
+ * alpha[n], with X bf16 [M, K] row-major, codes packed [N, K*bits/8] as
+ * the forward writes them, levels by the forward's formulas taken as exact
+ * reals (SEQ2 (2c+1)/4, SEQ2_B (2c+1)/3, ternary 2c/3, LSQ and binary c),
+ * evaluated in double. Output fp64 [M, N]. */
+int pqo_wq_matmul(int q, int64_t m, int64_t n, int64_t k, const uint16_t* x_bf16,
+                  const uint8_t* packed, const float* alpha, double* y) {
+    pqo_params p;
+    if (pqo_get_params(q, &p) || m < 0 || n < 0 || k < 0) return -1;
+    const int64_t per_byte = 8 / p.bits;
+    const unsigned mask = (1u << p.bits) - 1u;
+    if (k % per_byte != 0) return -1;
+    for (int64_t i = 0; i < m; ++i) {
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < k; ++t) {
+                unsigned byte = packed[j * (k / per_byte) + t / per_byte];
+                unsigned f = (byte >> (p.bits * (int)(t % per_byte))) & mask;
+                int c = (f & (1u << (p.bits - 1))) ? (int)f - (1 << p.bits) : (int)f;
+                double lev;
+                if (p.is_binary || p.kh == 1.0f) lev = (double)c;            /* binary, LSQ */
+                else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / (2.0 * p.kh);  /* SEQ */
+                else lev = 2.0 * c / 3.0;                                     /* ternary */
+                acc += (double)pqo_bf16_to_float(x_bf16[i * k + t]) * lev;
+            }
+            y[i * n + j] = acc * (double)alpha[j];
+        }
+    }
+    return 0;
+}
+
 /* One AdamW step over n parameters with given gradients (for pinning the
  * update rule against a library optimizer). */
 int pqo_adamw_step(int64_t n, float* p, const float* g, float* m, float* v,

@@ -86,6 +86,8 @@ class Oracle:
                                            ctypes.c_float, p, p, p, p, ctypes.c_float,
                                            ctypes.POINTER(AdamW), ctypes.POINTER(AdamW), p]
         L.pqo_reduce_bwd_adamw.restype = ctypes.c_int
+        L.pqo_wq_matmul.argtypes = [ctypes.c_int, i64, i64, i64, p, p, p, p]
+        L.pqo_wq_matmul.restype = ctypes.c_int
         L.pqo_adamw_step.argtypes = [i64, p, p, p, p, ctypes.POINTER(AdamW)]
         L.pqo_adamw_step.restype = ctypes.c_int
         L.pqo_default_grad_scale.argtypes = [ctypes.c_int, i64]
@@ -205,6 +207,19 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle reduce_bwd_adamw rejected its arguments")
         return w, alpha, m_w, v_w, m_a, v_a, da
+
+    def wq_matmul(self, q, x_bf16, packed, alpha, k):
+        """Y = X * (alpha * levels(codes))^T in fp64; x_bf16 [M, K] bits,
+        packed [N, K*bits/8]."""
+        x = np.ascontiguousarray(x_bf16).view(np.uint16)
+        packed = np.ascontiguousarray(packed, np.uint8)
+        m, n = x.shape[0], packed.shape[0]
+        alpha = np.ascontiguousarray(alpha, np.float32).reshape(n)
+        y = np.empty((m, n), np.float64)
+        rc = self.lib.pqo_wq_matmul(q, m, n, k, _ptr(x), _ptr(packed), _ptr(alpha), _ptr(y))
+        if rc != 0:
+            raise ValueError("oracle wq_matmul rejected its arguments")
+        return y
 
     def adamw_step(self, p, g, m, v, h):
         """One AdamW step on copies of fp32 arrays; returns (p, m, v)."""

@@ -517,6 +517,36 @@ def check_reduce_sums_in_fp32(O):
     assert np.array_equal(nw[~inside], w[~inside])
 
 
+def check_wq_matmul_vs_numpy(O):
+    """The low-bit matmul equals numpy's fp64 matmul of X with weights
+    decoded from the printed level sets (codes drawn from those a forward
+    writes), for every quantizer."""
+    rng = np.random.default_rng(61)
+    for q in ALL_QUANTIZERS:
+        bits = O.code_bits(q)
+        m, n, k = 3, 5, 32
+        exact = {SEQ2: {-2: -0.75, -1: -0.25, 0: 0.25, 1: 0.75},
+                 SEQ2_B: {-2: -1.0, -1: -1 / 3, 0: 1 / 3, 1: 1.0},
+                 TERNARY: {-1: -2 / 3, 0: 0.0, 1: 2 / 3},
+                 BINARY: {-1: -1.0, 1: 1.0}}.get(q)
+        if exact is None:  # LSQ integer grid
+            lo, hi = lsq_bounds(q)
+            exact = {c: float(c) for c in range(lo, hi + 1)}
+        codes = rng.choice(sorted(exact), (n, k))
+        L = np.vectorize(exact.get)(codes).astype(np.float64)
+        per = 8 // bits
+        fields = (codes & ((1 << bits) - 1)).astype(np.uint8).reshape(n, k // per, per)
+        packed = np.zeros((n, k // per), np.uint8)
+        for i in range(per):
+            packed |= fields[:, :, i] << (bits * i)
+        alpha = rng.uniform(0.01, 2.0, n).astype(np.float32)
+        xb = torch.randn(m, k).to(torch.bfloat16)
+        x = xb.float().numpy().astype(np.float64)
+        want = x @ (L * alpha[:, None].astype(np.float64)).T
+        got = O.wq_matmul(q, xb.view(torch.int16).numpy(), packed, alpha, k)
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-12), q
+
+
 ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_nearest_level, check_binary_sign, check_lsq_textbook,
               check_overflow_example, check_ties_half_even, check_idempotence,
@@ -525,4 +555,5 @@ ALL_CHECKS = [check_level_sets, check_seq_code_domain, check_ternary_bins,
               check_pack_roundtrip, check_dequant_golden,
               check_dequant_inverts_pack, check_adamw_vs_torch,
               check_adamw_first_step, check_bwd_adamw_composes,
-              check_reduce_equals_single_source, check_reduce_sums_in_fp32]
+              check_reduce_equals_single_source, check_reduce_sums_in_fp32,
+              check_wq_matmul_vs_numpy]

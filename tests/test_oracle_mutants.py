@@ -51,6 +51,9 @@ MUTANTS = {
     "reduce_no_multiplier": ("volatile float gbar = sum * grad_mult;", "volatile float gbar = sum;"),
     "reduce_first_source_only": ("volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);",
                                  "volatile float t = pqo_bf16_to_float(g_srcs[0][r * cols + j]);"),
+    "matmul_seq_level": ("else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / (2.0 * p.kh);",
+                         "else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / 4.0;"),
+    "matmul_no_alpha": ("y[i * n + j] = acc * (double)alpha[j];", "y[i * n + j] = acc;"),
     "dequant_no_alpha": ("volatile float prod = lev * alpha;",
                          "volatile float prod = lev;"),
     "binary_sign_zero": ("c = (x >= 0.0f) ? 1 : -1;", "c = (x > 0.0f) ? 1 : -1;"),
@@ -73,6 +76,9 @@ MUTANTS = {
     "reduce_no_multiplier": ("volatile float gbar = sum * grad_mult;", "volatile float gbar = sum;"),
     "reduce_first_source_only": ("volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);",
                                  "volatile float t = pqo_bf16_to_float(g_srcs[0][r * cols + j]);"),
+    "matmul_seq_level": ("else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / (2.0 * p.kh);",
+                         "else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / 4.0;"),
+    "matmul_no_alpha": ("y[i * n + j] = acc * (double)alpha[j];", "y[i * n + j] = acc;"),
     "dequant_no_alpha": ("volatile float prod = pqo_level_of_code(&p, c) * alpha[r];",
                          "volatile float prod = pqo_level_of_code(&p, c);"),
 }
