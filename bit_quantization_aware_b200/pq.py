@@ -90,6 +90,12 @@ def _declare(L):
                                       ctypes.POINTER(PQShard), ctypes.POINTER(PQAdamW),
                                       ctypes.POINTER(PQAdamW), p]
     L.pq_reduce_bwd_adamw.restype = i32
+    L.pq_wq_gemm.argtypes = [i32, i64, i64, i64, p, p, p, p, p, i64, p]
+    L.pq_wq_gemm.restype = i32
+    L.pq_wq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]
+    L.pq_wq_gemm_workspace_bytes.restype = i64
+    L.pq_device_status.argtypes = []
+    L.pq_device_status.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_dequant_codes_batch.restype = i32
     L.pq_dequant_codes.argtypes = [i32, i64, i64, p, p, p, p]
@@ -285,6 +291,43 @@ def pq_reduce_bwd_adamw(q, g_sources, grad_mult, shards, hp_w, hp_alpha, stream=
     _check("pq_reduce_bwd_adamw", lib().pq_reduce_bwd_adamw(
         q, len(g_sources), srcs, ctypes.c_float(grad_mult), len(shards), shards,
         ctypes.byref(hp_w), ctypes.byref(hp_alpha), _stream(stream)))
+
+
+def pq_wq_gemm_workspace_bytes(q, m, n, k) -> int:
+    return int(lib().pq_wq_gemm_workspace_bytes(q, m, n, k))
+
+
+def pq_wq_gemm(q, x, packed, alpha, y_out, workspace=None, stream=None):
+    """Y = X (alpha * levels(codes))^T on the tensor cores; x bf16 [m, k],
+    packed uint8 [n, k/4], alpha fp32 [n], y_out bf16 [m, n]."""
+    m, k = x.shape
+    n = packed.shape[0]
+    if (packed.dim() != 2 or packed.shape[1] * 8 != k * pq_code_bits(q)
+            or alpha.numel() != n or tuple(y_out.shape) != (m, n)
+            or not (x.is_contiguous() and packed.is_contiguous() and y_out.is_contiguous())):
+        raise ValueError("pq_wq_gemm: shapes must be x [m, k], packed [n, k*bits/8], "
+                         "alpha [n], y_out [m, n], all contiguous")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pq_wq_gemm", lib().pq_wq_gemm(
+        q, m, n, k, _ptr(x), _ptr(packed), _ptr(alpha), _ptr(y_out), _ptr(workspace),
+        ws_bytes, _stream(stream)))
+
+
+def pq_device_status() -> int:
+    return int(lib().pq_device_status())
+
+
+def wq_gemm(q, x, packed, alpha, stream=None):
+    """Allocate the output and workspace and run pq_wq_gemm."""
+    m, k = x.shape
+    n = packed.shape[0]
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    need = pq_wq_gemm_workspace_bytes(q, m, n, k)
+    if need < 0:
+        raise PQError("pq_wq_gemm_workspace_bytes", PQ_ERR_UNSUPPORTED)
+    ws = torch.empty(need, dtype=torch.uint8, device=x.device) if need > 0 else None
+    pq_wq_gemm(q, x, packed, alpha, y, ws, stream)
+    return y
 
 
 def pq_code_bits(q) -> int:

@@ -298,6 +298,40 @@ PQ_API pq_status_t pq_dequant_codes_batch(pq_quant_t q, int32_t n,
 PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
                                      const float* alpha, float* x_out, void* stream);
 
+/* Weight-only low-bit matmul on the tensor cores (tcgen05, fp32 in TMEM):
+ *   Y[m][n] = sum_k X[m][k] * level(code[n][k]) * alpha[n]
+ * for the 2-bit quantizers (PQ_BINARY, PQ_TERNARY, PQ_SEQ2, PQ_SEQ2_B,
+ * PQ_LSQ2; others return PQ_ERR_UNSUPPORTED). The pages' 2-bit inference
+ * kernels consume packed weights in this way [P4: a 2-bit GEMM kernel on
+ * CUTLASS; P3: the accuracy-latency trade-off]; this one is built for
+ * sm_100a. The levels' integer numerators (SEQ2 2c+1, SEQ2_B 2c+1, ternary
+ * 2c, LSQ2 and binary c) are exact in bf16; the factor (1/4, 1/3, 1/3, 1,
+ * 1) times alpha scales the fp32 sums, which are rounded once to bf16.
+ *   x_bf16   bf16 [m, k], row-major, 16-byte aligned, 1 <= m <= 128
+ *   packed   codes [n, k/4] as pq_fakequant_fwd writes them, 16-byte aligned
+ *   alpha    fp32 [n]
+ *   y_bf16   bf16 [m, n], row-major, overwritten
+ *   k        a multiple of 128
+ *   workspace, workspace_bytes: device scratch of at least
+ *            pq_wq_gemm_workspace_bytes(q, m, n, k) bytes, 256-byte
+ *            aligned (may be NULL when that is 0). Split-K partial sums and
+ *            counters live there; calls that share a workspace must not
+ *            overlap on the GPU. Results are deterministic.
+ * Waits inside the kernel are bounded; pq_device_status() reports one that
+ * gave up. Traffic: k/4 B of codes per output feature (+ x, y). */
+PQ_API pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k,
+                              const uint16_t* x_bf16, const uint8_t* packed,
+                              const float* alpha, uint16_t* y_bf16, void* workspace,
+                              int64_t workspace_bytes, void* stream);
+
+/* Workspace bytes pq_wq_gemm needs for this problem (0: none), -1 for an
+ * unsupported quantizer or shape. */
+PQ_API int64_t pq_wq_gemm_workspace_bytes(pq_quant_t q, int64_t m, int64_t n, int64_t k);
+
+/* Device status of the library's bounded waits: 0 if none gave up since
+ * the last call, else nonzero (and cleared). Synchronises the device. */
+PQ_API int pq_device_status(void);
+
 /* Storage width in bits of one packed code: 2 (binary, ternary, SEQ2,
  * SEQ2_B, LSQ2) or 4 (LSQ3, LSQ4); 0 for an unknown quantizer. */
 PQ_API int pq_code_bits(pq_quant_t q);

@@ -1,0 +1,79 @@
+"""Weight-only 2-bit matmul on the tensor cores against the oracle.
+
+Y = X (alpha * levels(codes))^T: the oracle computes it in fp64; the GPU
+multiplies exact bf16 level numerators by bf16 activations with fp32
+accumulation in TMEM and rounds the scaled sums once to bf16. Tolerance:
+2^-8 of |Y| (bf16 output rounding) plus 1e-4 of sum_k |x_k * w_k|
+(accumulation error bound, far below what a wrong tile layout gives)."""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantization_aware_b200 import inputs as I
+from bit_quantization_aware_b200 import pq
+from oracle import pq_oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+Q2 = [pq.PQ_SEQ2, pq.PQ_SEQ2_B, pq.PQ_TERNARY, pq.PQ_LSQ2, pq.PQ_BINARY]
+
+
+def _case(q, m, n, k, seed):
+    w = I.normal_weights(n, k, seed=seed, stream=0, device=DEV)
+    a = I.alpha_init(w, q)
+    _, packed = pq.fakequant_fwd(q, w, a, pack=True)
+    x = I.normal_weights(m, k, seed=seed, stream=5, std=1.0, device=DEV).to(torch.bfloat16)
+    return x, packed, a
+
+
+def _check(q, x, packed, a, y):
+    k = x.shape[1]
+    xb = x.view(torch.int16).cpu().numpy()
+    pk = packed.cpu().numpy()
+    an = a.cpu().numpy()
+    ref = pq_oracle.default().wq_matmul(q, xb, pk, an, k)
+    # sum_k |x_k * w_k| (for the tolerance only) from the dequantized weights
+    wd = pq_oracle.bf16_bits_to_float(pq_oracle.dequant(q, pk, an, k)).astype(np.float64)
+    ones = np.abs(x.float().cpu().numpy().astype(np.float64)) @ np.abs(wd).T
+    got = y.float().cpu().numpy().astype(np.float64)
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ones) + 1e-30
+    err = np.abs(got - ref)
+    worst = np.unravel_index(np.argmax(err / tol), err.shape)
+    assert np.all(err <= tol), (f"q={q} shape={x.shape}x{packed.shape}: worst at {worst}: "
+                                f"gpu={got[worst]} ref={ref[worst]} tol={tol[worst]}")
+
+
+@pytest.mark.parametrize("q", Q2)
+@pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 300, 256), (16, 1024, 4096),
+                                   (33, 640, 1024), (64, 2048, 2048), (128, 256, 512),
+                                   (7, 4096, 14336)])
+def test_wq_gemm_matches_oracle(q, m, n, k):
+    x, packed, a = _case(q, m, n, k, seed=m + n + k)
+    y = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    _check(q, x, packed, a, y)
+
+
+def test_wq_gemm_deterministic_and_repeatable():
+    """Split-K reduction in a fixed order: identical bits on repeated calls
+    sharing one workspace."""
+    q = pq.PQ_SEQ2
+    x, packed, a = _case(q, 8, 4096, 16384, seed=3)
+    y1 = pq.wq_gemm(q, x, packed, a)
+    y2 = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_wq_gemm_rejects_bad_arguments():
+    q = pq.PQ_SEQ2
+    x = torch.zeros((4, 200), dtype=torch.bfloat16, device=DEV)
+    packed = torch.zeros((128, 50), dtype=torch.uint8, device=DEV)
+    a = torch.ones(128, device=DEV)
+    y = torch.empty((4, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(pq.PQError):  # k not a multiple of 128
+        pq.pq_wq_gemm(q, x, packed, a, y)
+    with pytest.raises(pq.PQError):  # 4-bit codes are not served
+        pq.pq_wq_gemm(pq.PQ_LSQ4, torch.zeros((4, 256), dtype=torch.bfloat16, device=DEV),
+                      torch.zeros((128, 128), dtype=torch.uint8, device=DEV), a, y)
