@@ -26,6 +26,8 @@
 
 #include <stdint.h>
 
+#include <atomic>
+
 #include "pq.h"
 
 namespace pqg {
@@ -489,3 +491,36 @@ int pq_device_status(void) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- no-alloc entry point
+// Split-K scratch of pq_wq_gemm_noalloc: one fixed array per device, shared
+// by every call on that device; its address is looked up once per device.
+namespace pqg {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES];
+constexpr int kNoAllocDevices = 256;
+static std::atomic<void*> g_noalloc_addr[kNoAllocDevices];
+}  // namespace pqg
+
+extern "C" pq_status_t pq_wq_gemm_noalloc(pq_quant_t q, int64_t m, int64_t n, int64_t k,
+                                          const uint16_t* x_bf16, const uint8_t* packed,
+                                          const float* alpha, uint16_t* y_bf16, void* stream) {
+    uint32_t lo, hi;
+    float factor;
+    if (!table_of(q, lo, hi, factor)) return PQ_ERR_UNSUPPORTED;
+    if (m < 1 || m > 128 || n < 1 || k < kStageK || k % kStageK || !x_bf16 || !packed || !alpha ||
+        !y_bf16)
+        return PQ_ERR_INVALID_ARG;
+    if (pq_wq_gemm_workspace_bytes(q, m, n, k) > PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES)
+        return PQ_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PQ_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocDevices) return PQ_ERR_UNSUPPORTED;
+    void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!scratch) {
+        if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch)
+            return PQ_ERR_CUDA;
+        g_noalloc_addr[dev].store(scratch, std::memory_order_release);
+    }
+    return pq_wq_gemm(q, m, n, k, x_bf16, packed, alpha, y_bf16, scratch,
+                      PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES, stream);
+}

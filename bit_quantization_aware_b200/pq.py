@@ -92,6 +92,8 @@ def _declare(L):
     L.pq_reduce_bwd_adamw.restype = i32
     L.pq_wq_gemm.argtypes = [i32, i64, i64, i64, p, p, p, p, p, i64, p]
     L.pq_wq_gemm.restype = i32
+    L.pq_wq_gemm_noalloc.argtypes = [i32, i64, i64, i64, p, p, p, p, p]
+    L.pq_wq_gemm_noalloc.restype = i32
     L.pq_wq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]
     L.pq_wq_gemm_workspace_bytes.restype = i64
     L.pq_device_status.argtypes = []
@@ -311,6 +313,31 @@ def pq_wq_gemm(q, x, packed, alpha, y_out, workspace=None, stream=None):
     _check("pq_wq_gemm", lib().pq_wq_gemm(
         q, m, n, k, _ptr(x), _ptr(packed), _ptr(alpha), _ptr(y_out), _ptr(workspace),
         ws_bytes, _stream(stream)))
+
+
+WQ_GEMM_NOALLOC_SCRATCH_BYTES = 8 << 20  # PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES
+
+
+def pq_wq_gemm_noalloc(q, x, packed, alpha, y_out, stream=None):
+    """pq_wq_gemm with the library's fixed split-K scratch: allocates nothing,
+    on the device or through torch. Problems needing more than
+    WQ_GEMM_NOALLOC_SCRATCH_BYTES of scratch are rejected; calls that may
+    overlap on the GPU race on the shared scratch."""
+    m, k = x.shape
+    n = packed.shape[0]
+    if (packed.dim() != 2 or packed.shape[1] * 8 != k * pq_code_bits(q)
+            or alpha.numel() != n or tuple(y_out.shape) != (m, n)
+            or not (x.is_contiguous() and packed.is_contiguous() and y_out.is_contiguous())):
+        raise ValueError("pq_wq_gemm_noalloc: shapes must be x [m, k], packed [n, k*bits/8], "
+                         "alpha [n], y_out [m, n], all contiguous")
+    status = lib().pq_wq_gemm_noalloc(q, m, n, k, _ptr(x), _ptr(packed), _ptr(alpha),
+                                      _ptr(y_out), _stream(stream))
+    if status == PQ_ERR_UNSUPPORTED:
+        need = pq_wq_gemm_workspace_bytes(q, m, n, k)
+        if need > WQ_GEMM_NOALLOC_SCRATCH_BYTES:
+            raise PQError(f"pq_wq_gemm_noalloc (needs {need} B of split-K scratch, over the "
+                          f"fixed {WQ_GEMM_NOALLOC_SCRATCH_BYTES} B; use pq_wq_gemm)", status)
+    _check("pq_wq_gemm_noalloc", status)
 
 
 def pq_device_status() -> int:

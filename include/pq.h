@@ -328,6 +328,38 @@ PQ_API pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k,
  * unsupported quantizer or shape. */
 PQ_API int64_t pq_wq_gemm_workspace_bytes(pq_quant_t q, int64_t m, int64_t n, int64_t k);
 
+/* Upper limit on the split-K scratch pq_wq_gemm_noalloc can use (8 MiB). */
+#define PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES (8LL << 20)
+
+/* pq_wq_gemm without a caller workspace and without allocating: the split-K
+ * scratch is a fixed PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES array in the library's
+ * device memory, one per device. The method's pages have no counterpart
+ * to this entry point; it exists for callers that cannot allocate device
+ * memory at call time: code inside an allocator's out-of-memory or free
+ * callback (it must not re-enter the allocator), serving loops whose device
+ * memory is reserved in full up front by a caching pool, and latency-bound
+ * paths that cannot take the device-wide synchronisation of cudaFree.
+ * Arguments, layouts and results are those of pq_wq_gemm (same kernel, same
+ * split plan, same bits).
+ *   Limit: a problem whose pq_wq_gemm_workspace_bytes(q, m, n, k) exceeds
+ *          PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES returns PQ_ERR_UNSUPPORTED and
+ *          enqueues nothing; call pq_wq_gemm with a workspace instead.
+ *   Set-up: the first call on each device that passes the argument checks
+ *          looks up the array's device address once (cudaGetSymbolAddress;
+ *          a failure returns PQ_ERR_CUDA and the next call retries). Make
+ *          that first call before any stream capture.
+ *   Zeroing: the split-K counters at the end of the used scratch must be
+ *          zero when the kernel starts; every call clears them on `stream`
+ *          (cudaMemsetAsync) before its launch. The partial sums need no
+ *          clearing.
+ *   Concurrency: all calls on one device share the one array, so calls that
+ *          may overlap on the GPU (unordered streams, several host threads)
+ *          race on it and give wrong results; order them on one stream.
+ * No cudaMalloc, cudaFree or other allocating routine is called. */
+PQ_API pq_status_t pq_wq_gemm_noalloc(pq_quant_t q, int64_t m, int64_t n, int64_t k,
+                                      const uint16_t* x_bf16, const uint8_t* packed,
+                                      const float* alpha, uint16_t* y_bf16, void* stream);
+
 /* Device status of the library's bounded waits: 0 if none gave up since
  * the last call, else nonzero (and cleared). Synchronises the device. */
 PQ_API int pq_device_status(void);
