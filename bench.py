@@ -31,6 +31,7 @@ METRIC = "quantizer fwd+bwd Gweights/s per step and % of B200 HBM roofline"
 UNIT = "Gweights/s"
 WORKLOAD = "llama3_8b_linear_set_seq2_fwd_ste_bwd"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -39,10 +40,14 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--op", choices=["quantizer", "dequant", "bwd_adamw"], default="quantizer",
+    p.add_argument("--op", choices=["quantizer", "dequant", "bwd_adamw", "wq_gemm"],
+                   default="quantizer",
                    help="quantizer: the forward+backward step (the headline); "
                         "dequant: packed codes -> bf16 over the same layer set; "
-                        "bwd_adamw: the backward fused with the AdamW step")
+                        "bwd_adamw: the backward fused with the AdamW step; "
+                        "wq_gemm: Y = X W^T from the packed 2-bit codes on the tensor cores")
+    p.add_argument("--m", type=int, default=16,
+                   help="wq_gemm: activation rows (tokens of a decode batch), 1..128")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -72,13 +77,26 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+QUANTIZER_KERNEL_SOURCES = ("pq.cu", "pq_quant.cuh")  # define the step's kernels
+
+
 def kernel_source_hash():
+    """Hash of the sources that define the quantizer step's kernels."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantization_aware_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in QUANTIZER_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -632,6 +650,112 @@ def run_bwd_adamw(args):
     return 0
 
 
+def run_wq_gemm(args):
+    """Weight-only 2-bit matmul Y = X (alpha * levels)^T for every matrix of
+    the Llama-3-8B-shaped set (224 launches per step, captured in one CUDA
+    graph; the 1.75 GB of codes are far larger than L2, so every launch
+    reads its codes from HBM), 1 GPU, X of --m rows. Beside it, for
+    context, cuBLAS (torch.matmul) on the dense bf16 dequantized weights,
+    also graph-captured. Prints one JSON line."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.step import QuantStep
+
+    torch.cuda.set_device(0)
+    dev = "cuda:0"
+    m = args.m
+    q = pq.PQ_SEQ2
+    step = QuantStep(I.llama3_8b_set(), q, device=dev, pack=True)
+    step.generate(seed=3)
+    step.fwd_all()
+    torch.cuda.synchronize()
+    ks = sorted({b.m.cols for b in step.bufs})
+    ns = sorted({b.m.rows for b in step.bufs})
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    xs = {k: torch.randn((m, k), generator=gen, device=dev).to(torch.bfloat16) for k in ks}
+    ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in ns}
+    ys_ref = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in ns}
+    need = max(pq.pq_wq_gemm_workspace_bytes(q, m, b.m.rows, b.m.cols) for b in step.bufs)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+
+    def ours():
+        for b in step.bufs:
+            pq.pq_wq_gemm(q, xs[b.m.cols], b.packed, b.alpha, ys[b.m.rows], ws)
+
+    def dense():
+        for b in step.bufs:
+            torch.matmul(xs[b.m.cols], b.wq.t(), out=ys_ref[b.m.rows])
+
+    def timed(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(max(args.warmup, 3)):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps, g
+
+    ms, g_ours = timed(ours)
+    ms_dense, g_dense = timed(dense)
+    assert pq.pq_device_status() == 0
+    # the last matrix of the set, both ways (same weights, fp32 sums)
+    b = step.bufs[-1]
+    yo, yr = ys[b.m.rows].float(), ys_ref[b.m.rows].float()
+    rel = float((yo - yr).abs().max() / yr.abs().max().clamp_min(1e-30))
+    del g_ours, g_dense
+
+    weights = step.weights
+    bytes_step = sum(b.m.numel // 4 + b.m.rows * 4 + m * b.m.cols * 2 + m * b.m.rows * 2
+                     for b in step.bufs)
+    flops_step = 2 * m * weights
+    hbm, hbm_kind = measured_peaks()
+    tflops, tf_kind = measured_tensor_peak()
+    t_hbm = bytes_step / (hbm * 1e9)
+    t_tc = flops_step / (tflops * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": bytes_step / (ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s", "peak_source": f"{hbm_kind} hbm_gbs",
+                "algorithmic_bytes_per_step": bytes_step}
+    else:
+        roof = {"bound": "tensor", "achieved": flops_step / (ms * 1e-3) / 1e12, "peak": tflops,
+                "unit": "TFLOP/s", "peak_source": f"{tf_kind} bf16_tflops (burst)",
+                "algorithmic_flops_per_step": flops_step}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "pqg::wq_gemm_kernel<NT> (tcgen05.mma kind::f16, TMEM accumulator)"
+    print(json.dumps({
+        "metric": "weight-only 2-bit matmul Gweights/s", "op": "wq_gemm",
+        "value": weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16 x 2-bit codes, f32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": f"llama3_8b_linear_set_seq2_wq_gemm_m{m}", "m": m,
+                   "weights": weights, "launches_per_step": len(step.bufs),
+                   "l2": "codes 1.75 GB per step, larger than L2"},
+        "roofline": roof,
+        "tflops": flops_step / (ms * 1e-3) / 1e12,
+        "cublas_bf16_dense": {"ms_per_step": ms_dense, "speedup_of_ours": ms_dense / ms,
+                              "what": "torch.matmul(x, W_bf16.t()) per matrix, CUDA graph",
+                              "max_rel_diff_last_matrix": rel}}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -640,6 +764,8 @@ def main():
         return run_dequant(args)
     if args.op == "bwd_adamw":
         return run_bwd_adamw(args)
+    if args.op == "wq_gemm":
+        return run_wq_gemm(args)
     return run_ours(args)
 
 
