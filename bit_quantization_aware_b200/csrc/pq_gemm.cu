@@ -1,60 +1,87 @@
-// Weight-only low-bit matmul on sm_100a tensor cores (tcgen05 + TMEM).
+// Weight-only low-bit matmul on sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 //   Y[m][n] = sum_k X[m][k] * level(code[n][k]) * alpha[n]
 //
 // X: bf16 [M, K] activations (M <= 128, a decode-sized batch); codes: the
 // forward's packed 2-bit codes [N, K/4]; alpha: fp32 [N]; Y: bf16 [M, N].
-// Every 2-bit level is a small integer numerator times a per-quantizer
-// factor (SEQ2 (2c+1)/4, SEQ2_B (2c+1)/3, ternary 2c/3, LSQ2 and binary c),
-// so the weight tile is decoded to exact bf16 numerators and the factor
-// times alpha scales the fp32 accumulator in the epilogue.
 //
-// The weights are the wide operand: each CTA tile is 128 output features
-// (the MMA's M) by NT batch columns (the MMA's N, NT >= M), accumulated in
-// TMEM over K. A persistent CTA of 4 warps walks (feature block, K segment)
-// units; per pipeline stage of 128 K, every thread decodes its feature row's
-// 128 codes (32 bytes) into the 128B-swizzled K-major shared-memory layout
-// through a byte-permute table, the activations arrive by cp.async, and
-// thread 0 issues 8 tcgen05.mma (K = 16 each) and commits them to the
-// stage's mbarrier. Split-K partial sums go to a caller workspace; the last
-// CTA of a feature block adds them in segment order (deterministic).
+// Decoding. Every 2-bit level is affine in the code's offset-binary field
+// f' = f xor 2 (c = f' - 2): numerator = A f' + B with (A, B) = (2, -3) for
+// SEQ2 and SEQ2_B (2c + 1), (2, -4) for ternary (2c), (1, -2) for LSQ2 and
+// binary (c). So a weight is decoded to the bf16 value 1 + f'/4, built by
+// placing f' in the top two mantissa bits of 1.0 (one shift and one
+// three-input logic op per two weights), and the tensor cores accumulate
+//   D[r][j] = sum_k x[j][k] (1 + f'/4) = Sx[j] + (1/4) sum_k x[j][k] f'
+// in fp32, with Sx[j] = sum_k x[j][k]. A 128-row tile holds 127 weight rows
+// and one row of ones, whose accumulator is Sx itself, so
+//   Y = alpha * factor * (4A D + (B - 4A) Sx) = alpha * (P D + Q Sx).
+// The two weights decoded together are the code word's fields j and j + 8
+// (16 bits apart), so the K order inside every group of 16 is interleaved
+// (j, j + 8); the activation tile is permuted the same way in shared memory.
 //
-// Every mbarrier wait is bounded: on giving up, the kernel records a device
-// status, waits (bounded) for its own MMAs, frees its TMEM and returns.
+// Operands. A (decoded weights) lives in TMEM (tcgen05.st from the decode
+// warps; tcgen05.mma reads it there, with no shared-memory round trip);
+// B (activations) arrives by TMA in the 128B-swizzled K-major layout the
+// MMA reads; the codes arrive by TMA, 512 K (128 B) per row per chunk, in a
+// ring several chunks deep so that enough bytes are in flight per SM.
+//
+// Work split. The (row block, code chunk) items are cut into equal
+// contiguous ranges, one per CTA (stream-K); a range covers whole blocks and
+// at most two partial blocks. A partial block's pieces go to a caller
+// workspace and the last CTA to finish the block adds them in K order
+// (deterministic).
+//
+// Roles (19 warps): 8 decode warps (TMEM lane quarter = warp % 4, K half =
+// warp / 4), 4 epilogue warps, 4 activation permuters, one codes producer,
+// one activation producer, one MMA issuer. The activation ring is deeper
+// than the A ring and has its own barriers, so decoding never waits on it. Every mbarrier wait is bounded: on giving up the kernel
+// records a device status and an abort flag that ends every role's loop,
+// waits (bounded) for its own copies and MMAs in flight, frees its TMEM and
+// returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "pq.h"
 
 namespace pqg {
 
-constexpr int kThreads = 128;         // 4 warps = the 128 TMEM lanes
-constexpr int kBlockN = 128;          // features per tile (MMA M)
-constexpr int kStageK = 128;          // K per stage (two 64-wide swizzle atoms)
-constexpr int kStages = 3;
+constexpr int kFeat = 127;             // weight rows per tile; TMEM lane 127 = ones
+constexpr int kStageK = 256;           // K per MMA stage: 128 TMEM columns of A, 16 MMAs
+constexpr int kChunkK = 512;           // K per codes chunk: 128 B per row
+constexpr int kStagesPerChunk = kChunkK / kStageK;
+constexpr int kMinK = 128;             // K granularity of the problem
+constexpr int kDecWarps = 8;           // warps 0..7
+constexpr int kEpiWarp0 = 8;           // warps 8..11
+constexpr int kPermWarp0 = 12;         // warps 12..15
+constexpr int kPermWarps = 4;
+constexpr int kCodesWarp = 16, kXWarp = 17, kMmaWarp = 18;
+constexpr int kThreads = 19 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kCodesSlotBytes = 16384;
+constexpr uint32_t kCodesTx = kFeat * 128;
 constexpr uint32_t kMaxSpins = 1u << 22;
+constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
 
 // nonzero after a bounded wait gave up (read by pq_device_status)
 __device__ int g_status = 0;
 
 struct GemmParams {
-    const uint16_t* x;      // [M, K] bf16
-    const uint8_t* codes;   // [N, K/4]
-    const float* alpha;     // [N]
-    uint16_t* y;            // [M, N] bf16
-    float* partial;         // [S, M, N] fp32 (S > 1)
-    int* counters;          // [ceil(N/128)] (S > 1), zero on entry
+    const float* alpha;  // [N]
+    uint16_t* y;         // [M, N] bf16
+    float* partial;      // [2 * grid, kFeat, m4] fp32 (partial blocks only)
+    int* counters;       // [nblocks], zero on entry (partial blocks only)
     int64_t m, n, k;
-    int64_t kseg;           // K per segment (multiple of kStageK)
-    int32_t splits;         // S
-    int32_t nblocks;
-    uint32_t table_lo;      // bf16 numerators of fields 0..3, low bytes
-    uint32_t table_hi;      // ... high bytes
-    float factor;           // level = numerator * factor
+    int64_t m4;          // m rounded up to a multiple of 4 (partial row length)
+    int64_t nblocks, nchunks, items;
+    int32_t grid;
+    float P, Q;          // y = alpha * (P * D + Q * Sx)
 };
 
 // ----------------------------------------------------------- primitives
@@ -74,16 +101,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 // K-major, M = 128, N = nt.
 __host__ __device__ constexpr uint32_t idesc_bf16(int nt) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) |
-           (static_cast<uint32_t>(kBlockN >> 4) << 24);
+           (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
+// D (TMEM) (+)= A (TMEM) * B (shared memory)^T
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -93,25 +121,78 @@ __device__ __forceinline__ void mma_commit(uint32_t mbar) {
                  : "memory");
 }
 
+// NK MMAs of K = 16 over one stage: A columns advance by 8, the B
+// descriptor start address by 32 B inside a 64-K swizzle atom and by one
+// atom (ATOM_B bytes) every 4 MMAs.
+template <int NK, int ATOM_B>
+__device__ __forceinline__ void issue_stage(uint32_t d, uint32_t a, uint64_t b0, uint32_t idesc,
+                                            uint32_t acc0) {
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk)
+        mma_ts(d, a + 8u * kk, b0 + static_cast<uint64_t>(((kk >> 2) * ATOM_B + (kk & 3) * 32) >> 4),
+               idesc, kk == 0 ? acc0 : 1u);
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
 
-// Bounded wait for the given phase parity; false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait for the phase of the given parity (one thread). Gives up
+// early when another role raised the abort flag; raises it (and the device
+// status) when the spin limit is reached.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
     for (uint32_t i = 0; i < kMaxSpins; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(mbar), "r"(parity)
-            : "memory");
-        if (done) return true;
+        if (mbar_try(mbar, parity)) return true;
+        if ((i & 63u) == 63u && *abort) return false;
     }
+    *abort = 1;
     atomicExch(&g_status, 1);
     return false;
+}
+
+// The same, taken by lane 0 for the whole warp (the result is warp-uniform,
+// so the warp stays converged for the .sync.aligned tensor-memory ops).
+__device__ __forceinline__ bool warp_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(mbar, parity, abort) ? 1 : 0;
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+// Bounded wait that ignores the abort flag (draining on the way out).
+__device__ __forceinline__ void mbar_drain(uint32_t mbar, uint32_t parity) {
+    for (uint32_t i = 0; i < kMaxSpins; ++i)
+        if (mbar_try(mbar, parity)) return;
+    atomicExch(&g_status, 1);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t mbar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(x), "r"(y)
+        : "memory");
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -123,10 +204,8 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, uint32_t bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
-                 : "memory");
+__device__ __forceinline__ void epi_sync() {  // the 4 epilogue warps
+    asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 // 16 fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
@@ -144,56 +223,201 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Fields of byte b (4 codes of 2 bits) moved to bits 0, 8, 16, 24.
-__device__ __forceinline__ uint32_t spread2(uint32_t b) {
-    return ((b & 0x33u) * 0x1001u | (b & 0xCCu) * 0x40040u) & 0x03030303u;
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
 }
 
-// 8 codes (16 bits) -> 8 bf16 numerators (4 words) via the byte-planar table.
-__device__ __forceinline__ uint4 decode8(uint32_t h16, uint32_t lo, uint32_t hi) {
-    const uint32_t t0 = spread2(h16 & 0xFFu);
-    const uint32_t t1 = spread2(h16 >> 8);
-    uint4 o;
-    o.x = __byte_perm(lo, hi, t0 * 0x11u + 0x4040u);
-    o.y = __byte_perm(lo, hi, (t0 >> 16) * 0x11u + 0x4040u);
-    o.z = __byte_perm(lo, hi, t1 * 0x11u + 0x4040u);
-    o.w = __byte_perm(lo, hi, (t1 >> 16) * 0x11u + 0x4040u);
-    return o;
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
+                 "r"(w)
+                 : "memory");
+}
+
+// Fields j and j + 8 of a code word (two's complement, first column in the
+// lowest bits) as two bf16 values 1 + f'/4 (low half: field j), with
+// f' = f xor 2: the field lands in mantissa bits 5-6 of 1.0 and its sign
+// bit is flipped there.
+template <int J>
+__device__ __forceinline__ uint32_t pair_of(uint32_t w) {
+    const uint32_t s = J < 3 ? (w << (5 - 2 * J)) : (w >> (2 * J - 5));
+    return ((s & 0x00600060u) ^ 0x00400040u) | kOnes;
+}
+
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t* v) {
+    v[0] = pair_of<0>(w);
+    v[1] = pair_of<1>(w);
+    v[2] = pair_of<2>(w);
+    v[3] = pair_of<3>(w);
+    v[4] = pair_of<4>(w);
+    v[5] = pair_of<5>(w);
+    v[6] = pair_of<6>(w);
+    v[7] = pair_of<7>(w);
+}
+
+// Position in a ring of N mbarrier-guarded slots: slot index and the parity
+// of its current phase. A wait on parity (phase ^ 1) passes at once on a
+// fresh barrier, so a producer's first round needs no special case.
+template <int N>
+struct Ring {
+    uint32_t idx = 0, phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++idx == N) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// Bounded wait for the last min(issued, N) loads of a full-barrier ring.
+template <int N>
+__device__ __forceinline__ void drain_ring(uint32_t bar0, Ring<N> r, uint32_t issued) {
+    const uint32_t n = issued < static_cast<uint32_t>(N) ? issued : static_cast<uint32_t>(N);
+    for (uint32_t j = 0; j < n; ++j) {
+        if (r.idx == 0) {
+            r.idx = N;
+            r.phase ^= 1u;
+        }
+        --r.idx;
+        mbar_drain(bar0 + 8u * r.idx, r.phase);
+    }
+}
+
+// One piece of a CTA's range: row block b, code chunks [c0, c1).
+struct Piece {
+    int64_t b, c0, c1;
+};
+
+// Items [s, e) of CTA g (item = block * nchunks + chunk).
+__device__ __forceinline__ int64_t range_start(const GemmParams& p, int64_t g) {
+    return g * p.items / p.grid;
+}
+
+__device__ __forceinline__ bool next_piece(const GemmParams& p, int64_t& s, int64_t e, Piece& pc) {
+    if (s >= e) return false;
+    const int64_t b = s / p.nchunks;
+    const int64_t blk_end = (b + 1) * p.nchunks;
+    const int64_t pe = e < blk_end ? e : blk_end;
+    pc.b = b;
+    pc.c0 = s - b * p.nchunks;
+    pc.c1 = pe - b * p.nchunks;
+    s = pe;
+    return true;
+}
+
+// MMA stages of code chunk c (the last chunk of a row may be short).
+__device__ __forceinline__ int stages_of_chunk(const GemmParams& p, int64_t c) {
+    const int64_t rest = (p.k - c * kChunkK + kStageK - 1) / kStageK;
+    return rest < kStagesPerChunk ? static_cast<int>(rest) : kStagesPerChunk;
+}
+
+// K of the stage starting at k0: kStageK, or 128 for a short tail.
+__device__ __forceinline__ int stage_k(const GemmParams& p, int64_t k0) {
+    return p.k - k0 < kStageK ? static_cast<int>(p.k - k0) : kStageK;
+}
+
+// CTA whose range holds item i: the largest g with range_start(g) <= i.
+__device__ __forceinline__ int64_t cta_of_item(const GemmParams& p, int64_t i) {
+    return ((i + 1) * p.grid + p.items - 1) / p.items - 1;
 }
 
 template <int NT>
 struct Layout {
-    static constexpr int kAtomA = kBlockN * 128;        // 128 rows x 128 B
-    static constexpr int kAtomB = NT * 128;             // NT rows x 128 B
-    static constexpr int kStage = 2 * kAtomA + 2 * kAtomB;
-    static constexpr int kBarriers = kStages * kStage;  // offset of the barriers
-    static constexpr int kBytes = kBarriers + 256 + 1024;  // + barriers, slack for alignment
-    static constexpr uint32_t kCols = NT < 32 ? 32 : NT;   // TMEM columns (power of two)
+    static constexpr int kCodesSlots = NT == 16 ? 8 : NT == 32 ? 6 : 4;
+    static constexpr int kASlots = NT == 128 ? 2 : 3;           // A in TMEM, 128 columns each
+    static constexpr int kBSlots = NT <= 32 ? 6 : NT == 64 ? 4 : 2;
+    static_assert(kBSlots <= 2 * kASlots, "the activation producer reads stage completions "
+                                         "from the A ring; deeper B rings would alias phases");
+    static constexpr uint32_t kAccStride = NT == 128 ? 128 : 64;  // two accumulators
+    static constexpr uint32_t kACol0 = 2 * kAccStride;
+    static constexpr int kAtomB = NT * 128;             // NT rows x 128 B (64 K)
+    static constexpr int kBSlot = 4 * kAtomB;           // 256 K
+    static constexpr int kCodesOff = 0;
+    static constexpr int kBOff = kCodesSlots * kCodesSlotBytes;
+    static constexpr int kBarOff = kBOff + kBSlots * kBSlot;
+    // cfull, cempty [codes slots]; xfull [B slots]; afull, aempty [A
+    // slots]; accfull, accempty [2]; drain
+    static constexpr int kNumBars = 2 * kCodesSlots + kBSlots + 2 * kASlots + 4 + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort, last, ok
+    static constexpr int kSxOff = kMiscOff + 16;              // 128 floats
+    static constexpr int kBytes = kSxOff + 128 * 4 + 1024;    // + alignment slack
+    static_assert(kACol0 + 128 * kASlots <= kTmemCols, "TMEM columns");
 };
 
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+    return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
+                       __fadd_rn(a.w, b.w));
+}
+
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+    wq_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes,
+                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ GemmParams p) {
     using L = Layout<NT>;
+    constexpr int SC = L::kCodesSlots, SA = L::kASlots, SB = L::kBSlots;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarriers);  // kStages + 1
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kStages + 1);
-    int* flags = reinterpret_cast<int*>(tmem_slot + 1);  // [0] ok, [1] last-CTA
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t b_cfull = sbase + L::kBarOff, b_cempty = b_cfull + 8u * SC;
+    const uint32_t b_xfull = b_cempty + 8u * SC, b_afull = b_xfull + 8u * SB;
+    const uint32_t b_aempty = b_afull + 8u * SA, b_accfull = b_aempty + 8u * SA;
+    const uint32_t b_accempty = b_accfull + 16u, b_drain = b_accempty + 16u;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+    volatile int* epi_ok = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 12);
+    float* sx = reinterpret_cast<float*>(smem + L::kSxOff);
+
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const uint32_t sbase = smem_u32(smem);
+    const int lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s <= kStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        for (int s = 0; s < SC; ++s) {
+            mbar_init(b_cfull + 8u * s, 1);
+            mbar_init(b_cempty + 8u * s, kDecWarps);
+        }
+        for (int s = 0; s < SB; ++s) mbar_init(b_xfull + 8u * s, 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(b_afull + 8u * s, kDecWarps + kPermWarps);
+            mbar_init(b_aempty + 8u * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_accfull + 8u * b, 1);
+            mbar_init(b_accempty + 8u * b, 4);
+        }
+        mbar_init(b_drain, 1);
+        *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        flags[0] = 1;
+    }
+    if (tid == kCodesWarp * 32) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_codes))
+                     : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x))
+                     : "memory");
     }
     __syncwarp();
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(L::kCols)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -201,154 +425,346 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    constexpr uint32_t idesc = idesc_bf16(NT);
+    const int64_t rs = range_start(p, blockIdx.x), re = range_start(p, blockIdx.x + 1);
 
-    const int64_t kq = p.k >> 2;  // code bytes per feature row
-    int64_t it = 0;               // stages issued by this CTA (for the parities)
-    uint32_t done_phase = 0;
-    bool ok = true;
-    const int64_t units = static_cast<int64_t>(p.nblocks) * p.splits;
-    for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int nb = static_cast<int>(u / p.splits);
-        const int ks = static_cast<int>(u % p.splits);
-        const int64_t n0 = static_cast<int64_t>(nb) * kBlockN;
-        const int64_t kb = ks * p.kseg;
-        const int64_t ke = (kb + p.kseg) < p.k ? (kb + p.kseg) : p.k;
-        const int64_t nsteps = (ke - kb) / kStageK;
-        const int64_t row = n0 + tid;  // this thread's feature row
-        const uint8_t* crow = p.codes + (row < p.n ? row : 0) * kq;
-        for (int64_t step = 0; step < nsteps; ++step, ++it) {
-            const int s = static_cast<int>(it % kStages);
-            if (it >= kStages) {  // stage s free: its previous MMAs are done
-                if (tid == 0 && !mbar_wait(smem_u32(&bars[s]), ((it / kStages) - 1) & 1))
-                    flags[0] = 0;
-                __syncthreads();
-                if (!flags[0]) {
+    if (warp == kCodesWarp) {
+        // ---------------------------------------------- codes producer
+        if (lane == 0) {
+            Ring<SC> cr;
+            uint32_t issued = 0;
+            int64_t s = rs;
+            Piece pc;
+            bool ok = true;
+            while (ok && next_piece(p, s, re, pc)) {
+                for (int64_t c = pc.c0; c < pc.c1; ++c) {
+                    if (!mbar_wait(b_cempty + 8u * cr.idx, cr.phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(b_cfull + 8u * cr.idx, kCodesTx);
+                    tma_load_2d(sbase + L::kCodesOff + cr.idx * kCodesSlotBytes, &tm_codes,
+                                b_cfull + 8u * cr.idx, static_cast<int32_t>(c * (kChunkK / 4)),
+                                static_cast<int32_t>(pc.b * kFeat));
+                    cr.next();
+                    ++issued;
+                }
+            }
+            // the loads still in flight land before the CTA may exit
+            drain_ring(b_cfull, cr, issued);
+        }
+    } else if (warp == kXWarp) {
+        // ---------------------------------------- activation producer
+        if (lane == 0) {
+            Ring<SB> xr;
+            Ring<SA> er;  // A-ring position of stage gs - SB
+            uint32_t gs = 0;
+            int64_t s = rs;
+            Piece pc;
+            bool ok = true;
+            while (ok && next_piece(p, s, re, pc)) {
+                for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
+                    const int ns = stages_of_chunk(p, c);
+                    for (int i = 0; i < ns; ++i, ++gs) {
+                        if (gs >= static_cast<uint32_t>(SB)) {  // B slot free: stage gs - SB done
+                            if (!mbar_wait(b_aempty + 8u * er.idx, er.phase, abort)) {
+                                ok = false;
+                                break;
+                            }
+                            er.next();
+                        }
+                        const int64_t k0 = c * kChunkK + i * kStageK;
+                        const int boxes = stage_k(p, k0) / 64;
+                        const uint32_t dst = sbase + L::kBOff + xr.idx * L::kBSlot;
+                        mbar_expect_tx(b_xfull + 8u * xr.idx, static_cast<uint32_t>(boxes * NT * 128));
+                        for (int bx = 0; bx < boxes; ++bx)
+                            tma_load_2d(dst + bx * L::kAtomB, &tm_x, b_xfull + 8u * xr.idx,
+                                        static_cast<int32_t>(k0 + 64 * bx), 0);
+                        xr.next();
+                    }
+                }
+            }
+            drain_ring(b_xfull, xr, gs);
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------- MMA issuer
+        // The issuing thread blocks on every tcgen05.mma, so its loop keeps
+        // bookkeeping to a few 32-bit operations between MMAs.
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(NT);
+            Ring<SA> ar;
+            Ring<SB> br;
+            Ring<2> accr;
+            int64_t s = rs;
+            Piece pc;
+            bool ok = true;
+            while (ok && next_piece(p, s, re, pc)) {
+                if (!mbar_wait(b_accempty + 8u * accr.idx, accr.phase ^ 1u, abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + L::kAccStride * accr.idx;
+                uint32_t acc0 = 0;
+                for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
+                    const int ns = stages_of_chunk(p, c);
+                    const bool short_tail = stage_k(p, c * kChunkK + (ns - 1) * kStageK) != kStageK;
+                    for (int i = 0; i < ns; ++i) {
+                        if (!mbar_wait(b_afull + 8u * ar.idx, ar.phase, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a = tmem + L::kACol0 + 128u * ar.idx;
+                        const uint64_t b0 = sw128_desc(sbase + L::kBOff + br.idx * L::kBSlot);
+                        if (short_tail && i == ns - 1)
+                            issue_stage<8, L::kAtomB>(d, a, b0, idesc, acc0);
+                        else
+                            issue_stage<16, L::kAtomB>(d, a, b0, idesc, acc0);
+                        acc0 = 1;
+                        mma_commit(b_aempty + 8u * ar.idx);
+                        ar.next();
+                        br.next();
+                    }
+                }
+                if (!ok) break;
+                mma_commit(b_accfull + 8u * accr.idx);
+                accr.next();
+            }
+            // every MMA issued by this thread completes before TMEM is freed
+            mma_commit(b_drain);
+            mbar_drain(b_drain, 0);
+        }
+    } else if (warp < kDecWarps) {
+        // ------------------------------------------------------ decoders
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;  // TMEM lane = A row
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        Ring<SC> cr;
+        Ring<SA> ar;
+        int64_t s = rs;
+        Piece pc;
+        bool ok = true;
+        while (ok && next_piece(p, s, re, pc)) {
+            for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
+                if (!warp_wait(b_cfull + 8u * cr.idx, cr.phase, abort)) {
                     ok = false;
                     break;
                 }
-            }
-            const int64_t k0 = kb + step * kStageK;
-            const uint32_t a_base = sbase + s * L::kStage;
-            const uint32_t b_base = a_base + 2 * L::kAtomA;
-            // activations: NT rows x 256 B, rows >= M zero-filled
+                const uint32_t crow = sbase + L::kCodesOff + cr.idx * kCodesSlotBytes + r * 128;
+                const int ns = stages_of_chunk(p, c);
+                for (int i = 0; i < ns; ++i) {
+                    // this warp's 128 K of the stage exist unless the stage is a short tail
+                    const bool mine = stage_k(p, c * kChunkK + i * kStageK) > 128 * half;
+                    // 128 K of this row (32 code bytes) -> 64 TMEM columns, 64 K at a time
+                    const int ch = 4 * i + 2 * half;
+                    uint4 cw = make_uint4(0, 0, 0, 0);
+                    uint32_t v[32];
+                    if (mine) {
+                        cw = lds128(crow + ((ch ^ (r & 7)) << 4));
+                        decode_word(cw.x, v);
+                        decode_word(cw.y, v + 8);
+                        decode_word(cw.z, v + 16);
+                        decode_word(cw.w, v + 24);
+                        cw = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
+                    }
+                    if (!warp_wait(b_aempty + 8u * ar.idx, ar.phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (mine) {
+                        tc_fence_after();
+                        const uint32_t col = tmem + lane_addr + L::kACol0 + 128u * ar.idx + 64u * half;
+                        if (r == kFeat) {
 #pragma unroll
-            for (int i = 0; i < NT / 8; ++i) {
-                const int chunk = tid + i * kThreads;  // 0 .. NT*16-1
-                const int r = chunk >> 4;              // batch row
-                const int c = chunk & 15;              // 16-byte chunk of 256 B
-                const int atom = c >> 3, cc = c & 7;
-                const uint32_t dst = b_base + atom * L::kAtomB + r * 128 + ((cc ^ (r & 7)) << 4);
-                const bool valid = r < p.m;
-                const uint16_t* src = p.x + (valid ? r : 0) * p.k + k0 + c * 8;
-                cp_async16_zfill(dst, src, valid ? 16u : 0u);
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-            // weights: this thread's row, 128 codes -> 16 chunks of 8 bf16
-            uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-            if (row < p.n) {
-                const uint4* src = reinterpret_cast<const uint4*>(crow + (k0 >> 2));
-                w0 = __ldcs(src);
-                w1 = __ldcs(src + 1);
-            }
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                            for (int j = 0; j < 32; ++j) v[j] = kOnes;
+                        }
+                        tmem_st32(col, v);
+                        decode_word(cw.x, v);
+                        decode_word(cw.y, v + 8);
+                        decode_word(cw.z, v + 16);
+                        decode_word(cw.w, v + 24);
+                        if (r == kFeat) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {  // chunk j: codes 8j .. 8j+7
-                const uint32_t h16 = (words[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-                const uint4 v = decode8(h16, p.table_lo, p.table_hi);
-                const int atom = j >> 3, cc = j & 7;
-                const uint32_t dst = a_base + atom * L::kAtomA + tid * 128 + ((cc ^ (tid & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x),
-                             "r"(v.y), "r"(v.z), "r"(v.w)
-                             : "memory");
-            }
-            asm volatile("cp.async.wait_all;" ::: "memory");
-            fence_async_smem();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kStageK / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;  // 16 bf16 of K inside the atom
-                    const uint64_t ad = sw128_desc(a_base + (kk >> 2) * L::kAtomA + off);
-                    const uint64_t bd = sw128_desc(b_base + (kk >> 2) * L::kAtomB + off);
-                    mma_bf16(tmem, ad, bd, idesc, (step > 0 || kk > 0) ? 1u : 0u);
+                            for (int j = 0; j < 32; ++j) v[j] = kOnes;
+                        }
+                        tmem_st32(col + 32u, v);
+                        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                        tc_fence_before();
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_afull + 8u * ar.idx);
+                    ar.next();
                 }
-                mma_commit(smem_u32(&bars[s]));
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(b_cempty + 8u * cr.idx);
+                cr.next();
             }
         }
-        if (!ok) break;
-        // all MMAs of this unit done
-        if (tid == 0) {
-            mma_commit(smem_u32(&bars[kStages]));
-            if (!mbar_wait(smem_u32(&bars[kStages]), done_phase)) flags[0] = 0;
+    } else if (warp >= kPermWarp0 && warp < kPermWarp0 + kPermWarps) {
+        // ------------------- activation permuters: each group of 16 K -> (j, j + 8)
+        const int ptid = tid - kPermWarp0 * 32;
+        Ring<SB> br;
+        Ring<SA> ar;
+        int64_t s = rs;
+        Piece pc;
+        bool ok = true;
+        while (ok && next_piece(p, s, re, pc)) {
+            for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
+                const int ns = stages_of_chunk(p, c);
+                for (int i = 0; i < ns; ++i) {
+                    if (!warp_wait(b_xfull + 8u * br.idx, br.phase, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const int groups = stage_k(p, c * kChunkK + i * kStageK) / 16;
+                    const uint32_t bslot = sbase + L::kBOff + br.idx * L::kBSlot;
+                    for (int it = ptid; it < NT * groups; it += kPermWarps * 32) {
+                        const int bro = it % NT, g = it / NT;
+                        const int ch = 2 * (g & 3);
+                        const uint32_t rowa = bslot + (g >> 2) * L::kAtomB + bro * 128;
+                        const uint32_t a0 = rowa + ((ch ^ (bro & 7)) << 4);
+                        const uint32_t a1 = rowa + (((ch + 1) ^ (bro & 7)) << 4);
+                        const uint4 A = lds128(a0), B = lds128(a1);
+                        sts128(a0, __byte_perm(A.x, B.x, 0x5410), __byte_perm(A.x, B.x, 0x7632),
+                               __byte_perm(A.y, B.y, 0x5410), __byte_perm(A.y, B.y, 0x7632));
+                        sts128(a1, __byte_perm(A.z, B.z, 0x5410), __byte_perm(A.z, B.z, 0x7632),
+                               __byte_perm(A.w, B.w, 0x5410), __byte_perm(A.w, B.w, 0x7632));
+                    }
+                    fence_async_smem();
+                    // arrive only once this A-ring phase is the one for this stage
+                    if (!warp_wait(b_aempty + 8u * ar.idx, ar.phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_afull + 8u * ar.idx);
+                    ar.next();
+                    br.next();
+                }
+            }
         }
-        done_phase ^= 1;
-        __syncthreads();
-        if (!flags[0]) {
-            ok = false;
-            break;
-        }
-        tc_fence_after();
-        // epilogue: thread = feature row, NT columns = batch rows
-        const float scale = row < p.n ? __fmul_rn(__ldg(p.alpha + row), p.factor) : 0.0f;
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ------------------------------------------------------ epilogue
+        const int e = warp - kEpiWarp0;
+        const int r = e * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(e * 32) << 16;
+        const int epi_leader = kEpiWarp0 * 32;
+        Ring<2> accr;
+        int64_t s = rs;
+        Piece pc;
+        while (next_piece(p, s, re, pc)) {
+            const uint32_t ab = accr.idx;
+            // one thread waits; all four warps take the same branch
+            if (tid == epi_leader)
+                *epi_ok = mbar_wait(b_accfull + 8u * ab, accr.phase, abort) ? 1 : 0;
+            epi_sync();
+            if (!*epi_ok) break;
+            tc_fence_after();
+            const uint32_t d = tmem + lane_addr + L::kAccStride * ab;
+            // pass 1: Sx (TMEM lane 127) to shared memory
 #pragma unroll
-        for (int c0 = 0; c0 < NT; c0 += 16) {
-            float v[16];
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                float v[16];
+                __syncwarp();
+                tmem_ld16(d + c0, v);
+                if (r == kFeat) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sx[c0 + j] = v[j];
+                }
+            }
+            epi_sync();
+            const bool full = pc.c0 == 0 && pc.c1 == p.nchunks;
+            const int64_t feat = pc.b * kFeat + r;
+            const bool valid_row = r < kFeat && feat < p.n;
+            const float alpha = valid_row ? __ldg(p.alpha + feat) : 0.0f;
+            // workspace row of a partial piece: slot 0 if it opens this CTA's range
+            const int wslot = (pc.b * p.nchunks + pc.c0 == rs) ? 0 : 1;
+            float* prow = full ? nullptr
+                               : p.partial + ((static_cast<int64_t>(blockIdx.x) * 2 + wslot) * kFeat + r) * p.m4;
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                float v[16];
+                __syncwarp();
+                tmem_ld16(d + c0, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = fmaf(p.P, v[j], p.Q * sx[c0 + j]);
+                if (!valid_row) continue;
+                if (full) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < p.m)
+                            p.y[(c0 + j) * p.n + feat] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[j]));
+                } else {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        if (c0 + 4 * q4 < p.m4)
+                            *reinterpret_cast<float4*>(prow + c0 + 4 * q4) = make_float4(
+                                v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                }
+            }
+            tc_fence_before();
             __syncwarp();
-            tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int64_t m = c0 + j;
-                if (m < p.m && row < p.n) {
-                    if (p.splits == 1) {
-                        p.y[m * p.n + row] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v[j], scale)));
-                    } else {
-                        p.partial[(static_cast<int64_t>(ks) * p.m + m) * p.n + row] = v[j];
-                    }
-                }
-            }
-        }
-        tc_fence_before();
-        if (p.splits > 1) {
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) flags[1] = atomicAdd(&p.counters[nb], 1) == p.splits - 1;
-            __syncthreads();
-            if (flags[1]) {  // last segment of this feature block: add in order
+            if (lane == 0) mbar_arrive(b_accempty + 8u * ab);
+            if (!full) {
+                // the last of the block's pieces to finish adds them in K order
                 __threadfence();
-                if (row < p.n) {
-                    for (int64_t m = 0; m < p.m; ++m) {
-                        float acc = 0.0f;
-                        for (int s2 = 0; s2 < p.splits; ++s2)
-                            acc = __fadd_rn(acc, __ldcg(p.partial + (static_cast<int64_t>(s2) * p.m + m) *
-                                                                      p.n + row));
-                        p.y[m * p.n + row] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc, scale)));
+                epi_sync();
+                const int64_t i0 = pc.b * p.nchunks, i1 = i0 + p.nchunks - 1;
+                const int64_t g0 = cta_of_item(p, i0), g1 = cta_of_item(p, i1);
+                if (tid == epi_leader)
+                    *last_flag = atomicAdd(p.counters + pc.b, 1) == static_cast<int>(g1 - g0);
+                epi_sync();
+                if (*last_flag) {
+                    __threadfence();
+                    if (valid_row) {
+                        // CTA g0's piece opens its range iff the range starts at i0
+                        const int slot0 = range_start(p, g0) >= i0 ? 0 : 1;
+                        for (int64_t m0 = 0; m0 < p.m4; m0 += 16) {
+                            float4 acc[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int64_t g = g0; g <= g1; ++g) {
+                                const int sl = g == g0 ? slot0 : 0;
+                                const float4* src = reinterpret_cast<const float4*>(
+                                    p.partial + ((g * 2 + sl) * kFeat + r) * p.m4 + m0);
+                                float4 t[4];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    if (m0 + 4 * q < p.m4) t[q] = __ldcg(src + q);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    if (m0 + 4 * q < p.m4) acc[q] = add4(acc[q], t[q]);
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float a4[4] = {acc[q].x, acc[q].y, acc[q].z, acc[q].w};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int64_t mr = m0 + 4 * q + j;
+                                    if (mr < p.m)
+                                        p.y[mr * p.n + feat] =
+                                            __bfloat16_as_ushort(__float2bfloat16_rn(alpha * a4[j]));
+                                }
+                            }
+                        }
                     }
+                    if (tid == epi_leader) p.counters[pc.b] = 0;
                 }
-                if (tid == 0) p.counters[nb] = 0;
             }
+            epi_sync();  // sx, last_flag and epi_ok are reused by the next piece
+            accr.next();
         }
-        __syncthreads();  // TMEM reads done before the next unit's MMAs
     }
-    // teardown: drain this CTA's MMAs (bounded), free TMEM
-    if (tid == 0 && it > 0) {
-        mma_commit(smem_u32(&bars[kStages]));
-        mbar_wait(smem_u32(&bars[kStages]), done_phase);
-    }
+
+    // teardown: every role is done (or gave up); free TMEM
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(L::kCols)
+                     "r"(kTmemCols)
                      : "memory");
 }
 
 // ------------------------------------------------------------------- host
-
 
 static int sm_count() {
     int dev = 0, n = 0;
@@ -360,52 +776,62 @@ static int sm_count() {
 
 struct Plan {
     int nt;
-    int splits;
-    int64_t kseg;
-    int nblocks;
+    int64_t nblocks, nchunks, items;
+    int grid;
+    bool partials;  // some CTA range cuts a row block
 };
 
 static Plan plan(int64_t m, int64_t n, int64_t k) {
     Plan pl;
     pl.nt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
-    pl.nblocks = static_cast<int>((n + kBlockN - 1) / kBlockN);
-    const int64_t ksteps = k / kStageK;
-    const int64_t target = 2 * static_cast<int64_t>(sm_count());
-    int64_t s = (target + pl.nblocks - 1) / pl.nblocks;
-    const int64_t max_s = ksteps / 4 > 0 ? ksteps / 4 : 1;  // >= 4 stages per segment
-    if (s > max_s) s = max_s;
-    if (s < 1) s = 1;
-    const int64_t steps_per = (ksteps + s - 1) / s;
-    pl.kseg = steps_per * kStageK;
-    pl.splits = static_cast<int>((k + pl.kseg - 1) / pl.kseg);
+    pl.nblocks = (n + kFeat - 1) / kFeat;
+    pl.nchunks = (k + kChunkK - 1) / kChunkK;
+    pl.items = pl.nblocks * pl.nchunks;
+    const int64_t sms = sm_count();
+    pl.grid = static_cast<int>(pl.items < sms ? pl.items : sms);
+    pl.partials = false;
+    for (int64_t g = 0; g <= pl.grid; ++g)
+        if ((g * pl.items / pl.grid) % pl.nchunks != 0) pl.partials = true;
     return pl;
 }
 
-static bool table_of(int q, uint32_t& lo, uint32_t& hi, float& factor) {
-    // numerator of the code c of 2-bit field f (c = 0, 1, -2, -1)
-    const int cs[4] = {0, 1, -2, -1};
-    int num[4];
+// y = alpha * (P * D + Q * Sx) for D = sum x (1 + f'/4), Sx = sum x.
+static bool coeffs_of(int q, float& P, float& Q) {
+    double A, B, factor;
     switch (q) {
-        case PQ_SEQ2: for (int f = 0; f < 4; ++f) num[f] = 2 * cs[f] + 1; factor = 0.25f; break;
-        case PQ_SEQ2_B: for (int f = 0; f < 4; ++f) num[f] = 2 * cs[f] + 1; factor = 1.0f / 3.0f; break;
-        case PQ_TERNARY: for (int f = 0; f < 4; ++f) num[f] = 2 * cs[f]; factor = 1.0f / 3.0f; break;
-        case PQ_LSQ2: case PQ_BINARY: for (int f = 0; f < 4; ++f) num[f] = cs[f]; factor = 1.0f; break;
+        case PQ_SEQ2: A = 2; B = -3; factor = 0.25; break;
+        case PQ_SEQ2_B: A = 2; B = -3; factor = 1.0 / 3.0; break;
+        case PQ_TERNARY: A = 2; B = -4; factor = 1.0 / 3.0; break;
+        case PQ_LSQ2: case PQ_BINARY: A = 1; B = -2; factor = 1.0; break;
         default: return false;
     }
-    uint16_t e[4];
-    for (int f = 0; f < 4; ++f) {  // small integers are exact in bf16
-        const float v = static_cast<float>(num[f]);
-        uint32_t u;
-        __builtin_memcpy(&u, &v, 4);
-        e[f] = static_cast<uint16_t>(u >> 16);
-    }
-    lo = (e[0] & 0xFFu) | ((e[1] & 0xFFu) << 8) | ((e[2] & 0xFFu) << 16) | ((e[3] & 0xFFu) << 24);
-    hi = (e[0] >> 8) | ((e[1] >> 8) << 8) | ((e[2] >> 8) << 16) | (static_cast<uint32_t>(e[3] >> 8) << 24);
+    P = static_cast<float>(4.0 * A * factor);
+    Q = static_cast<float>((B - 4.0 * A) * factor);
     return true;
 }
 
+static int64_t partial_bytes(const Plan& pl, int64_t m) {
+    const int64_t m4 = (m + 3) / 4 * 4;
+    return (static_cast<int64_t>(pl.grid) * 2 * kFeat * m4 * 4 + 255) / 256 * 256;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
 template <int NT>
-static cudaError_t launch(const GemmParams& p, int64_t units, cudaStream_t s) {
+static cudaError_t launch(const CUtensorMap& tc, const CUtensorMap& tx, const GemmParams& p,
+                          cudaStream_t s) {
     using L = Layout<NT>;
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -416,9 +842,7 @@ static cudaError_t launch(const GemmParams& p, int64_t units, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int64_t sms = sm_count();
-    const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
-    wq_gemm_kernel<NT><<<grid, kThreads, L::kBytes, s>>>(p);
+    wq_gemm_kernel<NT><<<p.grid, kThreads, L::kBytes, s>>>(tc, tx, p);
     return cudaGetLastError();
 }
 
@@ -429,20 +853,20 @@ using namespace pqg;
 extern "C" {
 
 int64_t pq_wq_gemm_workspace_bytes(pq_quant_t q, int64_t m, int64_t n, int64_t k) {
-    uint32_t lo, hi;
-    float f;
-    if (!table_of(q, lo, hi, f) || m < 1 || m > 128 || n < 1 || k < kStageK || k % kStageK) return -1;
+    float P, Q;
+    if (!coeffs_of(q, P, Q) || m < 1 || m > 128 || n < 1 || k < kMinK || k % kMinK) return -1;
     const Plan pl = plan(m, n, k);
-    if (pl.splits == 1) return 0;
-    return static_cast<int64_t>(pl.splits) * m * n * 4 + static_cast<int64_t>(pl.nblocks) * 4 + 256;
+    if (!pl.partials) return 0;
+    return partial_bytes(pl, m) + pl.nblocks * 4;
 }
 
 pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k, const uint16_t* x_bf16,
                        const uint8_t* packed, const float* alpha, uint16_t* y_bf16, void* workspace,
                        int64_t workspace_bytes, void* stream) {
     GemmParams p = {};
-    if (!table_of(q, p.table_lo, p.table_hi, p.factor)) return PQ_ERR_UNSUPPORTED;
-    if (m < 1 || m > 128 || n < 1 || k < kStageK || k % kStageK) return PQ_ERR_INVALID_ARG;
+    if (!coeffs_of(q, p.P, p.Q)) return PQ_ERR_UNSUPPORTED;
+    if (m < 1 || m > 128 || n < 1 || k < kMinK || k % kMinK) return PQ_ERR_INVALID_ARG;
+    if (n > (int64_t{1} << 30) || k > (int64_t{1} << 30)) return PQ_ERR_INVALID_ARG;
     if (!x_bf16 || !packed || !alpha || !y_bf16) return PQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) || (reinterpret_cast<uintptr_t>(packed) & 15) ||
         (reinterpret_cast<uintptr_t>(y_bf16) & 1))
@@ -450,32 +874,54 @@ pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k, const uint
     const Plan pl = plan(m, n, k);
     const int64_t need = pq_wq_gemm_workspace_bytes(q, m, n, k);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    p.x = x_bf16;
-    p.codes = packed;
     p.alpha = alpha;
     p.y = y_bf16;
     p.m = m;
     p.n = n;
     p.k = k;
-    p.kseg = pl.kseg;
-    p.splits = pl.splits;
+    p.m4 = (m + 3) / 4 * 4;
     p.nblocks = pl.nblocks;
-    if (pl.splits > 1) {
+    p.nchunks = pl.nchunks;
+    p.items = pl.items;
+    p.grid = pl.grid;
+    if (need > 0) {
         if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
             return PQ_ERR_INVALID_ARG;
         p.partial = static_cast<float*>(workspace);
-        p.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                            static_cast<int64_t>(pl.splits) * m * n * 4);
-        if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(pl.nblocks) * 4, s) != cudaSuccess)
+        p.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes(pl, m));
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return PQ_ERR_CUDA;
+    CUtensorMap tc, tx;
+    {  // codes [n rows][k/4 bytes]: boxes of 127 rows x 128 B, 128B swizzle
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 4), static_cast<cuuint64_t>(n)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 4)};
+        const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kFeat)};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return PQ_ERR_CUDA;
     }
-    const int64_t units = static_cast<int64_t>(pl.nblocks) * pl.splits;
+    {  // activations [m rows][k bf16]: boxes of NT rows x 64 K, 128B swizzle
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(m)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k * 2)};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pl.nt)};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x_bf16), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return PQ_ERR_CUDA;
+    }
+    if (need > 0 &&
+        cudaMemsetAsync(p.counters, 0, static_cast<size_t>(pl.nblocks) * 4, s) != cudaSuccess)
+        return PQ_ERR_CUDA;
     cudaError_t e;
     switch (pl.nt) {
-        case 16: e = launch<16>(p, units, s); break;
-        case 32: e = launch<32>(p, units, s); break;
-        case 64: e = launch<64>(p, units, s); break;
-        default: e = launch<128>(p, units, s); break;
+        case 16: e = launch<16>(tc, tx, p, s); break;
+        case 32: e = launch<32>(tc, tx, p, s); break;
+        case 64: e = launch<64>(tc, tx, p, s); break;
+        default: e = launch<128>(tc, tx, p, s); break;
     }
     return e == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
@@ -504,10 +950,9 @@ static std::atomic<void*> g_noalloc_addr[kNoAllocDevices];
 extern "C" pq_status_t pq_wq_gemm_noalloc(pq_quant_t q, int64_t m, int64_t n, int64_t k,
                                           const uint16_t* x_bf16, const uint8_t* packed,
                                           const float* alpha, uint16_t* y_bf16, void* stream) {
-    uint32_t lo, hi;
-    float factor;
-    if (!table_of(q, lo, hi, factor)) return PQ_ERR_UNSUPPORTED;
-    if (m < 1 || m > 128 || n < 1 || k < kStageK || k % kStageK || !x_bf16 || !packed || !alpha ||
+    float P, Q;
+    if (!coeffs_of(q, P, Q)) return PQ_ERR_UNSUPPORTED;
+    if (m < 1 || m > 128 || n < 1 || k < kMinK || k % kMinK || !x_bf16 || !packed || !alpha ||
         !y_bf16)
         return PQ_ERR_INVALID_ARG;
     if (pq_wq_gemm_workspace_bytes(q, m, n, k) > PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES)

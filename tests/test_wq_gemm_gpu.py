@@ -46,7 +46,8 @@ def _check(q, x, packed, a, y):
 @pytest.mark.parametrize("q", Q2)
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 300, 256), (16, 1024, 4096),
                                    (33, 640, 1024), (64, 2048, 2048), (128, 256, 512),
-                                   (7, 4096, 14336)])
+                                   (7, 4096, 14336), (20, 1000, 640), (3, 130, 384),
+                                   (100, 509, 1536)])
 def test_wq_gemm_matches_oracle(q, m, n, k):
     x, packed, a = _case(q, m, n, k, seed=m + n + k)
     y = pq.wq_gemm(q, x, packed, a)
