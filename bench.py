@@ -48,6 +48,9 @@ def parse():
                         "wq_gemm: Y = X W^T from the packed 2-bit codes on the tensor cores")
     p.add_argument("--m", type=int, default=16,
                    help="wq_gemm: activation rows (tokens of a decode batch), 1..128")
+    p.add_argument("--shape", default="llama3_8b", choices=["llama3_8b", "16384"],
+                   help="wq_gemm: every matrix of the Llama-3-8B-shaped set, or one "
+                        "16384x16384 weight (the size the pages compare kernels at)")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -667,7 +670,13 @@ def run_wq_gemm(args):
     dev = "cuda:0"
     m = args.m
     q = pq.PQ_SEQ2
-    step = QuantStep(I.llama3_8b_set(), q, device=dev, pack=True)
+    if args.shape == "16384":
+        # one 16384^2 weight, several copies so that every replay reads HBM
+        # (codes 64 MiB and bf16 weights 512 MiB per copy; L2 is 126 MB)
+        mats = [I.Matrix(f"w{i}", 16384, 16384, i, 0) for i in range(4)]
+    else:
+        mats = I.llama3_8b_set()
+    step = QuantStep(mats, q, device=dev, pack=True)
     step.generate(seed=3)
     step.fwd_all()
     torch.cuda.synchronize()
@@ -745,9 +754,10 @@ def run_wq_gemm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16 x 2-bit codes, f32 accumulate",
         "data": "synthetic",
-        "config": {"workload": f"llama3_8b_linear_set_seq2_wq_gemm_m{m}", "m": m,
+        "config": {"workload": (f"llama3_8b_linear_set_seq2_wq_gemm_m{m}" if args.shape != "16384"
+                                else f"4x16384x16384_seq2_wq_gemm_m{m}"), "m": m,
                    "weights": weights, "launches_per_step": len(step.bufs),
-                   "l2": "codes 1.75 GB per step, larger than L2"},
+                   "l2": f"codes {step.weights / 4e9:.2f} GB per step, larger than L2"},
         "roofline": roof,
         "tflops": flops_step / (ms * 1e-3) / 1e12,
         "cublas_bf16_dense": {"ms_per_step": ms_dense, "speedup_of_ours": ms_dense / ms,
