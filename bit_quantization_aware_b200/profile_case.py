@@ -2,6 +2,8 @@
 
     python -m bit_quantization_aware_b200.profile_case --rows 14336 --cols 4096 \
         --quant seq2 --iters 3 [--pack]
+    python -m bit_quantization_aware_b200.profile_case --rows 16384 --cols 16384 \
+        --quant seq2 --iters 3 --gemm-m 1
 
 Draws seeded synthetic inputs on the device (N(0, 0.02) weights, alpha =
 max|w_row| or the quantizer's init, bf16 N(0, 1e-3) upstream gradient),
@@ -26,9 +28,13 @@ def main():
     p.add_argument("--quant", default="seq2", choices=sorted(pq.QUANTIZERS))
     p.add_argument("--iters", type=int, default=3)
     p.add_argument("--pack", action="store_true")
+    p.add_argument("--gemm-m", type=int, default=0,
+                   help="run the weight-only matmul with this many activation rows")
     a = p.parse_args()
     q = pq.QUANTIZERS[a.quant]
     dev = torch.device("cuda")
+    if a.gemm_m:
+        return gemm_case(a, q, dev)
     w = I.normal_weights(a.rows, a.cols, seed=0, stream=0, device=dev)
     alpha = I.alpha_init(w, q)
     g = I.grad_bf16(a.rows, a.cols, seed=0, stream=64, device=dev)
@@ -52,6 +58,30 @@ def main():
         fb = 6 + (pq.pq_code_bits(q) / 8 if a.pack else 0)
         print(f"iter {i}: fwd {tf * 1e6:.1f} us ({n * fb / tf / 1e9:.0f} GB/s), "
               f"bwd {tb * 1e6:.1f} us ({n * 10 / tb / 1e9:.0f} GB/s)")
+
+
+def gemm_case(a, q, dev):
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    bits = pq.pq_code_bits(q)
+    packed = torch.randint(0, 256, (a.rows, a.cols * bits // 8), dtype=torch.uint8,
+                           device=dev, generator=g)
+    alpha = torch.rand(a.rows, device=dev, generator=g) + 0.5
+    x = torch.randn(a.gemm_m, a.cols, device=dev, generator=g).to(torch.bfloat16)
+    y = torch.empty((a.gemm_m, a.rows), dtype=torch.bfloat16, device=dev)
+    need = pq.pq_wq_gemm_workspace_bytes(q, a.gemm_m, a.rows, a.cols)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    for i in range(a.iters):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        pq.pq_wq_gemm(q, x, packed, alpha, y, ws)
+        e[1].record()
+        torch.cuda.synchronize()
+        t = e[0].elapsed_time(e[1]) * 1e-3
+        print(f"iter {i}: wq_gemm {t * 1e6:.1f} us ({packed.numel() / t / 1e9:.0f} GB/s of codes)")
+    if pq.pq_device_status() != 0:
+        raise RuntimeError("a bounded device wait gave up")
 
 
 if __name__ == "__main__":
