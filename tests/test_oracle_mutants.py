@@ -54,7 +54,7 @@ MUTANTS = {
     "matmul_seq_level": ("else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / (2.0 * p.kh);",
                          "else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / 4.0;"),
     "matmul_no_alpha": ("y[i * n + j] = acc * (double)alpha[j];", "y[i * n + j] = acc;"),
-    "dequant_no_alpha": ("volatile float prod = lev * alpha;",
+    "fwd_level_no_alpha": ("volatile float prod = lev * alpha;",
                          "volatile float prod = lev;"),
     "binary_sign_zero": ("c = (x >= 0.0f) ? 1 : -1;", "c = (x > 0.0f) ? 1 : -1;"),
     "scale_multiplies": ("float x = w / alpha;", "float x = w * alpha;"),
@@ -67,18 +67,6 @@ MUTANTS = {
                                "int c = (int)f;"),
     "dequant_field_order": ("unsigned f = (byte >> (p.bits * (int)(j % per_byte))) & mask;",
                             "unsigned f = (byte >> (p.bits * (int)(per_byte - 1 - j % per_byte))) & mask;"),
-    "adamw_no_bias_correction": ("k.step = (float)(h->lr / (1.0 - pow(h->beta1, t)));", "k.step = (float)h->lr;"),
-    "adamw_no_eps": ("volatile float den = sc + k->eps;", "volatile float den = sc;"),
-    "adamw_no_sqrt": ("volatile float sq = sqrtf(*v);", "volatile float sq = *v;"),
-    "adamw_betas_swapped": ("volatile float a1 = k->b1 * *m;", "volatile float a1 = k->b2 * *m;"),
-    "adamw_decay_sign": ("k.decay = (float)(1.0 - h->lr * h->weight_decay);", "k.decay = (float)(1.0 + h->lr * h->weight_decay);"),
-    "adamw_alpha_uses_w_hparams": ("alpha[r] = pqo_adamw_update(&ka,", "alpha[r] = pqo_adamw_update(&kw,"),
-    "reduce_no_multiplier": ("volatile float gbar = sum * grad_mult;", "volatile float gbar = sum;"),
-    "reduce_first_source_only": ("volatile float t = sum + pqo_bf16_to_float(g_srcs[k][r * cols + j]);",
-                                 "volatile float t = pqo_bf16_to_float(g_srcs[0][r * cols + j]);"),
-    "matmul_seq_level": ("else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / (2.0 * p.kh);",
-                         "else if (p.shift != 0.0f) lev = (2.0 * c + 1.0) / 4.0;"),
-    "matmul_no_alpha": ("y[i * n + j] = acc * (double)alpha[j];", "y[i * n + j] = acc;"),
     "dequant_no_alpha": ("volatile float prod = pqo_level_of_code(&p, c) * alpha[r];",
                          "volatile float prod = pqo_level_of_code(&p, c);"),
 }
