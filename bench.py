@@ -316,6 +316,7 @@ def run_ours(args):
     ev_end = torch.cuda.Event(enable_timing=True)
     bwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    fwd_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     gpu_index = local
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -331,6 +332,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     ev_start.record(stream)
     for k in range(args.steps):
+        fwd_ev[k].record(stream)
         step.fwd_all()
         bwd_ev[k][0].record(stream)
         step.bwd_all()
@@ -342,7 +344,8 @@ def run_ours(args):
 
     ms_total = ev_start.elapsed_time(ev_end)
     bwd_ms = sum(a.elapsed_time(b) for a, b in bwd_ev)
-    ms_total, bwd_ms = reduce_max([ms_total, bwd_ms], f"cuda:{local}", world)
+    fwd_ms = sum(a.elapsed_time(b[0]) for a, b in zip(fwd_ev, bwd_ev))
+    ms_total, bwd_ms, fwd_ms = reduce_max([ms_total, bwd_ms, fwd_ms], f"cuda:{local}", world)
     ms_step = ms_total / args.steps
     value = step_throughput(weights, world, ms_step)
 
@@ -365,6 +368,16 @@ def run_ours(args):
                 "fwd_bwd_frac_of_peak": (step.bytes_fwd() + bwd_bytes_step)
                 / (ms_step * 1e-3) / 1e9 / peak}
 
+    def phase(ms_per_step, nbytes):
+        sec = ms_per_step * 1e-3
+        return {"ms_per_step": ms_per_step, "Gweights_s": step_throughput(weights, world, ms_per_step),
+                "GB_s": nbytes / sec / 1e9, "frac_of_peak": nbytes / sec / 1e9 / peak,
+                "algorithmic_bytes": nbytes}
+    phases = {"fwd": phase(fwd_ms / args.steps, step.bytes_fwd()),
+              "bwd": phase(bwd_ms / args.steps, bwd_bytes_step),
+              "fwd_bwd": phase(ms_step, step.bytes_fwd() + bwd_bytes_step),
+              "peak_GB_s": peak}
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(step, args, local, world)
@@ -384,7 +397,7 @@ def run_ours(args):
                 "bf16 N(0,1e-3) upstream grads, alpha = max|w_row|)",
                 "config": config_dict(world, weights),
                 "gpu_launches": step.launches_per_step * args.steps,
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "phases": phases, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
