@@ -668,11 +668,12 @@ def run_bwd_adamw(args):
 
 def run_wq_gemm(args):
     """Weight-only 2-bit matmul Y = X (alpha * levels)^T for every matrix of
-    the Llama-3-8B-shaped set (224 launches per step, captured in one CUDA
-    graph; the 1.75 GB of codes are far larger than L2, so every launch
-    reads its codes from HBM), 1 GPU, X of --m rows. Beside it, for
-    context, cuBLAS (torch.matmul) on the dense bf16 dequantized weights,
-    also graph-captured. Prints one JSON line."""
+    the Llama-3-8B-shaped set (224 matrices in grouped launches of up to 64,
+    captured in one CUDA graph; the 1.75 GB of codes are far larger than L2,
+    so every launch reads its codes from HBM), 1 GPU, X of --m rows. Beside
+    it, for context, the same with one launch per matrix, and cuBLAS
+    (torch.matmul) on the dense bf16 dequantized weights, also
+    graph-captured. Prints one JSON line."""
     import torch
 
     from bit_quantization_aware_b200 import inputs as I
@@ -702,10 +703,22 @@ def run_wq_gemm(args):
     ys_ref = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in ns}
     need = max(pq.pq_wq_gemm_workspace_bytes(q, m, b.m.rows, b.m.cols) for b in step.bufs)
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    # grouped launches: up to 64 matrices each, in equal groups
+    ngroups = (len(step.bufs) + 63) // 64
+    gsize = (len(step.bufs) + ngroups - 1) // ngroups
+    groups = [pq.gemm_problem_array([dict(x=xs[b.m.cols], packed=b.packed, alpha=b.alpha,
+                                          y=ys[b.m.rows]) for b in step.bufs[i:i + gsize]])
+              for i in range(0, len(step.bufs), gsize)]
+    gneed = max(pq.pq_wq_gemm_batch_workspace_bytes(q, m, g) for g in groups)
+    gws = torch.empty(max(gneed, 256), dtype=torch.uint8, device=dev)
 
-    def ours():
+    def ours_single():
         for b in step.bufs:
             pq.pq_wq_gemm(q, xs[b.m.cols], b.packed, b.alpha, ys[b.m.rows], ws)
+
+    def ours():
+        for g in groups:
+            pq.pq_wq_gemm_batch(q, m, g, gws)
 
     def dense():
         for b in step.bufs:
@@ -734,13 +747,14 @@ def run_wq_gemm(args):
         return e0.elapsed_time(e1) / args.steps, g
 
     ms, g_ours = timed(ours)
+    ms_single, g_single = timed(ours_single)
     ms_dense, g_dense = timed(dense)
     assert pq.pq_device_status() == 0
     # the last matrix of the set, both ways (same weights, fp32 sums)
     b = step.bufs[-1]
     yo, yr = ys[b.m.rows].float(), ys_ref[b.m.rows].float()
     rel = float((yo - yr).abs().max() / yr.abs().max().clamp_min(1e-30))
-    del g_ours, g_dense
+    del g_ours, g_single, g_dense
 
     weights = step.weights
     bytes_step = sum(b.m.numel // 4 + b.m.rows * 4 + m * b.m.cols * 2 + m * b.m.rows * 2
@@ -769,10 +783,13 @@ def run_wq_gemm(args):
         "data": "synthetic",
         "config": {"workload": (f"llama3_8b_linear_set_seq2_wq_gemm_m{m}" if args.shape != "16384"
                                 else f"4x16384x16384_seq2_wq_gemm_m{m}"), "m": m,
-                   "weights": weights, "launches_per_step": len(step.bufs),
+                   "weights": weights, "launches_per_step": len(groups),
+                   "matrices_per_launch": gsize,
                    "l2": f"codes {step.weights / 4e9:.2f} GB per step, larger than L2"},
         "roofline": roof,
         "tflops": flops_step / (ms * 1e-3) / 1e12,
+        "per_matrix_launches": {"ms_per_step": ms_single, "launches_per_step": len(step.bufs),
+                                "what": "pq_wq_gemm once per matrix, CUDA graph"},
         "cublas_bf16_dense": {"ms_per_step": ms_dense, "speedup_of_ours": ms_dense / ms,
                               "what": "torch.matmul(x, W_bf16.t()) per matrix, CUDA graph",
                               "max_rel_diff_last_matrix": rel}}), flush=True)

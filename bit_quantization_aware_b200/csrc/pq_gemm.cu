@@ -72,16 +72,32 @@ constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
 // nonzero after a bounded wait gave up (read by pq_device_status)
 __device__ int g_status = 0;
 
-struct GemmParams {
-    const float* alpha;  // [N]
-    uint16_t* y;         // [M, N] bf16
+// One matrix of a launch: its tensor maps, outputs and place in the work list.
+struct Problem {
+    CUtensorMap tc;      // codes [n rows][k/4 bytes], boxes of 127 rows x 128 B
+    CUtensorMap tx;      // activations [m rows][k], boxes of NT rows x 64 K
+    const float* alpha;  // [n]
+    uint16_t* y;         // [m, n] bf16
+    int64_t n, k;
+    int64_t nchunks;     // ceil(k / kChunkK)
+    int64_t item0;       // its first (block, chunk) item in the launch's list
+    int64_t block0;      // its first block counter
+};
+
+// Shared by the matrices of a launch (same activation rows m).
+struct GemmCommon {
     float* partial;      // [2 * grid, kFeat, m4] fp32 (partial blocks only)
-    int* counters;       // [nblocks], zero on entry (partial blocks only)
-    int64_t m, n, k;
-    int64_t m4;          // m rounded up to a multiple of 4 (partial row length)
-    int64_t nblocks, nchunks, items;
-    int32_t grid;
+    int* counters;       // [all blocks], zero on entry (partial blocks only)
+    int64_t m, m4;       // activation rows; m rounded up to a multiple of 4
+    int64_t items;       // items of all matrices
+    int32_t grid, count;
     float P, Q;          // y = alpha * (P * D + Q * Sx)
+};
+
+template <int MAXP>
+struct GemmParams {
+    GemmCommon c;
+    Problem prob[MAXP];
 };
 
 // ----------------------------------------------------------- primitives
@@ -299,41 +315,49 @@ __device__ __forceinline__ void drain_ring(uint32_t bar0, Ring<N> r, uint32_t is
     }
 }
 
-// One piece of a CTA's range: row block b, code chunks [c0, c1).
+// One piece of a CTA's range: matrix pi, row block b, code chunks [c0, c1).
 struct Piece {
+    int pi;
     int64_t b, c0, c1;
 };
 
-// Items [s, e) of CTA g (item = block * nchunks + chunk).
-__device__ __forceinline__ int64_t range_start(const GemmParams& p, int64_t g) {
+// Items [s, e) of CTA g. The items of matrix p are item0 + b * nchunks + chunk.
+__device__ __forceinline__ int64_t range_start(const GemmCommon& p, int64_t g) {
     return g * p.items / p.grid;
 }
 
-__device__ __forceinline__ bool next_piece(const GemmParams& p, int64_t& s, int64_t e, Piece& pc) {
+// Next piece of [s, e); cur is the matrix the walk is in (items only grow).
+template <int MAXP>
+__device__ __forceinline__ bool next_piece(const GemmParams<MAXP>& prm, int64_t& s, int64_t e,
+                                           Piece& pc, int& cur) {
     if (s >= e) return false;
-    const int64_t b = s / p.nchunks;
-    const int64_t blk_end = (b + 1) * p.nchunks;
+    while (cur + 1 < prm.c.count && s >= prm.prob[cur + 1].item0) ++cur;
+    const Problem& pb = prm.prob[cur];
+    const int64_t local = s - pb.item0;
+    const int64_t b = local / pb.nchunks;
+    const int64_t blk_end = pb.item0 + (b + 1) * pb.nchunks;
     const int64_t pe = e < blk_end ? e : blk_end;
+    pc.pi = cur;
     pc.b = b;
-    pc.c0 = s - b * p.nchunks;
-    pc.c1 = pe - b * p.nchunks;
+    pc.c0 = local - b * pb.nchunks;
+    pc.c1 = pe - pb.item0 - b * pb.nchunks;
     s = pe;
     return true;
 }
 
-// MMA stages of code chunk c (the last chunk of a row may be short).
-__device__ __forceinline__ int stages_of_chunk(const GemmParams& p, int64_t c) {
-    const int64_t rest = (p.k - c * kChunkK + kStageK - 1) / kStageK;
+// MMA stages of code chunk c of a K-long row (the last chunk may be short).
+__device__ __forceinline__ int stages_of_chunk(int64_t k, int64_t c) {
+    const int64_t rest = (k - c * kChunkK + kStageK - 1) / kStageK;
     return rest < kStagesPerChunk ? static_cast<int>(rest) : kStagesPerChunk;
 }
 
 // K of the stage starting at k0: kStageK, or 128 for a short tail.
-__device__ __forceinline__ int stage_k(const GemmParams& p, int64_t k0) {
-    return p.k - k0 < kStageK ? static_cast<int>(p.k - k0) : kStageK;
+__device__ __forceinline__ int stage_k(int64_t k, int64_t k0) {
+    return k - k0 < kStageK ? static_cast<int>(k - k0) : kStageK;
 }
 
 // CTA whose range holds item i: the largest g with range_start(g) <= i.
-__device__ __forceinline__ int64_t cta_of_item(const GemmParams& p, int64_t i) {
+__device__ __forceinline__ int64_t cta_of_item(const GemmCommon& p, int64_t i) {
     return ((i + 1) * p.grid + p.items - 1) / p.items - 1;
 }
 
@@ -365,11 +389,11 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
                        __fadd_rn(a.w, b.w));
 }
 
-template <int NT>
+template <int NT, int MAXP>
 __global__ void __launch_bounds__(kThreads, 1)
-    wq_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes,
-                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ GemmParams p) {
+    wq_gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
     using L = Layout<NT>;
+    const GemmCommon& p = prm.c;
     constexpr int SC = L::kCodesSlots, SA = L::kASlots, SB = L::kBSlots;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -408,10 +432,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid == kCodesWarp * 32) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_codes))
-                     : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x))
-                     : "memory");
+        for (int i = 0; i < prm.c.count && i < 4; ++i) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&prm.prob[i].tc))
+                         : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&prm.prob[i].tx))
+                         : "memory");
+        }
     }
     __syncwarp();
     if (warp == 0) {
@@ -434,15 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t issued = 0;
             int64_t s = rs;
             Piece pc;
+            int cur = 0;
             bool ok = true;
-            while (ok && next_piece(p, s, re, pc)) {
+            while (ok && next_piece(prm, s, re, pc, cur)) {
                 for (int64_t c = pc.c0; c < pc.c1; ++c) {
                     if (!mbar_wait(b_cempty + 8u * cr.idx, cr.phase ^ 1u, abort)) {
                         ok = false;
                         break;
                     }
                     mbar_expect_tx(b_cfull + 8u * cr.idx, kCodesTx);
-                    tma_load_2d(sbase + L::kCodesOff + cr.idx * kCodesSlotBytes, &tm_codes,
+                    tma_load_2d(sbase + L::kCodesOff + cr.idx * kCodesSlotBytes, &prm.prob[pc.pi].tc,
                                 b_cfull + 8u * cr.idx, static_cast<int32_t>(c * (kChunkK / 4)),
                                 static_cast<int32_t>(pc.b * kFeat));
                     cr.next();
@@ -460,10 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t gs = 0;
             int64_t s = rs;
             Piece pc;
+            int cur = 0;
             bool ok = true;
-            while (ok && next_piece(p, s, re, pc)) {
+            while (ok && next_piece(prm, s, re, pc, cur)) {
                 for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk(p, c);
+                    const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
                     for (int i = 0; i < ns; ++i, ++gs) {
                         if (gs >= static_cast<uint32_t>(SB)) {  // B slot free: stage gs - SB done
                             if (!mbar_wait(b_aempty + 8u * er.idx, er.phase, abort)) {
@@ -473,11 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             er.next();
                         }
                         const int64_t k0 = c * kChunkK + i * kStageK;
-                        const int boxes = stage_k(p, k0) / 64;
+                        const int boxes = stage_k(prm.prob[pc.pi].k, k0) / 64;
                         const uint32_t dst = sbase + L::kBOff + xr.idx * L::kBSlot;
                         mbar_expect_tx(b_xfull + 8u * xr.idx, static_cast<uint32_t>(boxes * NT * 128));
                         for (int bx = 0; bx < boxes; ++bx)
-                            tma_load_2d(dst + bx * L::kAtomB, &tm_x, b_xfull + 8u * xr.idx,
+                            tma_load_2d(dst + bx * L::kAtomB, &prm.prob[pc.pi].tx, b_xfull + 8u * xr.idx,
                                         static_cast<int32_t>(k0 + 64 * bx), 0);
                         xr.next();
                     }
@@ -496,15 +524,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             Ring<2> accr;
             int64_t s = rs;
             Piece pc;
+            int cur = 0;
             bool ok = true;
-            while (ok && next_piece(p, s, re, pc)) {
+            while (ok && next_piece(prm, s, re, pc, cur)) {
                 if (!mbar_wait(b_accempty + 8u * accr.idx, accr.phase ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + L::kAccStride * accr.idx;
                 uint32_t acc0 = 0;
                 for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk(p, c);
-                    const bool short_tail = stage_k(p, c * kChunkK + (ns - 1) * kStageK) != kStageK;
+                    const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
+                    const bool short_tail = stage_k(prm.prob[pc.pi].k, c * kChunkK + (ns - 1) * kStageK) != kStageK;
                     for (int i = 0; i < ns; ++i) {
                         if (!mbar_wait(b_afull + 8u * ar.idx, ar.phase, abort)) {
                             ok = false;
@@ -540,18 +569,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<SA> ar;
         int64_t s = rs;
         Piece pc;
+        int cur = 0;
         bool ok = true;
-        while (ok && next_piece(p, s, re, pc)) {
+        while (ok && next_piece(prm, s, re, pc, cur)) {
             for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
                 if (!warp_wait(b_cfull + 8u * cr.idx, cr.phase, abort)) {
                     ok = false;
                     break;
                 }
                 const uint32_t crow = sbase + L::kCodesOff + cr.idx * kCodesSlotBytes + r * 128;
-                const int ns = stages_of_chunk(p, c);
+                const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
                 for (int i = 0; i < ns; ++i) {
                     // this warp's 128 K of the stage exist unless the stage is a short tail
-                    const bool mine = stage_k(p, c * kChunkK + i * kStageK) > 128 * half;
+                    const bool mine = stage_k(prm.prob[pc.pi].k, c * kChunkK + i * kStageK) > 128 * half;
                     // 128 K of this row (32 code bytes) -> 64 TMEM columns, 64 K at a time
                     const int ch = 4 * i + 2 * half;
                     uint4 cw = make_uint4(0, 0, 0, 0);
@@ -604,16 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<SA> ar;
         int64_t s = rs;
         Piece pc;
+        int cur = 0;
         bool ok = true;
-        while (ok && next_piece(p, s, re, pc)) {
+        while (ok && next_piece(prm, s, re, pc, cur)) {
             for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                const int ns = stages_of_chunk(p, c);
+                const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
                 for (int i = 0; i < ns; ++i) {
                     if (!warp_wait(b_xfull + 8u * br.idx, br.phase, abort)) {
                         ok = false;
                         break;
                     }
-                    const int groups = stage_k(p, c * kChunkK + i * kStageK) / 16;
+                    const int groups = stage_k(prm.prob[pc.pi].k, c * kChunkK + i * kStageK) / 16;
                     const uint32_t bslot = sbase + L::kBOff + br.idx * L::kBSlot;
                     for (int it = ptid; it < NT * groups; it += kPermWarps * 32) {
                         const int bro = it % NT, g = it / NT;
@@ -649,7 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<2> accr;
         int64_t s = rs;
         Piece pc;
-        while (next_piece(p, s, re, pc)) {
+        int cur = 0;
+        while (next_piece(prm, s, re, pc, cur)) {
             const uint32_t ab = accr.idx;
             // one thread waits; all four warps take the same branch
             if (tid == epi_leader)
@@ -670,12 +702,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             epi_sync();
-            const bool full = pc.c0 == 0 && pc.c1 == p.nchunks;
+            const Problem& pb = prm.prob[pc.pi];
+            const bool full = pc.c0 == 0 && pc.c1 == pb.nchunks;
             const int64_t feat = pc.b * kFeat + r;
-            const bool valid_row = r < kFeat && feat < p.n;
-            const float alpha = valid_row ? __ldg(p.alpha + feat) : 0.0f;
+            const bool valid_row = r < kFeat && feat < pb.n;
+            const float alpha = valid_row ? __ldg(pb.alpha + feat) : 0.0f;
             // workspace row of a partial piece: slot 0 if it opens this CTA's range
-            const int wslot = (pc.b * p.nchunks + pc.c0 == rs) ? 0 : 1;
+            const int wslot = (pb.item0 + pc.b * pb.nchunks + pc.c0 == rs) ? 0 : 1;
             float* prow = full ? nullptr
                                : p.partial + ((static_cast<int64_t>(blockIdx.x) * 2 + wslot) * kFeat + r) * p.m4;
 #pragma unroll
@@ -690,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (c0 + j < p.m)
-                            p.y[(c0 + j) * p.n + feat] =
+                            pb.y[(c0 + j) * pb.n + feat] =
                                 __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[j]));
                 } else {
 #pragma unroll
@@ -707,10 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the last of the block's pieces to finish adds them in K order
                 __threadfence();
                 epi_sync();
-                const int64_t i0 = pc.b * p.nchunks, i1 = i0 + p.nchunks - 1;
+                const int64_t i0 = pb.item0 + pc.b * pb.nchunks, i1 = i0 + pb.nchunks - 1;
                 const int64_t g0 = cta_of_item(p, i0), g1 = cta_of_item(p, i1);
                 if (tid == epi_leader)
-                    *last_flag = atomicAdd(p.counters + pc.b, 1) == static_cast<int>(g1 - g0);
+                    *last_flag = atomicAdd(p.counters + pb.block0 + pc.b, 1) == static_cast<int>(g1 - g0);
                 epi_sync();
                 if (*last_flag) {
                     __threadfence();
@@ -740,13 +773,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int j = 0; j < 4; ++j) {
                                     const int64_t mr = m0 + 4 * q + j;
                                     if (mr < p.m)
-                                        p.y[mr * p.n + feat] =
+                                        pb.y[mr * pb.n + feat] =
                                             __bfloat16_as_ushort(__float2bfloat16_rn(alpha * a4[j]));
                                 }
                             }
                         }
                     }
-                    if (tid == epi_leader) p.counters[pc.b] = 0;
+                    if (tid == epi_leader) p.counters[pb.block0 + pc.b] = 0;
                 }
             }
             epi_sync();  // sx, last_flag and epi_ok are reused by the next piece
@@ -774,24 +807,42 @@ static int sm_count() {
     return n;
 }
 
+constexpr int kMaxBatch = 64;  // matrices per launch (their descriptors travel as parameters)
+
 struct Plan {
     int nt;
-    int64_t nblocks, nchunks, items;
+    int64_t items, blocks;  // over all matrices of the launch
     int grid;
-    bool partials;  // some CTA range cuts a row block
+    bool partials;          // some CTA range cuts a row block
 };
 
-static Plan plan(int64_t m, int64_t n, int64_t k) {
+// Work list of a launch: matrix i's items start at item0[i], its block
+// counters at block0[i].
+static Plan plan(int64_t m, const pq_gemm_problem_t* pr, int count, int64_t* item0,
+                 int64_t* block0, int64_t* nchunks) {
     Plan pl;
     pl.nt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
-    pl.nblocks = (n + kFeat - 1) / kFeat;
-    pl.nchunks = (k + kChunkK - 1) / kChunkK;
-    pl.items = pl.nblocks * pl.nchunks;
+    int64_t items = 0, blocks = 0;
+    for (int i = 0; i < count; ++i) {
+        const int64_t nb = (pr[i].n + kFeat - 1) / kFeat;
+        const int64_t nc = (pr[i].k + kChunkK - 1) / kChunkK;
+        item0[i] = items;
+        block0[i] = blocks;
+        nchunks[i] = nc;
+        items += nb * nc;
+        blocks += nb;
+    }
+    pl.items = items;
+    pl.blocks = blocks;
     const int64_t sms = sm_count();
-    pl.grid = static_cast<int>(pl.items < sms ? pl.items : sms);
+    pl.grid = static_cast<int>(items < sms ? items : sms);
     pl.partials = false;
-    for (int64_t g = 0; g <= pl.grid; ++g)
-        if ((g * pl.items / pl.grid) % pl.nchunks != 0) pl.partials = true;
+    int cur = 0;
+    for (int64_t g = 1; g < pl.grid; ++g) {
+        const int64_t st = g * items / pl.grid;
+        while (cur + 1 < count && st >= item0[cur + 1]) ++cur;
+        if ((st - item0[cur]) % nchunks[cur] != 0) pl.partials = true;
+    }
     return pl;
 }
 
@@ -829,21 +880,123 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-template <int NT>
-static cudaError_t launch(const CUtensorMap& tc, const CUtensorMap& tx, const GemmParams& p,
-                          cudaStream_t s) {
+// Argument checks of one matrix (no CUDA call).
+static pq_status_t check_problem(int64_t m, const pq_gemm_problem_t& pr) {
+    if (m < 1 || m > 128 || pr.n < 1 || pr.k < kMinK || pr.k % kMinK) return PQ_ERR_INVALID_ARG;
+    if (pr.n > (int64_t{1} << 30) || pr.k > (int64_t{1} << 30)) return PQ_ERR_INVALID_ARG;
+    if (!pr.x_bf16 || !pr.packed || !pr.alpha || !pr.y_bf16) return PQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(pr.x_bf16) & 15) ||
+        (reinterpret_cast<uintptr_t>(pr.packed) & 15) || (reinterpret_cast<uintptr_t>(pr.y_bf16) & 1))
+        return PQ_ERR_MISALIGNED;
+    return PQ_OK;
+}
+
+// Tensor maps of one matrix: codes [n rows][k/4 bytes] in boxes of 127 rows
+// x 128 B, activations [m rows][k] in boxes of nt rows x 64 K, both with the
+// 128B swizzle the MMA and the decoders read.
+static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt,
+                        const pq_gemm_problem_t& pr, Problem& out) {
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k / 4), static_cast<cuuint64_t>(pr.n)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.k / 4)};
+        const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kFeat)};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&out.tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(pr.packed), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k), static_cast<cuuint64_t>(m)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.k * 2)};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(nt)};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&out.tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(pr.x_bf16), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+template <int NT, int MAXP>
+static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     using L = Layout<NT>;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         const cudaError_t e = cudaFuncSetAttribute(
-            wq_gemm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+            wq_gemm_kernel<NT, MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    wq_gemm_kernel<NT><<<p.grid, kThreads, L::kBytes, s>>>(tc, tx, p);
+    wq_gemm_kernel<NT, MAXP><<<prm.c.grid, kThreads, L::kBytes, s>>>(prm);
     return cudaGetLastError();
+}
+
+static int64_t workspace_bytes(int q, int64_t m, const pq_gemm_problem_t* pr, int count) {
+    float P, Q;
+    if (!coeffs_of(q, P, Q) || count < 1 || count > kMaxBatch || !pr) return -1;
+    for (int i = 0; i < count; ++i) {
+        if (m < 1 || m > 128 || pr[i].n < 1 || pr[i].k < kMinK || pr[i].k % kMinK ||
+            pr[i].n > (int64_t{1} << 30) || pr[i].k > (int64_t{1} << 30))
+            return -1;
+    }
+    int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks);
+    if (!pl.partials) return 0;
+    return partial_bytes(pl, m) + pl.blocks * 4;
+}
+
+template <int MAXP>
+static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count, void* workspace,
+                       int64_t ws_bytes, cudaStream_t s) {
+    GemmParams<MAXP> P{};  // the kernel's parameters (tensor maps included)
+    if (!coeffs_of(q, P.c.P, P.c.Q)) return PQ_ERR_UNSUPPORTED;
+    if (count < 1 || count > MAXP || !pr) return PQ_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const pq_status_t st = check_problem(m, pr[i]);
+        if (st != PQ_OK) return st;
+    }
+    int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks);
+    const int64_t need = pl.partials ? partial_bytes(pl, m) + pl.blocks * 4 : 0;
+    P.c.m = m;
+    P.c.m4 = (m + 3) / 4 * 4;
+    P.c.items = pl.items;
+    P.c.grid = pl.grid;
+    P.c.count = count;
+    if (need > 0) {
+        if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+            return PQ_ERR_INVALID_ARG;
+        P.c.partial = static_cast<float*>(workspace);
+        P.c.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes(pl, m));
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return PQ_ERR_CUDA;
+    for (int i = 0; i < count; ++i) {
+        Problem& d = P.prob[i];
+        if (!encode_maps(enc, m, pl.nt, pr[i], d)) return PQ_ERR_CUDA;
+        d.alpha = pr[i].alpha;
+        d.y = pr[i].y_bf16;
+        d.n = pr[i].n;
+        d.k = pr[i].k;
+        d.nchunks = nchunks[i];
+        d.item0 = item0[i];
+        d.block0 = block0[i];
+    }
+    if (need > 0 &&
+        cudaMemsetAsync(P.c.counters, 0, static_cast<size_t>(pl.blocks) * 4, s) != cudaSuccess)
+        return PQ_ERR_CUDA;
+    cudaError_t e;
+    switch (pl.nt) {
+        case 16: e = launch<16, MAXP>(P, s); break;
+        case 32: e = launch<32, MAXP>(P, s); break;
+        case 64: e = launch<64, MAXP>(P, s); break;
+        default: e = launch<128, MAXP>(P, s); break;
+    }
+    return e == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
 
 }  // namespace pqg
@@ -853,77 +1006,35 @@ using namespace pqg;
 extern "C" {
 
 int64_t pq_wq_gemm_workspace_bytes(pq_quant_t q, int64_t m, int64_t n, int64_t k) {
-    float P, Q;
-    if (!coeffs_of(q, P, Q) || m < 1 || m > 128 || n < 1 || k < kMinK || k % kMinK) return -1;
-    const Plan pl = plan(m, n, k);
-    if (!pl.partials) return 0;
-    return partial_bytes(pl, m) + pl.nblocks * 4;
+    pq_gemm_problem_t pr = {};
+    pr.n = n;
+    pr.k = k;
+    return workspace_bytes(q, m, &pr, 1);
+}
+
+int64_t pq_wq_gemm_batch_workspace_bytes(pq_quant_t q, int64_t m, int32_t count,
+                                         const pq_gemm_problem_t* problems) {
+    return workspace_bytes(q, m, problems, count);
 }
 
 pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k, const uint16_t* x_bf16,
                        const uint8_t* packed, const float* alpha, uint16_t* y_bf16, void* workspace,
                        int64_t workspace_bytes, void* stream) {
-    GemmParams p = {};
-    if (!coeffs_of(q, p.P, p.Q)) return PQ_ERR_UNSUPPORTED;
-    if (m < 1 || m > 128 || n < 1 || k < kMinK || k % kMinK) return PQ_ERR_INVALID_ARG;
-    if (n > (int64_t{1} << 30) || k > (int64_t{1} << 30)) return PQ_ERR_INVALID_ARG;
-    if (!x_bf16 || !packed || !alpha || !y_bf16) return PQ_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) || (reinterpret_cast<uintptr_t>(packed) & 15) ||
-        (reinterpret_cast<uintptr_t>(y_bf16) & 1))
-        return PQ_ERR_MISALIGNED;
-    const Plan pl = plan(m, n, k);
-    const int64_t need = pq_wq_gemm_workspace_bytes(q, m, n, k);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    p.alpha = alpha;
-    p.y = y_bf16;
-    p.m = m;
-    p.n = n;
-    p.k = k;
-    p.m4 = (m + 3) / 4 * 4;
-    p.nblocks = pl.nblocks;
-    p.nchunks = pl.nchunks;
-    p.items = pl.items;
-    p.grid = pl.grid;
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
-            return PQ_ERR_INVALID_ARG;
-        p.partial = static_cast<float*>(workspace);
-        p.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes(pl, m));
-    }
-    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-    if (!enc) return PQ_ERR_CUDA;
-    CUtensorMap tc, tx;
-    {  // codes [n rows][k/4 bytes]: boxes of 127 rows x 128 B, 128B swizzle
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 4), static_cast<cuuint64_t>(n)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 4)};
-        const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kFeat)};
-        const cuuint32_t es[2] = {1, 1};
-        if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
-                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return PQ_ERR_CUDA;
-    }
-    {  // activations [m rows][k bf16]: boxes of NT rows x 64 K, 128B swizzle
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(m)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k * 2)};
-        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pl.nt)};
-        const cuuint32_t es[2] = {1, 1};
-        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x_bf16), dims,
-                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return PQ_ERR_CUDA;
-    }
-    if (need > 0 &&
-        cudaMemsetAsync(p.counters, 0, static_cast<size_t>(pl.nblocks) * 4, s) != cudaSuccess)
-        return PQ_ERR_CUDA;
-    cudaError_t e;
-    switch (pl.nt) {
-        case 16: e = launch<16>(tc, tx, p, s); break;
-        case 32: e = launch<32>(tc, tx, p, s); break;
-        case 64: e = launch<64>(tc, tx, p, s); break;
-        default: e = launch<128>(tc, tx, p, s); break;
-    }
-    return e == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
+    pq_gemm_problem_t pr;
+    pr.n = n;
+    pr.k = k;
+    pr.x_bf16 = x_bf16;
+    pr.packed = packed;
+    pr.alpha = alpha;
+    pr.y_bf16 = y_bf16;
+    return run<1>(q, m, &pr, 1, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+pq_status_t pq_wq_gemm_batch(pq_quant_t q, int64_t m, int32_t count,
+                             const pq_gemm_problem_t* problems, void* workspace,
+                             int64_t workspace_bytes, void* stream) {
+    return run<kMaxBatch>(q, m, problems, count, workspace, workspace_bytes,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int pq_device_status(void) {

@@ -77,6 +77,13 @@ class PQShard(ctypes.Structure):
                 ("grad_scale", ctypes.c_float)]
 
 
+class PQGemmProblem(ctypes.Structure):
+    """``pq_gemm_problem_t``: one matrix of a grouped weight-only matmul."""
+    _fields_ = [("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("x_bf16", ctypes.c_void_p), ("packed", ctypes.c_void_p),
+                ("alpha", ctypes.c_void_p), ("y_bf16", ctypes.c_void_p)]
+
+
 def _declare(L):
     i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.pq_fakequant_fwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
@@ -92,6 +99,10 @@ def _declare(L):
     L.pq_reduce_bwd_adamw.restype = i32
     L.pq_wq_gemm.argtypes = [i32, i64, i64, i64, p, p, p, p, p, i64, p]
     L.pq_wq_gemm.restype = i32
+    L.pq_wq_gemm_batch.argtypes = [i32, i64, i32, ctypes.POINTER(PQGemmProblem), p, i64, p]
+    L.pq_wq_gemm_batch.restype = i32
+    L.pq_wq_gemm_batch_workspace_bytes.argtypes = [i32, i64, i32, ctypes.POINTER(PQGemmProblem)]
+    L.pq_wq_gemm_batch_workspace_bytes.restype = i64
     L.pq_wq_gemm_noalloc.argtypes = [i32, i64, i64, i64, p, p, p, p, p]
     L.pq_wq_gemm_noalloc.restype = i32
     L.pq_wq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]
@@ -313,6 +324,45 @@ def pq_wq_gemm(q, x, packed, alpha, y_out, workspace=None, stream=None):
     _check("pq_wq_gemm", lib().pq_wq_gemm(
         q, m, n, k, _ptr(x), _ptr(packed), _ptr(alpha), _ptr(y_out), _ptr(workspace),
         ws_bytes, _stream(stream)))
+
+
+def gemm_problem_array(descs):
+    """Build a ``pq_gemm_problem_t[]`` from dicts with keys x (bf16 [m, k]),
+    packed (uint8 [n, k/4]), alpha (fp32 [n]) and y (bf16 [m, n])."""
+    arr = (PQGemmProblem * len(descs))()
+    for i, d in enumerate(descs):
+        pr = arr[i]
+        pr.n, pr.k = int(d["packed"].shape[0]), int(d["x"].shape[1])
+        pr.x_bf16, pr.packed = _ptr(d["x"]), _ptr(d["packed"])
+        pr.alpha, pr.y_bf16 = _ptr(d["alpha"]), _ptr(d["y"])
+    return arr
+
+
+def pq_wq_gemm_batch_workspace_bytes(q, m, problems) -> int:
+    return int(lib().pq_wq_gemm_batch_workspace_bytes(q, m, len(problems), problems))
+
+
+def pq_wq_gemm_batch(q, m, problems, workspace=None, stream=None):
+    """Grouped weight-only matmul over a ``pq_gemm_problem_t[]`` (see
+    ``gemm_problem_array``); all matrices share q and the activation rows m."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pq_wq_gemm_batch", lib().pq_wq_gemm_batch(
+        q, m, len(problems), problems, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def wq_gemm_batch(q, xs, packeds, alphas, stream=None):
+    """Allocate outputs and workspace and run pq_wq_gemm_batch; returns the
+    list of Y (bf16 [m, n])."""
+    m = xs[0].shape[0]
+    ys = [torch.empty((m, pk.shape[0]), dtype=torch.bfloat16, device=pk.device) for pk in packeds]
+    arr = gemm_problem_array([dict(x=x, packed=pk, alpha=a, y=y)
+                              for x, pk, a, y in zip(xs, packeds, alphas, ys)])
+    need = pq_wq_gemm_batch_workspace_bytes(q, m, arr)
+    if need < 0:
+        raise PQError("pq_wq_gemm_batch_workspace_bytes", PQ_ERR_INVALID_ARG)
+    ws = torch.empty(need, dtype=torch.uint8, device=xs[0].device) if need > 0 else None
+    pq_wq_gemm_batch(q, m, arr, ws, stream)
+    return ys
 
 
 WQ_GEMM_NOALLOC_SCRATCH_BYTES = 8 << 20  # PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES

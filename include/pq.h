@@ -328,6 +328,34 @@ PQ_API pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k,
  * unsupported quantizer or shape. */
 PQ_API int64_t pq_wq_gemm_workspace_bytes(pq_quant_t q, int64_t m, int64_t n, int64_t k);
 
+/* One matrix of a grouped weight-only matmul: Y = X (alpha * levels)^T with
+ * the layouts and alignment of pq_wq_gemm; all matrices of a call share the
+ * quantizer and the activation rows m (each may have its own X). */
+typedef struct {
+    int64_t n, k;               /* weight rows and columns (k a multiple of 128) */
+    const uint16_t* x_bf16;     /* [m, k] bf16, 16-byte aligned */
+    const uint8_t* packed;      /* [n, k/4] codes, 16-byte aligned */
+    const float* alpha;         /* [n] */
+    uint16_t* y_bf16;           /* [m, n] bf16, overwritten */
+} pq_gemm_problem_t;
+
+/* pq_wq_gemm over 1..64 matrices in one launch: their (row block, K chunk)
+ * work items are split evenly over the GPU's SMs as one list, so the fixed
+ * cost of a launch (pipeline fill, epilogue) is paid once for the group.
+ * `problems` is a host array of `count` entries, read before the call
+ * returns. Results equal separate pq_wq_gemm calls within rounding (the
+ * split of K into partial sums may differ) and are deterministic.
+ * Workspace: pq_wq_gemm_batch_workspace_bytes(...) bytes, 256-byte aligned
+ * (NULL when 0); calls sharing a workspace must not overlap on the GPU.
+ * count outside 1..64 or any bad matrix: PQ_ERR_INVALID_ARG, nothing run. */
+PQ_API pq_status_t pq_wq_gemm_batch(pq_quant_t q, int64_t m, int32_t count,
+                                    const pq_gemm_problem_t* problems, void* workspace,
+                                    int64_t workspace_bytes, void* stream);
+
+/* Workspace bytes pq_wq_gemm_batch needs (0: none), -1 if invalid. */
+PQ_API int64_t pq_wq_gemm_batch_workspace_bytes(pq_quant_t q, int64_t m, int32_t count,
+                                                const pq_gemm_problem_t* problems);
+
 /* Upper limit on the split-K scratch pq_wq_gemm_noalloc can use (8 MiB). */
 #define PQ_WQ_GEMM_NOALLOC_SCRATCH_BYTES (8LL << 20)
 

@@ -78,3 +78,56 @@ def test_wq_gemm_rejects_bad_arguments():
     with pytest.raises(pq.PQError):  # 4-bit codes are not served
         pq.pq_wq_gemm(pq.PQ_LSQ4, torch.zeros((4, 256), dtype=torch.bfloat16, device=DEV),
                       torch.zeros((128, 128), dtype=torch.uint8, device=DEV), a, y)
+
+
+def test_wq_gemm_batch_matches_oracle():
+    """One launch over matrices of different shapes (same m), including a
+    ragged n, a short K tail and a matrix smaller than one row block."""
+    q, m = pq.PQ_SEQ2, 5
+    shapes = [(4096, 4096), (1000, 640), (100, 128), (14336, 4096), (300, 14336), (127, 512)]
+    xs, pks, als = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        x, packed, a = _case(q, m, n, k, seed=100 + i)
+        xs.append(x)
+        pks.append(packed)
+        als.append(a)
+    ys = pq.wq_gemm_batch(q, xs, pks, als)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    for x, packed, a, y in zip(xs, pks, als, ys):
+        _check(q, x, packed, a, y)
+
+
+@pytest.mark.parametrize("q", [pq.PQ_TERNARY, pq.PQ_SEQ2_B])
+def test_wq_gemm_batch_of_64_is_deterministic(q):
+    m = 16
+    shapes = [(1024 + 127 * (i % 5), 512 * (1 + i % 4)) for i in range(64)]
+    xs, pks, als = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        x, packed, a = _case(q, m, n, k, seed=7 * i + 1)
+        xs.append(x)
+        pks.append(packed)
+        als.append(a)
+    y1 = pq.wq_gemm_batch(q, xs, pks, als)
+    y2 = pq.wq_gemm_batch(q, xs, pks, als)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    for a_, b_ in zip(y1, y2):
+        assert torch.equal(a_.view(torch.int16), b_.view(torch.int16))
+    for i in (0, 17, 63):
+        _check(q, xs[i], pks[i], als[i], y1[i])
+
+
+def test_wq_gemm_batch_rejects_bad_counts():
+    q = pq.PQ_SEQ2
+    x = torch.zeros((2, 128), dtype=torch.bfloat16, device=DEV)
+    packed = torch.zeros((127, 32), dtype=torch.uint8, device=DEV)
+    a = torch.ones(127, device=DEV)
+    y = torch.empty((2, 127), dtype=torch.bfloat16, device=DEV)
+    one = dict(x=x, packed=packed, alpha=a, y=y)
+    with pytest.raises(pq.PQError):
+        pq.pq_wq_gemm_batch(q, 2, pq.gemm_problem_array([one] * 65))
+    bad = dict(one)
+    bad["x"] = torch.zeros((2, 200), dtype=torch.bfloat16, device=DEV)  # k not a multiple of 128
+    with pytest.raises(pq.PQError):
+        pq.pq_wq_gemm_batch(q, 2, pq.gemm_problem_array([one, bad]))
