@@ -71,6 +71,8 @@ constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
 
 // nonzero after a bounded wait gave up (read by pq_device_status)
 __device__ int g_status = 0;
+// iteration cap of the waits that may give up (drains keep kMaxSpins)
+__device__ uint32_t g_wait_spins = kMaxSpins;
 
 // One matrix of a launch: its tensor maps, outputs and place in the work list.
 struct Problem {
@@ -178,7 +180,8 @@ __device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity) {
 // early when another role raised the abort flag; raises it (and the device
 // status) when the spin limit is reached.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < kMaxSpins; ++i) {
+    const uint32_t cap = g_wait_spins;
+    for (uint32_t i = 0; i < cap; ++i) {
         if (mbar_try(mbar, parity)) return true;
         if ((i & 63u) == 63u && *abort) return false;
     }
@@ -1039,12 +1042,18 @@ pq_status_t pq_wq_gemm_batch(pq_quant_t q, int64_t m, int32_t count,
 
 int pq_device_status(void) {
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return PQ_ERR_CUDA;
     if (v) {
         const int zero = 0;
         cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+        return PQ_ERR_TIMEOUT;
     }
-    return v;
+    return PQ_OK;
+}
+
+pq_status_t pq_set_wait_spins(uint32_t spins) {
+    const uint32_t v = spins ? spins : kMaxSpins;
+    return cudaMemcpyToSymbol(g_wait_spins, &v, sizeof(v)) == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
 
 }  // extern "C"

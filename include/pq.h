@@ -388,9 +388,20 @@ PQ_API pq_status_t pq_wq_gemm_noalloc(pq_quant_t q, int64_t m, int64_t n, int64_
                                       const uint16_t* x_bf16, const uint8_t* packed,
                                       const float* alpha, uint16_t* y_bf16, void* stream);
 
-/* Device status of the library's bounded waits: 0 if none gave up since
- * the last call, else nonzero (and cleared). Synchronises the device. */
+/* Device status of the library's bounded waits (the weight-only matmul
+ * waits on mbarriers; every wait has an iteration cap): PQ_OK if none gave
+ * up since the last call, PQ_ERR_TIMEOUT if one did (the status is then
+ * cleared), PQ_ERR_CUDA if the status could not be read. A kernel whose wait
+ * gave up stops all its roles, lets its copies and MMAs in flight finish,
+ * frees its tensor memory and returns; its outputs are then undefined and
+ * the CUDA context stays usable. Synchronises the device. */
 PQ_API int pq_device_status(void);
+
+/* Iteration cap of the waits above (0 restores the default, a few seconds
+ * in all). A small cap makes waits give up before their data arrives, which
+ * exercises the timeout path; waits for copies and MMAs already in flight
+ * keep the default cap. Applies to later launches on the current device. */
+PQ_API pq_status_t pq_set_wait_spins(uint32_t spins);
 
 /* Storage width in bits of one packed code: 2 (binary, ternary, SEQ2,
  * SEQ2_B, LSQ2) or 4 (LSQ3, LSQ4); 0 for an unknown quantizer. */

@@ -131,3 +131,24 @@ def test_wq_gemm_batch_rejects_bad_counts():
     bad["x"] = torch.zeros((2, 200), dtype=torch.bfloat16, device=DEV)  # k not a multiple of 128
     with pytest.raises(pq.PQError):
         pq.pq_wq_gemm_batch(q, 2, pq.gemm_problem_array([one, bad]))
+
+
+def test_wq_gemm_wait_timeout_reports_and_recovers():
+    """With a wait cap of one try, the kernel's waits give up before their
+    data arrives: the device status says PQ_ERR_TIMEOUT once, and with the
+    default cap restored the next call is correct (the context is usable)."""
+    q = pq.PQ_SEQ2
+    x, packed, a = _case(q, 1, 127 * 148, 4096, seed=11)
+    assert pq.pq_device_status() == pq.PQ_OK
+    try:
+        pq.pq_set_wait_spins(1)
+        pq.wq_gemm(q, x, packed, a)
+        torch.cuda.synchronize()
+    finally:
+        pq.pq_set_wait_spins(0)
+    assert pq.pq_device_status() == pq.PQ_ERR_TIMEOUT
+    assert pq.pq_device_status() == pq.PQ_OK  # cleared by the read
+    y = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == pq.PQ_OK
+    _check(q, x, packed, a, y)
