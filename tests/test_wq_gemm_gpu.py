@@ -152,3 +152,34 @@ def test_wq_gemm_wait_timeout_reports_and_recovers():
     torch.cuda.synchronize()
     assert pq.pq_device_status() == pq.PQ_OK
     _check(q, x, packed, a, y)
+
+
+def _check_rows(q, x, packed, a, y, rows):
+    """_check on a subset of output features (the oracle runs on those rows)."""
+    k = x.shape[1]
+    idx = torch.as_tensor(rows, device=packed.device)
+    _check(q, x, packed.index_select(0, idx).contiguous(), a.index_select(0, idx).contiguous(),
+           y.index_select(1, idx).contiguous())
+
+
+def test_wq_gemm_full_size_grouped_sampled():
+    """One Llama-3-8B layer at full size plus a 16384^2 weight, in one grouped
+    launch at m = 16 (the benchmark's launch configuration); 64 sampled
+    output features of every matrix (first and last included) against the
+    oracle."""
+    q, m = pq.PQ_SEQ2, 16
+    shapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096),
+              (14336, 4096), (4096, 14336), (16384, 16384)]
+    xs, pks, als = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        x, packed, a = _case(q, m, n, k, seed=900 + i)
+        xs.append(x)
+        pks.append(packed)
+        als.append(a)
+    ys = pq.wq_gemm_batch(q, xs, pks, als)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == pq.PQ_OK
+    rng = np.random.default_rng(5)
+    for (n, k), x, packed, a, y in zip(shapes, xs, pks, als, ys):
+        rows = sorted(set([0, n - 1] + list(rng.choice(n, 62, replace=False))))
+        _check_rows(q, x, packed, a, y, rows)
