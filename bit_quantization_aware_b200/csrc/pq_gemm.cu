@@ -800,6 +800,155 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
 }
 
+// ------------------------------------------------- one activation row
+// For m = 1 the tensor cores retire at most 2048 weights per ~46-cycle MMA
+// per SM, far below what the codes' bandwidth allows, so a single row takes
+// a CUDA-core path: each weight is decoded to the fp32 value 1 + f'/4 (one
+// shift and one logic op) and multiplied into paired fp32 accumulators
+// (two FMAs per instruction); the same affine identity gives
+// y = alpha * (P * D + Q * Sx). x is held in shared memory as fp32 (each
+// CTA converts it once per matrix and sums it in a fixed order); warps take
+// tasks of 1, 2 or 4 rows from a per-matrix counter; lane l reads 16-byte chunks
+// l, l + 32, ... of each row, so every load of a warp is 512 contiguous
+// bytes; a fixed shuffle tree sums a row's lane partials (deterministic).
+namespace pqv {
+
+constexpr int kThreads = 512;
+constexpr int64_t kMaxK = 32768;         // x as fp32 in shared memory: 128 KB
+
+struct VecProblem {
+    const uint16_t* x;   // [k] bf16
+    const uint8_t* codes;  // [n, k/4]
+    const float* alpha;  // [n]
+    uint16_t* y;         // [n] bf16
+    int64_t n, k;
+    int* counter;        // task counter, zero on entry
+    int32_t rows;        // rows per task: 1, 2 or 4 (about one task per warp or more)
+};
+
+template <int MAXP>
+struct VecParams {
+    int32_t count;
+    float P, Q;
+    VecProblem prob[MAXP];
+};
+
+// Field j (0..15) of a code word as the fp32 value 1 + f'/4, f' = field xor 2.
+template <int J>
+__device__ __forceinline__ float dec32(uint32_t w) {
+    const uint32_t s = J <= 10 ? (w << (21 - 2 * J)) : (w >> (2 * J - 21));
+    return __uint_as_float(((s & 0x00600000u) ^ 0x00400000u) | 0x3F800000u);
+}
+
+// acc += x[0..15] * fields of w (x as 8 float2 pairs)
+__device__ __forceinline__ float2 word_fma(uint32_t w, const float2* x, float2 acc) {
+    acc = __ffma2_rn(x[0], make_float2(dec32<0>(w), dec32<1>(w)), acc);
+    acc = __ffma2_rn(x[1], make_float2(dec32<2>(w), dec32<3>(w)), acc);
+    acc = __ffma2_rn(x[2], make_float2(dec32<4>(w), dec32<5>(w)), acc);
+    acc = __ffma2_rn(x[3], make_float2(dec32<6>(w), dec32<7>(w)), acc);
+    acc = __ffma2_rn(x[4], make_float2(dec32<8>(w), dec32<9>(w)), acc);
+    acc = __ffma2_rn(x[5], make_float2(dec32<10>(w), dec32<11>(w)), acc);
+    acc = __ffma2_rn(x[6], make_float2(dec32<12>(w), dec32<13>(w)), acc);
+    acc = __ffma2_rn(x[7], make_float2(dec32<14>(w), dec32<15>(w)), acc);
+    return acc;
+}
+
+// One task: rows task*R .. task*R + R - 1 of a matrix, whole K; lane l
+// takes 16-byte code chunks l, l + 32, ...; x from shared memory is reused
+// by the R rows.
+template <int R>
+__device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t kq, int64_t nchunk,
+                                         int lane, float P, float qsx, const float4* xs4) {
+    const int64_t row0 = static_cast<int64_t>(task) * R;
+    const uint8_t* rp[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t row = row0 + r < pb.n ? row0 + r : pb.n - 1;
+        rp[r] = pb.codes + row * kq;
+    }
+    float2 acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = make_float2(0.0f, 0.0f);
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        uint4 w[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) w[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + c * 16));
+        const float4* xc = xs4 + c * 16;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float2 xv[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 f = xc[(4 * q4 + u + c) & 15];
+                xv[2 * u] = make_float2(f.x, f.y);
+                xv[2 * u + 1] = make_float2(f.z, f.w);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint32_t word = q4 == 0 ? w[r].x : q4 == 1 ? w[r].y : q4 == 2 ? w[r].z : w[r].w;
+                acc[r] = word_fma(word, xv, acc[r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float d = __fadd_rn(acc[r].x, acc[r].y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d = __fadd_rn(d, __shfl_xor_sync(0xFFFFFFFFu, d, o));
+        const int64_t row = row0 + r;
+        if (lane == r && row < pb.n)
+            pb.y[row] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldg(pb.alpha + row) * fmaf(P, d, qsx)));
+    }
+}
+
+template <int MAXP>
+__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const __grid_constant__ VecParams<MAXP> prm) {
+    extern __shared__ float4 xs4[];  // per 64-K chunk c: 16 float4 slots, slot s at (s + c) & 15
+    __shared__ float warp_sum[kThreads / 32];
+    __shared__ float sx_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int pi = 0; pi < prm.count; ++pi) {
+        const VecProblem& pb = prm.prob[pi];
+        const int64_t nq = pb.k / 4;  // float4 slots of x
+        // x -> fp32 shared memory (swizzled per chunk) and its sum
+        float part = 0.0f;
+        for (int64_t i = tid; i < nq; i += kThreads) {
+            const uint2 h = __ldg(reinterpret_cast<const uint2*>(pb.x) + i);
+            const float4 v = make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xFFFF0000u),
+                                         __uint_as_float(h.y << 16), __uint_as_float(h.y & 0xFFFF0000u));
+            const int64_t c = i >> 4, sl = i & 15;
+            xs4[c * 16 + ((sl + c) & 15)] = v;
+            part = __fadd_rn(__fadd_rn(part, v.x), __fadd_rn(v.y, __fadd_rn(v.z, v.w)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xFFFFFFFFu, part, o));
+        if (lane == 0) warp_sum[warp] = part;
+        __syncthreads();
+        if (tid == 0) {
+            float t = 0.0f;
+            for (int w = 0; w < kThreads / 32; ++w) t = __fadd_rn(t, warp_sum[w]);
+            sx_sh = t;
+        }
+        __syncthreads();
+        const float sx = sx_sh;
+        const float qsx = prm.Q * sx;
+        const int64_t kq = pb.k / 4, nchunk = pb.k / 64;
+        const int64_t ntasks = (pb.n + pb.rows - 1) / pb.rows;
+        for (;;) {
+            int task = 0;
+            if (lane == 0) task = atomicAdd(pb.counter, 1);
+            task = __shfl_sync(0xFFFFFFFFu, task, 0);
+            if (task >= ntasks) break;
+            if (pb.rows == 4) row_task<4>(pb, task, kq, nchunk, lane, prm.P, qsx, xs4);
+            else if (pb.rows == 2) row_task<2>(pb, task, kq, nchunk, lane, prm.P, qsx, xs4);
+            else row_task<1>(pb, task, kq, nchunk, lane, prm.P, qsx, xs4);
+        }
+        __syncthreads();  // the next matrix overwrites x
+    }
+}
+
+}  // namespace pqv
+
 // ------------------------------------------------------------------- host
 
 static int sm_count() {
@@ -938,6 +1087,61 @@ static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// A single activation row with x fitting shared memory takes the CUDA-core path.
+static bool vector_path(int64_t m, const pq_gemm_problem_t* pr, int count) {
+    if (m != 1) return false;
+    for (int i = 0; i < count; ++i)
+        if (pr[i].k > pqv::kMaxK) return false;
+    return true;
+}
+
+template <int MAXP>
+static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, void* workspace,
+                              int64_t ws_bytes, cudaStream_t s) {
+    pqv::VecParams<MAXP> V{};
+    if (!coeffs_of(q, V.P, V.Q)) return PQ_ERR_UNSUPPORTED;
+    if (!workspace || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return PQ_ERR_INVALID_ARG;
+    int* counters = static_cast<int*>(workspace);
+    int64_t maxk = 0;
+    for (int i = 0; i < count; ++i) {
+        V.prob[i].x = pr[i].x_bf16;
+        V.prob[i].codes = pr[i].packed;
+        V.prob[i].alpha = pr[i].alpha;
+        V.prob[i].y = pr[i].y_bf16;
+        V.prob[i].n = pr[i].n;
+        V.prob[i].k = pr[i].k;
+        V.prob[i].counter = counters + i;
+        if (pr[i].k > maxk) maxk = pr[i].k;
+    }
+    V.count = count;
+    const size_t smem = static_cast<size_t>(maxk) * 4;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(pqv::gemv_kernel<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(pqv::kMaxK * 4)) != cudaSuccess)
+            return PQ_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pqv::gemv_kernel<MAXP>, pqv::kThreads,
+                                                      smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    // rows per task (x loads are shared by the rows of a task): a lone
+    // matrix takes the largest of 4, 2, 1 that still gives about one task
+    // per warp of the grid; a group takes 4 (measured best: its matrices
+    // follow one another, so fewer instructions per weight win there)
+    const int64_t warps = static_cast<int64_t>(sm_count()) * per_sm * (pqv::kThreads / 32);
+    for (int i = 0; i < count; ++i)
+        V.prob[i].rows = count > 1 ? 4 : pr[i].n >= 4 * warps ? 4 : pr[i].n >= 2 * warps ? 2 : 1;
+    if (cudaMemsetAsync(counters, 0, static_cast<size_t>(count) * 4, s) != cudaSuccess)
+        return PQ_ERR_CUDA;
+    pqv::gemv_kernel<MAXP><<<sm_count() * per_sm, pqv::kThreads, smem, s>>>(V);
+    return cudaGetLastError() == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
+}
+
 static int64_t workspace_bytes(int q, int64_t m, const pq_gemm_problem_t* pr, int count) {
     float P, Q;
     if (!coeffs_of(q, P, Q) || count < 1 || count > kMaxBatch || !pr) return -1;
@@ -946,6 +1150,7 @@ static int64_t workspace_bytes(int q, int64_t m, const pq_gemm_problem_t* pr, in
             pr[i].n > (int64_t{1} << 30) || pr[i].k > (int64_t{1} << 30))
             return -1;
     }
+    if (vector_path(m, pr, count)) return 256;  // one task counter per matrix
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
     const Plan pl = plan(m, pr, count, item0, block0, nchunks);
     if (!pl.partials) return 0;
@@ -962,6 +1167,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         const pq_status_t st = check_problem(m, pr[i]);
         if (st != PQ_OK) return st;
     }
+    if (vector_path(m, pr, count)) return run_vector<MAXP>(q, pr, count, workspace, ws_bytes, s);
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
     const Plan pl = plan(m, pr, count, item0, block0, nchunks);
     const int64_t need = pl.partials ? partial_bytes(pl, m) + pl.blocks * 4 : 0;

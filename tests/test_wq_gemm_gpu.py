@@ -47,7 +47,8 @@ def _check(q, x, packed, a, y):
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (5, 300, 256), (16, 1024, 4096),
                                    (33, 640, 1024), (64, 2048, 2048), (128, 256, 512),
                                    (7, 4096, 14336), (20, 1000, 640), (3, 130, 384),
-                                   (100, 509, 1536)])
+                                   (100, 509, 1536), (1, 300, 640), (1, 5, 128),
+                                   (1, 14336, 4096), (1, 64, 32896)])
 def test_wq_gemm_matches_oracle(q, m, n, k):
     x, packed, a = _case(q, m, n, k, seed=m + n + k)
     y = pq.wq_gemm(q, x, packed, a)
@@ -138,7 +139,7 @@ def test_wq_gemm_wait_timeout_reports_and_recovers():
     data arrives: the device status says PQ_ERR_TIMEOUT once, and with the
     default cap restored the next call is correct (the context is usable)."""
     q = pq.PQ_SEQ2
-    x, packed, a = _case(q, 1, 127 * 148, 4096, seed=11)
+    x, packed, a = _case(q, 2, 127 * 148, 4096, seed=11)  # m > 1: the tensor-core path
     assert pq.pq_device_status() == pq.PQ_OK
     try:
         pq.pq_set_wait_spins(1)
@@ -183,3 +184,23 @@ def test_wq_gemm_full_size_grouped_sampled():
     for (n, k), x, packed, a, y in zip(shapes, xs, pks, als, ys):
         rows = sorted(set([0, n - 1] + list(rng.choice(n, 62, replace=False))))
         _check_rows(q, x, packed, a, y, rows)
+
+
+def test_wq_gemm_batch_single_row_matches_oracle():
+    """One activation row (the CUDA-core path) over matrices of several
+    shapes in one launch."""
+    q, m = pq.PQ_SEQ2_B, 1
+    shapes = [(4096, 4096), (1000, 640), (7, 128), (14336, 4096), (300, 14336)]
+    xs, pks, als = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        x, packed, a = _case(q, m, n, k, seed=300 + i)
+        xs.append(x)
+        pks.append(packed)
+        als.append(a)
+    y1 = pq.wq_gemm_batch(q, xs, pks, als)
+    y2 = pq.wq_gemm_batch(q, xs, pks, als)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == pq.PQ_OK
+    for x, packed, a, ya, yb in zip(xs, pks, als, y1, y2):
+        assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+        _check(q, x, packed, a, ya)
