@@ -833,23 +833,30 @@ struct VecParams {
     VecProblem prob[MAXP];
 };
 
-// Field j (0..15) of a code word as the fp32 value 1 + f'/4, f' = field xor 2.
+// Field j (0..7) of a code half-word h as the fp32 value 1 + f'/4 with
+// f' = field xor 2: the field is moved to mantissa bits 21-22 by a multiply
+// (an FMA-pipe instruction, which leaves the ALU pipe to the mask), then
+// masked, its sign bit flipped, and the exponent of 1.0 set.
 template <int J>
-__device__ __forceinline__ float dec32(uint32_t w) {
-    const uint32_t s = J <= 10 ? (w << (21 - 2 * J)) : (w >> (2 * J - 21));
+__device__ __forceinline__ float dec32(uint32_t h) {
+    uint32_t s;
+    asm("mul.lo.u32 %0, %1, %2;" : "=r"(s) : "r"(h), "n"(1u << (21 - 2 * J)));
     return __uint_as_float(((s & 0x00600000u) ^ 0x00400000u) | 0x3F800000u);
 }
 
-// acc += x[0..15] * fields of w (x as 8 float2 pairs)
+// acc += x[0..15] * fields of w (x as 8 float2 pairs, paired FMAs); fields
+// 8..15 are taken from the upper half after one shift, so every field needs
+// only a left shift.
 __device__ __forceinline__ float2 word_fma(uint32_t w, const float2* x, float2 acc) {
+    const uint32_t hi = w >> 16;
     acc = __ffma2_rn(x[0], make_float2(dec32<0>(w), dec32<1>(w)), acc);
     acc = __ffma2_rn(x[1], make_float2(dec32<2>(w), dec32<3>(w)), acc);
     acc = __ffma2_rn(x[2], make_float2(dec32<4>(w), dec32<5>(w)), acc);
     acc = __ffma2_rn(x[3], make_float2(dec32<6>(w), dec32<7>(w)), acc);
-    acc = __ffma2_rn(x[4], make_float2(dec32<8>(w), dec32<9>(w)), acc);
-    acc = __ffma2_rn(x[5], make_float2(dec32<10>(w), dec32<11>(w)), acc);
-    acc = __ffma2_rn(x[6], make_float2(dec32<12>(w), dec32<13>(w)), acc);
-    acc = __ffma2_rn(x[7], make_float2(dec32<14>(w), dec32<15>(w)), acc);
+    acc = __ffma2_rn(x[4], make_float2(dec32<0>(hi), dec32<1>(hi)), acc);
+    acc = __ffma2_rn(x[5], make_float2(dec32<2>(hi), dec32<3>(hi)), acc);
+    acc = __ffma2_rn(x[6], make_float2(dec32<4>(hi), dec32<5>(hi)), acc);
+    acc = __ffma2_rn(x[7], make_float2(dec32<6>(hi), dec32<7>(hi)), acc);
     return acc;
 }
 
