@@ -4,12 +4,18 @@
         --quant seq2 --iters 3 [--pack]
     python -m bit_quantization_aware_b200.profile_case --rows 16384 --cols 16384 \
         --quant seq2 --iters 3 --gemm-m 1
+    python -m bit_quantization_aware_b200.profile_case ... --op dequant | bwd_adamw
 
 Draws seeded synthetic inputs on the device (N(0, 0.02) weights, alpha =
 max|w_row| or the quantizer's init, bf16 N(0, 1e-3) upstream gradient),
 then runs forward and backward ``iters`` times on the current stream and
 prints the per-iteration CUDA-event times. Sized by the caller; a
 14336x4096 matrix moves about 0.9 GB per iteration, more than L2.
+
+``--op dequant`` runs the packed-code dequantization instead (codes from a
+forward), ``--op bwd_adamw`` the backward fused with one AdamW step, and
+``--gemm-m M`` the weight-only matmul with M activation rows on seeded
+random codes (only codes, scales, X and Y are allocated).
 """
 from __future__ import annotations
 
@@ -30,11 +36,14 @@ def main():
     p.add_argument("--pack", action="store_true")
     p.add_argument("--gemm-m", type=int, default=0,
                    help="run the weight-only matmul with this many activation rows")
+    p.add_argument("--op", default="quantizer", choices=["quantizer", "dequant", "bwd_adamw"])
     a = p.parse_args()
     q = pq.QUANTIZERS[a.quant]
     dev = torch.device("cuda")
     if a.gemm_m:
         return gemm_case(a, q, dev)
+    if a.op != "quantizer":
+        return next_case(a, q, dev)
     w = I.normal_weights(a.rows, a.cols, seed=0, stream=0, device=dev)
     alpha = I.alpha_init(w, q)
     g = I.grad_bf16(a.rows, a.cols, seed=0, stream=64, device=dev)
@@ -58,6 +67,41 @@ def main():
         fb = 6 + (pq.pq_code_bits(q) / 8 if a.pack else 0)
         print(f"iter {i}: fwd {tf * 1e6:.1f} us ({n * fb / tf / 1e9:.0f} GB/s), "
               f"bwd {tb * 1e6:.1f} us ({n * 10 / tb / 1e9:.0f} GB/s)")
+
+
+def next_case(a, q, dev):
+    w = I.normal_weights(a.rows, a.cols, seed=0, stream=0, device=dev)
+    alpha = I.alpha_init(w, q)
+    n = a.rows * a.cols
+    if a.op == "dequant":
+        wq, packed = pq.fakequant_fwd(q, w, alpha, pack=True)
+        out = torch.empty_like(wq)
+        nbytes = n * 2 + packed.numel() + a.rows * 4
+
+        def go():
+            pq.pq_dequant_codes(q, packed, alpha, out)
+    else:
+        g = I.grad_bf16(a.rows, a.cols, seed=0, stream=64, device=dev)
+        m_w, v_w = torch.zeros_like(w), torch.zeros_like(w)
+        m_a, v_a = torch.zeros_like(alpha), torch.zeros_like(alpha)
+        arr = pq.adamw_matrix_array([dict(rows=a.rows, cols=a.cols, w=w, alpha=alpha, g=g,
+                                          m_w=m_w, v_w=v_w, m_alpha=m_a, v_alpha=v_a,
+                                          grad_scale=pq.pq_default_grad_scale(q, a.cols))])
+        nbytes = 26 * n + 24 * a.rows
+        t = [0]
+
+        def go():
+            t[0] += 1
+            pq.pq_fakequant_bwd_adamw(q, arr, pq.adamw(t[0], 2e-5), pq.adamw(t[0], 2e-5))
+    torch.cuda.synchronize()
+    for i in range(a.iters):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        go()
+        e[1].record()
+        torch.cuda.synchronize()
+        dt = e[0].elapsed_time(e[1]) * 1e-3
+        print(f"iter {i}: {a.op} {dt * 1e6:.1f} us ({nbytes / dt / 1e9:.0f} GB/s algorithmic)")
 
 
 def gemm_case(a, q, dev):
