@@ -807,14 +807,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // shift and one logic op) and multiplied into paired fp32 accumulators
 // (two FMAs per instruction); the same affine identity gives
 // y = alpha * (P * D + Q * Sx). x is held in shared memory as fp32 (each
-// CTA converts it once per matrix and sums it in a fixed order); warps take
+// CTA converts it once per matrix and sums it in a fixed order; each 64-K
+// chunk is padded so lanes reading consecutive chunks hit different banks); warps take
 // tasks of 1, 2 or 4 rows from a per-matrix counter; lane l reads 16-byte chunks
 // l, l + 32, ... of each row, so every load of a warp is 512 contiguous
 // bytes; a fixed shuffle tree sums a row's lane partials (deterministic).
 namespace pqv {
 
 constexpr int kThreads = 512;
-constexpr int64_t kMaxK = 32768;         // x as fp32 in shared memory: 128 KB
+constexpr int64_t kMaxK = 32768;         // x as fp32 in shared memory: 136 KB padded
+// 64 x values (16 float4) per chunk, padded to 17 float4: the 8 lanes of a
+// quarter-warp read 8 consecutive chunks at the same offset, 68 floats apart,
+// which falls in 8 different bank groups
+constexpr int kChunkF4 = 17;
 
 struct VecProblem {
     const uint16_t* x;   // [k] bf16
@@ -880,13 +885,13 @@ __device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t
         uint4 w[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) w[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + c * 16));
-        const float4* xc = xs4 + c * 16;
+        const float4* xc = xs4 + c * kChunkF4;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             float2 xv[8];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float4 f = xc[(4 * q4 + u + c) & 15];
+                const float4 f = xc[4 * q4 + u];
                 xv[2 * u] = make_float2(f.x, f.y);
                 xv[2 * u + 1] = make_float2(f.z, f.w);
             }
@@ -909,22 +914,21 @@ __device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t
 }
 
 template <int MAXP>
-__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const __grid_constant__ VecParams<MAXP> prm) {
-    extern __shared__ float4 xs4[];  // per 64-K chunk c: 16 float4 slots, slot s at (s + c) & 15
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const __grid_constant__ VecParams<MAXP> prm) {
+    extern __shared__ float4 xs4[];  // 64-K chunk c at float4 c * kChunkF4 (padded)
     __shared__ float warp_sum[kThreads / 32];
     __shared__ float sx_sh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int pi = 0; pi < prm.count; ++pi) {
         const VecProblem& pb = prm.prob[pi];
         const int64_t nq = pb.k / 4;  // float4 slots of x
-        // x -> fp32 shared memory (swizzled per chunk) and its sum
+        // x -> fp32 shared memory (chunks padded to 17 float4) and its sum
         float part = 0.0f;
         for (int64_t i = tid; i < nq; i += kThreads) {
             const uint2 h = __ldg(reinterpret_cast<const uint2*>(pb.x) + i);
             const float4 v = make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xFFFF0000u),
                                          __uint_as_float(h.y << 16), __uint_as_float(h.y & 0xFFFF0000u));
-            const int64_t c = i >> 4, sl = i & 15;
-            xs4[c * 16 + ((sl + c) & 15)] = v;
+            xs4[(i >> 4) * kChunkF4 + (i & 15)] = v;
             part = __fadd_rn(__fadd_rn(part, v.x), __fadd_rn(v.y, __fadd_rn(v.z, v.w)));
         }
 #pragma unroll
@@ -1122,13 +1126,13 @@ static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, voi
         if (pr[i].k > maxk) maxk = pr[i].k;
     }
     V.count = count;
-    const size_t smem = static_cast<size_t>(maxk) * 4;
+    const size_t smem = static_cast<size_t>(maxk / 64) * pqv::kChunkF4 * 16;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(pqv::gemv_kernel<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(pqv::kMaxK * 4)) != cudaSuccess)
+                                 static_cast<int>(pqv::kMaxK / 64 * pqv::kChunkF4 * 16)) != cudaSuccess)
             return PQ_ERR_CUDA;
         attr_set[dev] = true;
     }
