@@ -273,10 +273,18 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
 // lowest bits) as two bf16 values 1 + f'/4 (low half: field j), with
 // f' = f xor 2: the field lands in mantissa bits 5-6 of 1.0 and its sign
 // bit is flipped there.
+// select(b, a ^ c, c) in one three-input logic op: where the mask b is set,
+// a with the sign bits of c flipped; elsewhere the constant bits of c.
+__device__ __forceinline__ uint32_t mask_flip_or(uint32_t a, uint32_t b_imm_mask, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b_imm_mask), "r"(c));
+    return d;
+}
+
 template <int J>
 __device__ __forceinline__ uint32_t pair_of(uint32_t w) {
     const uint32_t s = J < 3 ? (w << (5 - 2 * J)) : (w >> (2 * J - 5));
-    return ((s & 0x00600060u) ^ 0x00400040u) | kOnes;
+    return mask_flip_or(s, 0x00600060u, 0x00400040u | kOnes);
 }
 
 __device__ __forceinline__ void decode_word(uint32_t w, uint32_t* v) {
@@ -846,7 +854,7 @@ template <int J>
 __device__ __forceinline__ float dec32(uint32_t h) {
     uint32_t s;
     asm("mul.lo.u32 %0, %1, %2;" : "=r"(s) : "r"(h), "n"(1u << (21 - 2 * J)));
-    return __uint_as_float(((s & 0x00600000u) ^ 0x00400000u) | 0x3F800000u);
+    return __uint_as_float(mask_flip_or(s, 0x00600000u, 0x00400000u | 0x3F800000u));
 }
 
 // acc += x[0..15] * fields of w (x as 8 float2 pairs, paired FMAs); fields
