@@ -71,8 +71,9 @@ constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
 
 // nonzero after a bounded wait gave up (read by pq_device_status)
 __device__ int g_status = 0;
-// iteration cap of the waits that may give up (drains keep kMaxSpins)
-__device__ uint32_t g_wait_spins = kMaxSpins;
+// nonzero: every launch raises its abort flag at start, so its waits give up
+// as if their cap had been reached (pq_debug_abort_waits; tests the path)
+__device__ int g_force_abort = 0;
 
 // One matrix of a launch: its tensor maps, outputs and place in the work list.
 struct Problem {
@@ -179,9 +180,10 @@ __device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity) {
 // Bounded wait for the phase of the given parity (one thread). Gives up
 // early when another role raised the abort flag; raises it (and the device
 // status) when the spin limit is reached.
+// The loop is kept to the barrier try and a periodic abort check: other
+// work in it (even a rarely executed load) measurably slowed the pipeline.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    const uint32_t cap = g_wait_spins;
-    for (uint32_t i = 0; i < cap; ++i) {
+    for (uint32_t i = 0; i < kMaxSpins; ++i) {
         if (mbar_try(mbar, parity)) return true;
         if ((i & 63u) == 63u && *abort) return false;
     }
@@ -284,7 +286,7 @@ __device__ __forceinline__ uint32_t mask_flip_or(uint32_t a, uint32_t b_imm_mask
 template <int J>
 __device__ __forceinline__ uint32_t pair_of(uint32_t w) {
     const uint32_t s = J < 3 ? (w << (5 - 2 * J)) : (w >> (2 * J - 5));
-    return mask_flip_or(s, 0x00600060u, 0x00400040u | kOnes);
+    return ((s & 0x00600060u) ^ 0x00400040u) | kOnes;
 }
 
 __device__ __forceinline__ void decode_word(uint32_t w, uint32_t* v) {
@@ -439,7 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(b_accempty + 8u * b, 4);
         }
         mbar_init(b_drain, 1);
-        *abort = 0;
+        const int forced = *static_cast<volatile int*>(&g_force_abort);
+        *abort = forced;
+        if (forced) atomicExch(&g_status, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid == kCodesWarp * 32) {
@@ -1276,9 +1280,9 @@ int pq_device_status(void) {
     return PQ_OK;
 }
 
-pq_status_t pq_set_wait_spins(uint32_t spins) {
-    const uint32_t v = spins ? spins : kMaxSpins;
-    return cudaMemcpyToSymbol(g_wait_spins, &v, sizeof(v)) == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
+pq_status_t pq_debug_abort_waits(int on) {
+    const int v = on ? 1 : 0;
+    return cudaMemcpyToSymbol(g_force_abort, &v, sizeof(v)) == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
 
 }  // extern "C"

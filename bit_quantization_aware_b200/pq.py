@@ -109,8 +109,8 @@ def _declare(L):
     L.pq_wq_gemm_workspace_bytes.restype = i64
     L.pq_device_status.argtypes = []
     L.pq_device_status.restype = i32
-    L.pq_set_wait_spins.argtypes = [ctypes.c_uint32]
-    L.pq_set_wait_spins.restype = i32
+    L.pq_debug_abort_waits.argtypes = [i32]
+    L.pq_debug_abort_waits.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
     L.pq_dequant_codes_batch.restype = i32
     L.pq_dequant_codes.argtypes = [i32, i64, i64, p, p, p, p]
@@ -397,9 +397,9 @@ def pq_device_status() -> int:
     return int(lib().pq_device_status())
 
 
-def pq_set_wait_spins(spins: int) -> None:
-    """Iteration cap of the library's bounded device waits (0 = default)."""
-    _check("pq_set_wait_spins", lib().pq_set_wait_spins(int(spins)))
+def pq_debug_abort_waits(on: bool) -> None:
+    """Test switch: later matmul launches give up their waits at once."""
+    _check("pq_debug_abort_waits", lib().pq_debug_abort_waits(1 if on else 0))
 
 
 def wq_gemm(q, x, packed, alpha, stream=None):

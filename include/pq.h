@@ -397,11 +397,12 @@ PQ_API pq_status_t pq_wq_gemm_noalloc(pq_quant_t q, int64_t m, int64_t n, int64_
  * the CUDA context stays usable. Synchronises the device. */
 PQ_API int pq_device_status(void);
 
-/* Iteration cap of the waits above (0 restores the default, a few seconds
- * in all). A small cap makes waits give up before their data arrives, which
- * exercises the timeout path; waits for copies and MMAs already in flight
- * keep the default cap. Applies to later launches on the current device. */
-PQ_API pq_status_t pq_set_wait_spins(uint32_t spins);
+/* Test switch for the timeout path: while on, every later launch of the
+ * matmul's tensor-core path raises its abort flag at start, so its waits give
+ * up as a wait that reached its cap does (roles stop, copies and MMAs in
+ * flight drain, TMEM is freed) and pq_device_status reports PQ_ERR_TIMEOUT;
+ * outputs of those launches are undefined. Off (0) by default. */
+PQ_API pq_status_t pq_debug_abort_waits(int on);
 
 /* Storage width in bits of one packed code: 2 (binary, ternary, SEQ2,
  * SEQ2_B, LSQ2) or 4 (LSQ3, LSQ4); 0 for an unknown quantizer. */

@@ -33,7 +33,7 @@ def test_header_declares_entry_points():
               "pq_scaled_weights", "pq_dequant_codes", "pq_dequant_codes_batch",
               "pq_fakequant_bwd_adamw", "pq_reduce_bwd_adamw",
               "pq_wq_gemm", "pq_wq_gemm_workspace_bytes", "pq_device_status",
-              "pq_wq_gemm_noalloc", "pq_wq_gemm_batch", "pq_wq_gemm_batch_workspace_bytes", "pq_set_wait_spins",
+              "pq_wq_gemm_noalloc", "pq_wq_gemm_batch", "pq_wq_gemm_batch_workspace_bytes", "pq_debug_abort_waits",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
               "pq_last_cuda_error"):
         assert n in names

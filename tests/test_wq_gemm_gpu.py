@@ -135,18 +135,18 @@ def test_wq_gemm_batch_rejects_bad_counts():
 
 
 def test_wq_gemm_wait_timeout_reports_and_recovers():
-    """With a wait cap of one try, the kernel's waits give up before their
-    data arrives: the device status says PQ_ERR_TIMEOUT once, and with the
-    default cap restored the next call is correct (the context is usable)."""
+    """With the abort switch on, the kernel's waits give up as a wait that
+    reached its cap does: the device status says PQ_ERR_TIMEOUT once, and
+    with the switch off the next call is correct (the context is usable)."""
     q = pq.PQ_SEQ2
     x, packed, a = _case(q, 2, 127 * 148, 4096, seed=11)  # m > 1: the tensor-core path
     assert pq.pq_device_status() == pq.PQ_OK
     try:
-        pq.pq_set_wait_spins(1)
+        pq.pq_debug_abort_waits(True)
         pq.wq_gemm(q, x, packed, a)
         torch.cuda.synchronize()
     finally:
-        pq.pq_set_wait_spins(0)
+        pq.pq_debug_abort_waits(False)
     assert pq.pq_device_status() == pq.PQ_ERR_TIMEOUT
     assert pq.pq_device_status() == pq.PQ_OK  # cleared by the read
     y = pq.wq_gemm(q, x, packed, a)
