@@ -774,7 +774,10 @@ def run_wq_gemm(args):
                 "algorithmic_flops_per_step": flops_step}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    roof["kernel"] = "pqg::wq_gemm_kernel<NT> (tcgen05.mma kind::f16, TMEM accumulator)"
+    # one activation row with k <= 32768 is served by the CUDA-core kernel
+    roof["kernel"] = ("pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)"
+                      if m == 1 and max(b.m.cols for b in step.bufs) <= 32768 else
+                      "pqg::wq_gemm_kernel<NT> (tcgen05.mma kind::f16, TMEM accumulator)")
     print(json.dumps({
         "metric": "weight-only 2-bit matmul Gweights/s", "op": "wq_gemm",
         "value": weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
