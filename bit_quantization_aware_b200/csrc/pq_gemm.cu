@@ -879,7 +879,8 @@ __device__ __forceinline__ float2 word_fma(uint32_t w, const float2* x, float2 a
 
 // One task: rows task*R .. task*R + R - 1 of a matrix, whole K; lane l
 // takes 16-byte code chunks l, l + 32, ...; x from shared memory is reused
-// by the R rows.
+// by the R rows. The loads of a lane's next chunk are issued before the
+// current one is computed, so a load's latency overlaps a chunk of math.
 template <int R>
 __device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t kq, int64_t nchunk,
                                          int lane, float P, float qsx, const float4* xs4) {
@@ -893,10 +894,17 @@ __device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t
     float2 acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = make_float2(0.0f, 0.0f);
-    for (int64_t c = lane; c < nchunk; c += 32) {
-        uint4 w[R];
+    uint4 w[R];
+    if (lane < nchunk) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) w[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + c * 16));
+        for (int r = 0; r < R; ++r) w[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + lane * 16));
+    }
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        uint4 wn[R];
+        if (c + 32 < nchunk) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) wn[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + (c + 32) * 16));
+        }
         const float4* xc = xs4 + c * kChunkF4;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -913,6 +921,8 @@ __device__ __forceinline__ void row_task(const VecProblem& pb, int task, int64_t
                 acc[r] = word_fma(word, xv, acc[r]);
             }
         }
+#pragma unroll
+        for (int r = 0; r < R; ++r) w[r] = wn[r];
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
