@@ -85,6 +85,7 @@ struct Problem {
     int64_t nchunks;     // ceil(k / kChunkK)
     int64_t item0;       // its first (block, chunk) item in the launch's list
     int64_t block0;      // its first block counter
+    const int* xexp;     // integer mode: per activation row, the exponent E of max|x|
 };
 
 // Shared by the matrices of a launch (same activation rows m).
@@ -95,6 +96,7 @@ struct GemmCommon {
     int64_t items;       // items of all matrices
     int32_t grid, count;
     float P, Q;          // y = alpha * (P * D + Q * Sx)
+    double P4, PQ;       // integer mode: y = alpha * (P4 * sum x f' + PQ * Sx)
 };
 
 template <int MAXP>
@@ -123,15 +125,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int nt) {
            (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-// D (TMEM) (+)= A (TMEM) * B (shared memory)^T
+// Instruction descriptor, kind::i8: s32 accumulator, A unsigned 8-bit, B
+// signed 8-bit, both K-major, M = 128, N = nt.
+__host__ __device__ constexpr uint32_t idesc_i8(int nt) {
+    return (2u << 4) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) |
+           (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// D (TMEM) (+)= A (TMEM) * B (shared memory)^T; K = 16 (bf16) or 32 (8-bit)
+template <bool I8>
 __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+    if (I8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "r"(tmem_a), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+            "r"(tmem_a), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
@@ -140,15 +158,16 @@ __device__ __forceinline__ void mma_commit(uint32_t mbar) {
                  : "memory");
 }
 
-// NK MMAs of K = 16 over one stage: A columns advance by 8, the B
-// descriptor start address by 32 B inside a 64-K swizzle atom and by one
-// atom (ATOM_B bytes) every 4 MMAs.
-template <int NK, int ATOM_B>
+// NK MMAs over one stage, each reading 32 bytes of K per row (16 bf16 or
+// 32 8-bit values): A columns advance by 8, the B descriptor start address
+// by 32 B inside a 128-B swizzle atom and by one atom (ATOM_B bytes) every
+// 4 MMAs.
+template <int NK, int ATOM_B, bool I8>
 __device__ __forceinline__ void issue_stage(uint32_t d, uint32_t a, uint64_t b0, uint32_t idesc,
                                             uint32_t acc0) {
 #pragma unroll
     for (int kk = 0; kk < NK; ++kk)
-        mma_ts(d, a + 8u * kk, b0 + static_cast<uint64_t>(((kk >> 2) * ATOM_B + (kk & 3) * 32) >> 4),
+        mma_ts<I8>(d, a + 8u * kk, b0 + static_cast<uint64_t>(((kk >> 2) * ATOM_B + (kk & 3) * 32) >> 4),
                idesc, kk == 0 ? acc0 : 1u);
 }
 
@@ -289,6 +308,17 @@ __device__ __forceinline__ uint32_t pair_of(uint32_t w) {
     return ((s & 0x00600060u) ^ 0x00400040u) | kOnes;
 }
 
+// Integer mode: the 16 fields of a code word as four words of 8-bit
+// offset-binary values f' = f xor 2 in 0..3; output s holds fields s, s + 4,
+// s + 8, s + 12 (one per byte), so the K order inside every group of 16 is
+// the 4 x 4 transpose (position 4s + b holds field s + 4b).
+__device__ __forceinline__ void decode_word_u8(uint32_t w, uint32_t* v) {
+    v[0] = mask_flip_or(w, 0x03030303u, 0x02020202u);
+    v[1] = mask_flip_or(w >> 2, 0x03030303u, 0x02020202u);
+    v[2] = mask_flip_or(w >> 4, 0x03030303u, 0x02020202u);
+    v[3] = mask_flip_or(w >> 6, 0x03030303u, 0x02020202u);
+}
+
 __device__ __forceinline__ void decode_word(uint32_t w, uint32_t* v) {
     v[0] = pair_of<0>(w);
     v[1] = pair_of<1>(w);
@@ -358,15 +388,18 @@ __device__ __forceinline__ bool next_piece(const GemmParams<MAXP>& prm, int64_t&
     return true;
 }
 
-// MMA stages of code chunk c of a K-long row (the last chunk may be short).
+// MMA stages of SK K each in code chunk c of a K-long row (the last chunk
+// may be short).
+template <int SK>
 __device__ __forceinline__ int stages_of_chunk(int64_t k, int64_t c) {
-    const int64_t rest = (k - c * kChunkK + kStageK - 1) / kStageK;
-    return rest < kStagesPerChunk ? static_cast<int>(rest) : kStagesPerChunk;
+    const int64_t rest = (k - c * kChunkK + SK - 1) / SK;
+    return rest < kChunkK / SK ? static_cast<int>(rest) : kChunkK / SK;
 }
 
-// K of the stage starting at k0: kStageK, or 128 for a short tail.
+// K of the stage starting at k0: SK, or less (a multiple of 128) for a short tail.
+template <int SK>
 __device__ __forceinline__ int stage_k(int64_t k, int64_t k0) {
-    return k - k0 < kStageK ? static_cast<int>(k - k0) : kStageK;
+    return k - k0 < SK ? static_cast<int>(k - k0) : SK;
 }
 
 // CTA whose range holds item i: the largest g with range_start(g) <= i.
@@ -397,15 +430,35 @@ struct Layout {
     static_assert(kACol0 + 128 * kASlots <= kTmemCols, "TMEM columns");
 };
 
+// Integer mode: the four digit-plane accumulators of one activation row,
+// sum_p acc_p * 256^p, as an exact double (|value| < 2^47).
+__device__ __forceinline__ double planes_value(const float* v) {
+    const long long t = static_cast<long long>(__float_as_int(v[0])) +
+                        (static_cast<long long>(__float_as_int(v[1])) << 8) +
+                        (static_cast<long long>(__float_as_int(v[2])) << 16) +
+                        (static_cast<long long>(__float_as_int(v[3])) << 24);
+    return static_cast<double>(t);
+}
+
+// 2^e as a double, for e in [-1022, 1023].
+__device__ __forceinline__ double exp2_int(int e) {
+    return __longlong_as_double(static_cast<long long>(e + 1023) << 52);
+}
+
 __device__ __forceinline__ float4 add4(float4 a, float4 b) {
     return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
                        __fadd_rn(a.w, b.w));
 }
 
-template <int NT, int MAXP>
+// I8: the integer mode (kind::i8; A = offset-binary fields as u8, B = the
+// activations' signed base-256 digit planes, NT = 4 x activation rows),
+// 512 K per stage; otherwise bf16 (kind::f16), 256 K per stage.
+template <int NT, int MAXP, bool I8>
 __global__ void __launch_bounds__(kThreads, 1)
     wq_gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
     using L = Layout<NT>;
+    constexpr int SK = I8 ? 2 * kStageK : kStageK;  // K per stage
+    constexpr int KB = I8 ? 128 : 64;                // K per 128-B activation box
     const GemmCommon& p = prm.c;
     constexpr int SC = L::kCodesSlots, SA = L::kASlots, SB = L::kBSlots;
     extern __shared__ uint8_t smem_raw[];
@@ -506,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             while (ok && next_piece(prm, s, re, pc, cur)) {
                 for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
+                    const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
                     for (int i = 0; i < ns; ++i, ++gs) {
                         if (gs >= static_cast<uint32_t>(SB)) {  // B slot free: stage gs - SB done
                             if (!mbar_wait(b_aempty + 8u * er.idx, er.phase, abort)) {
@@ -515,13 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             er.next();
                         }
-                        const int64_t k0 = c * kChunkK + i * kStageK;
-                        const int boxes = stage_k(prm.prob[pc.pi].k, k0) / 64;
+                        const int64_t k0 = c * kChunkK + i * SK;
+                        const int boxes = stage_k<SK>(prm.prob[pc.pi].k, k0) / KB;
                         const uint32_t dst = sbase + L::kBOff + xr.idx * L::kBSlot;
                         mbar_expect_tx(b_xfull + 8u * xr.idx, static_cast<uint32_t>(boxes * NT * 128));
                         for (int bx = 0; bx < boxes; ++bx)
                             tma_load_2d(dst + bx * L::kAtomB, &prm.prob[pc.pi].tx, b_xfull + 8u * xr.idx,
-                                        static_cast<int32_t>(k0 + 64 * bx), 0);
+                                        static_cast<int32_t>(k0 + KB * bx), 0);
                         xr.next();
                     }
                 }
@@ -533,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The issuing thread blocks on every tcgen05.mma, so its loop keeps
         // bookkeeping to a few 32-bit operations between MMAs.
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(NT);
+            constexpr uint32_t idesc = I8 ? idesc_i8(NT) : idesc_bf16(NT);
             Ring<SA> ar;
             Ring<SB> br;
             Ring<2> accr;
@@ -547,8 +600,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d = tmem + L::kAccStride * accr.idx;
                 uint32_t acc0 = 0;
                 for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
-                    const bool short_tail = stage_k(prm.prob[pc.pi].k, c * kChunkK + (ns - 1) * kStageK) != kStageK;
+                    const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
+                    const int tail_k = stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + (ns - 1) * SK);
                     for (int i = 0; i < ns; ++i) {
                         if (!mbar_wait(b_afull + 8u * ar.idx, ar.phase, abort)) {
                             ok = false;
@@ -557,10 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         const uint32_t a = tmem + L::kACol0 + 128u * ar.idx;
                         const uint64_t b0 = sw128_desc(sbase + L::kBOff + br.idx * L::kBSlot);
-                        if (short_tail && i == ns - 1)
-                            issue_stage<8, L::kAtomB>(d, a, b0, idesc, acc0);
+                        if (tail_k == SK || i != ns - 1)
+                            issue_stage<16, L::kAtomB, I8>(d, a, b0, idesc, acc0);
+                        else if (!I8 || tail_k == 256)
+                            issue_stage<8, L::kAtomB, I8>(d, a, b0, idesc, acc0);
+                        else if (tail_k == 128)
+                            issue_stage<4, L::kAtomB, I8>(d, a, b0, idesc, acc0);
                         else
-                            issue_stage<16, L::kAtomB>(d, a, b0, idesc, acc0);
+                            issue_stage<12, L::kAtomB, I8>(d, a, b0, idesc, acc0);
                         acc0 = 1;
                         mma_commit(b_aempty + 8u * ar.idx);
                         ar.next();
@@ -593,21 +650,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint32_t crow = sbase + L::kCodesOff + cr.idx * kCodesSlotBytes + r * 128;
-                const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
+                const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
                 for (int i = 0; i < ns; ++i) {
-                    // this warp's 128 K of the stage exist unless the stage is a short tail
-                    const bool mine = stage_k(prm.prob[pc.pi].k, c * kChunkK + i * kStageK) > 128 * half;
-                    // 128 K of this row (32 code bytes) -> 64 TMEM columns, 64 K at a time
-                    const int ch = 4 * i + 2 * half;
-                    uint4 cw = make_uint4(0, 0, 0, 0);
-                    uint32_t v[32];
-                    if (mine) {
-                        cw = lds128(crow + ((ch ^ (r & 7)) << 4));
-                        decode_word(cw.x, v);
-                        decode_word(cw.y, v + 8);
-                        decode_word(cw.z, v + 16);
-                        decode_word(cw.w, v + 24);
-                        cw = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
+                    // this warp's half of the stage exists unless the stage is a short tail
+                    const bool mine = stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + i * SK) > SK / 2 * half;
+                    // bf16: 128 K of this row (32 code bytes) -> 64 TMEM columns;
+                    // integer mode: 256 K (64 code bytes) -> 64 TMEM columns
+                    const int ch = I8 ? 4 * half : 4 * i + 2 * half;
+                    uint32_t v[32], v2[32];
+                    uint4 c2 = make_uint4(0, 0, 0, 0), c3 = c2;
+                    if (I8 && mine) {
+                        // the first half decoded before the wait; the rest after the first store
+                        const uint4 c0 = lds128(crow + ((ch ^ (r & 7)) << 4));
+                        const uint4 c1 = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
+                        c2 = lds128(crow + (((ch + 2) ^ (r & 7)) << 4));
+                        c3 = lds128(crow + (((ch + 3) ^ (r & 7)) << 4));
+                        decode_word_u8(c0.x, v);
+                        decode_word_u8(c0.y, v + 4);
+                        decode_word_u8(c0.z, v + 8);
+                        decode_word_u8(c0.w, v + 12);
+                        decode_word_u8(c1.x, v + 16);
+                        decode_word_u8(c1.y, v + 20);
+                        decode_word_u8(c1.z, v + 24);
+                        decode_word_u8(c1.w, v + 28);
+                        if (r == kFeat) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = 0x01010101u;
+                        }
+                    } else if (!I8 && mine) {
+                        // decode the whole stage before waiting for its slot
+                        const uint4 c0 = lds128(crow + ((ch ^ (r & 7)) << 4));
+                        const uint4 c1 = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
+                        decode_word(c0.x, v);
+                        decode_word(c0.y, v + 8);
+                        decode_word(c0.z, v + 16);
+                        decode_word(c0.w, v + 24);
+                        decode_word(c1.x, v2);
+                        decode_word(c1.y, v2 + 8);
+                        decode_word(c1.z, v2 + 16);
+                        decode_word(c1.w, v2 + 24);
+                        if (r == kFeat) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = v2[j] = kOnes;
+                        }
                     }
                     if (!warp_wait(b_aempty + 8u * ar.idx, ar.phase ^ 1u, abort)) {
                         ok = false;
@@ -616,20 +701,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mine) {
                         tc_fence_after();
                         const uint32_t col = tmem + lane_addr + L::kACol0 + 128u * ar.idx + 64u * half;
-                        if (r == kFeat) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = kOnes;
-                        }
                         tmem_st32(col, v);
-                        decode_word(cw.x, v);
-                        decode_word(cw.y, v + 8);
-                        decode_word(cw.z, v + 16);
-                        decode_word(cw.w, v + 24);
-                        if (r == kFeat) {
+                        if (I8) {
+                            decode_word_u8(c2.x, v2);
+                            decode_word_u8(c2.y, v2 + 4);
+                            decode_word_u8(c2.z, v2 + 8);
+                            decode_word_u8(c2.w, v2 + 12);
+                            decode_word_u8(c3.x, v2 + 16);
+                            decode_word_u8(c3.y, v2 + 20);
+                            decode_word_u8(c3.z, v2 + 24);
+                            decode_word_u8(c3.w, v2 + 28);
+                            if (r == kFeat) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = kOnes;
+                                for (int j = 0; j < 32; ++j) v2[j] = 0x01010101u;
+                            }
                         }
-                        tmem_st32(col + 32u, v);
+                        tmem_st32(col + 32u, v2);
                         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                         tc_fence_before();
                     }
@@ -653,13 +740,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         while (ok && next_piece(prm, s, re, pc, cur)) {
             for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                const int ns = stages_of_chunk(prm.prob[pc.pi].k, c);
+                const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
                 for (int i = 0; i < ns; ++i) {
                     if (!warp_wait(b_xfull + 8u * br.idx, br.phase, abort)) {
                         ok = false;
                         break;
                     }
-                    const int groups = stage_k(prm.prob[pc.pi].k, c * kChunkK + i * kStageK) / 16;
+                    // the integer mode's digit planes arrive already in MMA order
+                    const int groups = I8 ? 0 : stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + i * SK) / 16;
                     const uint32_t bslot = sbase + L::kBOff + br.idx * L::kBSlot;
                     for (int it = ptid; it < NT * groups; it += kPermWarps * 32) {
                         const int bro = it % NT, g = it / NT;
@@ -712,8 +800,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 tmem_ld16(d + c0, v);
                 if (r == kFeat) {
+                    if (I8) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) sx[c0 + j] = v[j];
+                        for (int jj = 0; jj < 4; ++jj)
+                            reinterpret_cast<double*>(sx)[c0 / 4 + jj] = planes_value(v + 4 * jj);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sx[c0 + j] = v[j];
+                    }
                 }
             }
             epi_sync();
@@ -731,6 +825,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
                 __syncwarp();
                 tmem_ld16(d + c0, v);
+                if (I8) {
+                    // columns 4j .. 4j + 3 are activation row j's digit planes;
+                    // x = digits * 2^(E - 29)
+                    float o[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = c0 / 4 + jj;
+                        const double scale = j < p.m ? exp2_int(__ldg(pb.xexp + j) - 29) : 0.0;
+                        o[jj] = static_cast<float>(
+                            (p.P4 * planes_value(v + 4 * jj) + p.PQ * reinterpret_cast<const double*>(sx)[j]) * scale);
+                    }
+                    if (!valid_row) continue;
+                    if (full) {
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            if (c0 / 4 + jj < p.m)
+                                pb.y[(c0 / 4 + jj) * pb.n + feat] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(alpha * o[jj]));
+                    } else if (c0 / 4 < p.m4) {
+                        *reinterpret_cast<float4*>(prow + c0 / 4) = make_float4(o[0], o[1], o[2], o[3]);
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = fmaf(p.P, v[j], p.Q * sx[c0 + j]);
                 if (!valid_row) continue;
@@ -994,6 +1111,69 @@ static int sm_count() {
 
 constexpr int kMaxBatch = 64;  // matrices per launch (their descriptors travel as parameters)
 
+// Integer mode pre-pass: each distinct activation matrix as signed base-256
+// digit planes. Row j of x is scaled by 2^(29 - E), E = floor(log2 max|x_j|),
+// and rounded to the nearest integer v (|v| < 2^30; exact for every x within
+// 2^22 of the row's largest magnitude, bf16 having 8 significant bits);
+// v = d0 + 256 d1 + 65536 d2 + 2^24 d3 with every digit in [-128, 127].
+// Plane p of row j is row 4j + p of a [4m][k] int8 matrix, its K order
+// inside every group of 16 transposed 4 x 4 like the decoded weights.
+struct XPlanes {
+    const uint16_t* x[kMaxBatch];
+    int8_t* planes[kMaxBatch];
+    int* exps[kMaxBatch];
+    int64_t k[kMaxBatch];
+    int32_t m;
+};
+
+__global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XPlanes prm) {
+    __shared__ float red[8];
+    __shared__ int e_sh;
+    const int xi = blockIdx.x / prm.m, j = blockIdx.x % prm.m;
+    const int64_t k = prm.k[xi];
+    const uint16_t* xr = prm.x[xi] + j * k;
+    float mx = 0.0f;
+    for (int64_t i = threadIdx.x; i < k; i += 256)
+        mx = fmaxf(mx, fabsf(__uint_as_float(static_cast<uint32_t>(xr[i]) << 16)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = red[0];
+        for (int w = 1; w < 8; ++w) t = fmaxf(t, red[w]);
+        const uint32_t b = __float_as_uint(t);
+        // floor(log2 t) from the bits, subnormals included; 0 for an all-zero row
+        e_sh = t == 0.0f ? 0 : (b >> 23) ? static_cast<int>(b >> 23) - 127 : -118 - __clz(b);
+        prm.exps[xi][j] = e_sh;
+    }
+    __syncthreads();
+    const double sc = exp2_int(29 - e_sh);
+    int8_t* pl = prm.planes[xi] + 4 * j * k;
+    for (int64_t g = threadIdx.x; g < k / 16; g += 256) {
+        const uint4 h0 = reinterpret_cast<const uint4*>(xr + 16 * g)[0];
+        const uint4 h1 = reinterpret_cast<const uint4*>(xr + 16 * g)[1];
+        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        uint32_t pw[4][4] = {};
+#pragma unroll
+        for (int f = 0; f < 16; ++f) {
+            const uint32_t bits = (f & 1) ? (hw[f >> 1] & 0xFFFF0000u) : (hw[f >> 1] << 16);
+            int v = __double2int_rn(static_cast<double>(__uint_as_float(bits)) * sc);
+            const int pos = 4 * (f & 3) + (f >> 2);
+#pragma unroll
+            for (int pp = 0; pp < 3; ++pp) {
+                const int dgt = ((v + 128) & 255) - 128;
+                v = (v - dgt) >> 8;
+                pw[pp][pos >> 2] |= static_cast<uint32_t>(dgt & 255) << (8 * (pos & 3));
+            }
+            pw[3][pos >> 2] |= static_cast<uint32_t>(v & 255) << (8 * (pos & 3));
+        }
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp)
+            *reinterpret_cast<uint4*>(pl + pp * k + 16 * g) = make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
+    }
+}
+
 struct Plan {
     int nt;
     int64_t items, blocks;  // over all matrices of the launch
@@ -1004,9 +1184,10 @@ struct Plan {
 // Work list of a launch: matrix i's items start at item0[i], its block
 // counters at block0[i].
 static Plan plan(int64_t m, const pq_gemm_problem_t* pr, int count, int64_t* item0,
-                 int64_t* block0, int64_t* nchunks) {
+                 int64_t* block0, int64_t* nchunks, bool i8) {
     Plan pl;
-    pl.nt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
+    const int64_t rows = i8 ? 4 * m : m;  // B rows: activations, or their 4 digit planes
+    pl.nt = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
     int64_t items = 0, blocks = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t nb = (pr[i].n + kFeat - 1) / kFeat;
@@ -1046,6 +1227,31 @@ static bool coeffs_of(int q, float& P, float& Q) {
     return true;
 }
 
+// Integer mode: y = alpha * factor * (A * sum x f' + B * Sx) in double.
+static bool coeffs_i8(int q, double& P4, double& PQ) {
+    double A, B, factor;
+    switch (q) {
+        case PQ_SEQ2: A = 2; B = -3; factor = 0.25; break;
+        case PQ_SEQ2_B: A = 2; B = -3; factor = 1.0 / 3.0; break;
+        case PQ_TERNARY: A = 2; B = -4; factor = 1.0 / 3.0; break;
+        case PQ_LSQ2: case PQ_BINARY: A = 1; B = -2; factor = 1.0; break;
+        default: return false;
+    }
+    P4 = A * factor;
+    PQ = B * factor;
+    return true;
+}
+
+// The integer mode serves 2..16 activation rows (one row takes the CUDA-core
+// path when its x fits shared memory).
+static bool integer_mode(int64_t m) { return m <= 16; }
+
+static int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace of one activation matrix in the integer mode: its digit planes
+// [4m][k] int8 and the exponents [m] int32.
+static int64_t xplanes_bytes(int64_t m, int64_t k) { return round256(4 * m * k) + round256(4 * m); }
+
 static int64_t partial_bytes(const Plan& pl, int64_t m) {
     const int64_t m4 = (m + 3) / 4 * 4;
     return (static_cast<int64_t>(pl.grid) * 2 * kFeat * m4 * 4 + 255) / 256 * 256;
@@ -1080,7 +1286,7 @@ static pq_status_t check_problem(int64_t m, const pq_gemm_problem_t& pr) {
 // x 128 B, activations [m rows][k] in boxes of nt rows x 64 K, both with the
 // 128B swizzle the MMA and the decoders read.
 static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt,
-                        const pq_gemm_problem_t& pr, Problem& out) {
+                        const pq_gemm_problem_t& pr, Problem& out, const int8_t* planes) {
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k / 4), static_cast<cuuint64_t>(pr.n)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.k / 4)};
@@ -1090,6 +1296,15 @@ static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt
                 strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
+    }
+    if (planes) {  // integer mode: digit planes [4m rows][k] int8, boxes of nt rows x 128 K
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k), static_cast<cuuint64_t>(4 * m)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.k)};
+        const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
+        const cuuint32_t es[2] = {1, 1};
+        return enc(&out.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(planes), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k), static_cast<cuuint64_t>(m)};
@@ -1104,7 +1319,7 @@ static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt
     return true;
 }
 
-template <int NT, int MAXP>
+template <int NT, int MAXP, bool I8>
 static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     using L = Layout<NT>;
     static bool attr_set[64] = {false};
@@ -1112,11 +1327,11 @@ static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         const cudaError_t e = cudaFuncSetAttribute(
-            wq_gemm_kernel<NT, MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+            wq_gemm_kernel<NT, MAXP, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    wq_gemm_kernel<NT, MAXP><<<prm.c.grid, kThreads, L::kBytes, s>>>(prm);
+    wq_gemm_kernel<NT, MAXP, I8><<<prm.c.grid, kThreads, L::kBytes, s>>>(prm);
     return cudaGetLastError();
 }
 
@@ -1184,10 +1399,13 @@ static int64_t workspace_bytes(int q, int64_t m, const pq_gemm_problem_t* pr, in
             return -1;
     }
     if (vector_path(m, pr, count)) return 256;  // one task counter per matrix
+    const bool i8 = integer_mode(m);
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
-    const Plan pl = plan(m, pr, count, item0, block0, nchunks);
-    if (!pl.partials) return 0;
-    return partial_bytes(pl, m) + pl.blocks * 4;
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks, i8);
+    int64_t b = pl.partials ? partial_bytes(pl, m) + round256(pl.blocks * 4) : 0;
+    if (i8)  // sized as if every matrix had its own activations
+        for (int i = 0; i < count; ++i) b += xplanes_bytes(m, pr[i].k);
+    return b;
 }
 
 template <int MAXP>
@@ -1201,9 +1419,32 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         if (st != PQ_OK) return st;
     }
     if (vector_path(m, pr, count)) return run_vector<MAXP>(q, pr, count, workspace, ws_bytes, s);
+    const bool i8 = integer_mode(m);
+    if (i8 && !coeffs_i8(q, P.c.P4, P.c.PQ)) return PQ_ERR_UNSUPPORTED;
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
-    const Plan pl = plan(m, pr, count, item0, block0, nchunks);
-    const int64_t need = pl.partials ? partial_bytes(pl, m) + pl.blocks * 4 : 0;
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks, i8);
+    const int64_t base = pl.partials ? partial_bytes(pl, m) + round256(pl.blocks * 4) : 0;
+    // integer mode: one digit-plane set per distinct activation matrix
+    int slot[kMaxBatch];
+    int nslots = 0;
+    XPlanes X{};
+    int64_t need = base;
+    if (i8) {
+        X.m = static_cast<int32_t>(m);
+        for (int i = 0; i < count; ++i) {
+            int t = 0;
+            while (t < nslots && !(X.x[t] == pr[i].x_bf16 && X.k[t] == pr[i].k)) ++t;
+            if (t == nslots) {
+                X.x[t] = pr[i].x_bf16;
+                X.k[t] = pr[i].k;
+                X.planes[t] = reinterpret_cast<int8_t*>(need);  // offsets until the base is known
+                X.exps[t] = reinterpret_cast<int*>(need + round256(4 * m * pr[i].k));
+                need += xplanes_bytes(m, pr[i].k);
+                ++nslots;
+            }
+            slot[i] = t;
+        }
+    }
     P.c.m = m;
     P.c.m4 = (m + 3) / 4 * 4;
     P.c.items = pl.items;
@@ -1214,12 +1455,18 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
             return PQ_ERR_INVALID_ARG;
         P.c.partial = static_cast<float*>(workspace);
         P.c.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes(pl, m));
+        for (int t = 0; t < nslots; ++t) {
+            X.planes[t] = static_cast<int8_t*>(workspace) + reinterpret_cast<intptr_t>(X.planes[t]);
+            X.exps[t] = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                               reinterpret_cast<intptr_t>(X.exps[t]));
+        }
     }
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return PQ_ERR_CUDA;
     for (int i = 0; i < count; ++i) {
         Problem& d = P.prob[i];
-        if (!encode_maps(enc, m, pl.nt, pr[i], d)) return PQ_ERR_CUDA;
+        if (!encode_maps(enc, m, pl.nt, pr[i], d, i8 ? X.planes[slot[i]] : nullptr)) return PQ_ERR_CUDA;
+        d.xexp = i8 ? X.exps[slot[i]] : nullptr;
         d.alpha = pr[i].alpha;
         d.y = pr[i].y_bf16;
         d.n = pr[i].n;
@@ -1228,15 +1475,22 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         d.item0 = item0[i];
         d.block0 = block0[i];
     }
-    if (need > 0 &&
+    if (pl.partials &&
         cudaMemsetAsync(P.c.counters, 0, static_cast<size_t>(pl.blocks) * 4, s) != cudaSuccess)
         return PQ_ERR_CUDA;
+    if (i8) {
+        xplanes_kernel<<<nslots * static_cast<int>(m), 256, 0, s>>>(X);
+        if (cudaGetLastError() != cudaSuccess) return PQ_ERR_CUDA;
+    }
     cudaError_t e;
-    switch (pl.nt) {
-        case 16: e = launch<16, MAXP>(P, s); break;
-        case 32: e = launch<32, MAXP>(P, s); break;
-        case 64: e = launch<64, MAXP>(P, s); break;
-        default: e = launch<128, MAXP>(P, s); break;
+    switch (pl.nt + (i8 ? 1 : 0)) {
+        case 17: e = launch<16, MAXP, true>(P, s); break;
+        case 33: e = launch<32, MAXP, true>(P, s); break;
+        case 65: e = launch<64, MAXP, true>(P, s); break;
+        case 16: e = launch<16, MAXP, false>(P, s); break;
+        case 32: e = launch<32, MAXP, false>(P, s); break;
+        case 64: e = launch<64, MAXP, false>(P, s); break;
+        default: e = launch<128, MAXP, false>(P, s); break;
     }
     return e == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
