@@ -774,22 +774,34 @@ def run_wq_gemm(args):
                 "algorithmic_flops_per_step": flops_step}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    # one activation row with k <= 32768 is served by the CUDA-core kernel
-    roof["kernel"] = ("pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)"
-                      if m == 1 and max(b.m.cols for b in step.bufs) <= 32768 else
-                      "pqg::wq_gemm_kernel<NT> (tcgen05.mma kind::f16, TMEM accumulator)")
+    # the kernel of the grouped launches: one activation row times a lone
+    # matrix (k <= 32768) takes the CUDA-core kernel, 1..16 rows otherwise the
+    # integer tensor-core mode (after its activation digit-plane pre-pass),
+    # more rows the bf16 tensor-core mode
+    integer_mode = m <= 16 and not (m == 1 and gsize == 1 and max(ks) <= 32768)
+    if m == 1 and gsize == 1 and max(ks) <= 32768:
+        roof["kernel"] = "pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)"
+    elif integer_mode:
+        roof["kernel"] = ("pqg::wq_gemm_kernel<NT, MAXP, true> (tcgen05.mma kind::i8, TMEM accumulator)"
+                          " after pqg::xplanes_kernel")
+    else:
+        roof["kernel"] = "pqg::wq_gemm_kernel<NT, MAXP, false> (tcgen05.mma kind::f16, TMEM accumulator)"
     print(json.dumps({
         "metric": "weight-only 2-bit matmul Gweights/s", "op": "wq_gemm",
         "value": weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "dtype": "bf16 x 2-bit codes, f32 accumulate",
+        "higher_is_better": True,
+        "dtype": ("s8 digit planes of bf16 activations x u8 2-bit code fields, s32 accumulate"
+                  if integer_mode else "bf16 x 2-bit codes, f32 accumulate"),
         "data": "synthetic",
         "config": {"workload": (f"llama3_8b_linear_set_seq2_wq_gemm_m{m}" if args.shape != "16384"
                                 else f"4x16384x16384_seq2_wq_gemm_m{m}"), "m": m,
                    "weights": weights, "launches_per_step": len(groups),
+                   "kernels_per_step": len(groups) * (2 if integer_mode else 1),
                    "matrices_per_launch": gsize,
                    "l2": f"codes {step.weights / 4e9:.2f} GB per step, larger than L2"},
         "roofline": roof,
+        "gpu_launches": len(groups) * (2 if integer_mode else 1) * args.steps,
         "tflops": flops_step / (ms * 1e-3) / 1e12,
         "per_matrix_launches": {"ms_per_step": ms_single, "launches_per_step": len(step.bufs),
                                 "what": "pq_wq_gemm once per matrix, CUDA graph"},

@@ -1118,23 +1118,32 @@ constexpr int kMaxBatch = 64;  // matrices per launch (their descriptors travel 
 // v = d0 + 256 d1 + 65536 d2 + 2^24 d3 with every digit in [-128, 127].
 // Plane p of row j is row 4j + p of a [4m][k] int8 matrix, its K order
 // inside every group of 16 transposed 4 x 4 like the decoded weights.
+// A row is split into `slices` CTAs; each finds the row's max|x| itself
+// (the row is small and in L2) and converts its share of 16-element groups.
 struct XPlanes {
     const uint16_t* x[kMaxBatch];
     int8_t* planes[kMaxBatch];
     int* exps[kMaxBatch];
     int64_t k[kMaxBatch];
-    int32_t m;
+    int32_t m, slices;
 };
 
 __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XPlanes prm) {
     __shared__ float red[8];
     __shared__ int e_sh;
-    const int xi = blockIdx.x / prm.m, j = blockIdx.x % prm.m;
+    const int row = blockIdx.x / prm.slices, slice = blockIdx.x % prm.slices;
+    const int xi = row / prm.m, j = row % prm.m;
     const int64_t k = prm.k[xi];
     const uint16_t* xr = prm.x[xi] + j * k;
-    float mx = 0.0f;
-    for (int64_t i = threadIdx.x; i < k; i += 256)
-        mx = fmaxf(mx, fabsf(__uint_as_float(static_cast<uint32_t>(xr[i]) << 16)));
+    // max |x| of the row: the bf16 bits with the sign cleared order like the values
+    uint32_t mb = 0;
+    for (int64_t i = threadIdx.x; i < k / 8; i += 256) {
+        const uint4 h = __ldg(reinterpret_cast<const uint4*>(xr) + i);
+        const uint32_t a = __vmaxu2(__vmaxu2(h.x & 0x7FFF7FFFu, h.y & 0x7FFF7FFFu),
+                                    __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));  // per half
+        mb = max(mb, max(a & 0xFFFFu, a >> 16));
+    }
+    float mx = __uint_as_float(mb << 16);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
@@ -1145,12 +1154,14 @@ __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XP
         const uint32_t b = __float_as_uint(t);
         // floor(log2 t) from the bits, subnormals included; 0 for an all-zero row
         e_sh = t == 0.0f ? 0 : (b >> 23) ? static_cast<int>(b >> 23) - 127 : -118 - __clz(b);
-        prm.exps[xi][j] = e_sh;
+        if (slice == 0) prm.exps[xi][j] = e_sh;
     }
     __syncthreads();
     const double sc = exp2_int(29 - e_sh);
     int8_t* pl = prm.planes[xi] + 4 * j * k;
-    for (int64_t g = threadIdx.x; g < k / 16; g += 256) {
+    const int64_t groups = k / 16;
+    const int64_t g1 = groups * (slice + 1) / prm.slices;
+    for (int64_t g = groups * slice / prm.slices + threadIdx.x; g < g1; g += 256) {
         const uint4 h0 = reinterpret_cast<const uint4*>(xr + 16 * g)[0];
         const uint4 h1 = reinterpret_cast<const uint4*>(xr + 16 * g)[1];
         const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
@@ -1335,9 +1346,12 @@ static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// A single activation row with x fitting shared memory takes the CUDA-core path.
+// A single activation row times a lone matrix, x fitting shared memory, takes
+// the CUDA-core path (measured faster there; a group of matrices runs faster
+// through the integer tensor-core mode, whose pipeline does not restart per
+// matrix).
 static bool vector_path(int64_t m, const pq_gemm_problem_t* pr, int count) {
-    if (m != 1) return false;
+    if (m != 1 || count != 1) return false;
     for (int i = 0; i < count; ++i)
         if (pr[i].k > pqv::kMaxK) return false;
     return true;
@@ -1479,7 +1493,15 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         cudaMemsetAsync(P.c.counters, 0, static_cast<size_t>(pl.blocks) * 4, s) != cudaSuccess)
         return PQ_ERR_CUDA;
     if (i8) {
-        xplanes_kernel<<<nslots * static_cast<int>(m), 256, 0, s>>>(X);
+        // at most one CTA per SM over all rows, each converting >= 64 groups
+        int64_t maxk = 0;
+        for (int t = 0; t < nslots; ++t) maxk = X.k[t] > maxk ? X.k[t] : maxk;
+        const int64_t rows = nslots * m;
+        int64_t sl = sm_count() / rows;
+        const int64_t cap = maxk / (16 * 64);
+        sl = sl < cap ? sl : cap;
+        X.slices = static_cast<int32_t>(sl < 1 ? 1 : sl);
+        xplanes_kernel<<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X);
         if (cudaGetLastError() != cudaSuccess) return PQ_ERR_CUDA;
     }
     cudaError_t e;
