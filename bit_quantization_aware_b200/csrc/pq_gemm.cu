@@ -19,6 +19,19 @@
 // (16 bits apart), so the K order inside every group of 16 is interleaved
 // (j, j + 8); the activation tile is permuted the same way in shared memory.
 //
+// Integer mode (m <= 16). The 8-bit MMA kinds take K = 32 per instruction at
+// the cost of a K = 16 bf16 one, so the weights are decoded instead to their
+// offset-binary fields f' as unsigned bytes (one shift and one three-input
+// logic op per four weights) and multiplied (kind::i8, s32 accumulators) by
+// the activations in fixed point: a pre-pass scales each activation row by
+// 2^(29 - E), E = floor(log2 max|x|), rounds to integers and writes their four
+// signed base-256 digits as four planes, so the tensor cores form the exact
+// integer sums of digits times fields, combined in fp64 in the epilogue:
+//   Y = alpha * factor * (A * sum x f' + B * Sx)
+// with Sx from the row of ones as before. The decoded bytes of a word are
+// fields (s, s + 4, s + 8, s + 12), so the K order inside every group of 16
+// is a 4 x 4 transpose, which the pre-pass applies to the planes.
+//
 // Operands. A (decoded weights) lives in TMEM (tcgen05.st from the decode
 // warps; tcgen05.mma reads it there, with no shared-memory round trip);
 // B (activations) arrives by TMA in the 128B-swizzled K-major layout the

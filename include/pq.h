@@ -305,8 +305,18 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  * kernels consume packed weights in this way [P4: a 2-bit GEMM kernel on
  * CUTLASS; P3: the accuracy-latency trade-off]; this one is built for
  * sm_100a. The levels' integer numerators (SEQ2 2c+1, SEQ2_B 2c+1, ternary
- * 2c, LSQ2 and binary c) are exact in bf16; the factor (1/4, 1/3, 1/3, 1,
- * 1) times alpha scales the fp32 sums, which are rounded once to bf16.
+ * 2c, LSQ2 and binary c) are affine in the code's offset-binary field
+ * f' = c + 2; the factor (1/4, 1/3, 1/3, 1, 1) times alpha scales the sums,
+ * which are rounded once to bf16. Two modes:
+ *   m <= 16 (integer mode; m = 1 only for the grouped call): each activation
+ *     row is scaled by a power of two to 30-bit fixed point, rounded to the
+ *     nearest integer (exact for every value within 2^22 of the row's largest
+ *     magnitude; otherwise off by at most 2^-30 of it) and split into four
+ *     signed base-256 digits; the tensor cores (kind::i8) form the exact
+ *     integer sums of digits times fields, combined in fp64.
+ *   m > 16 (bf16 mode): weights decoded to bf16 1 + f'/4 (exact), products
+ *     accumulated in fp32 by the tensor cores (kind::f16).
+ * A lone matrix with m = 1 runs on the CUDA cores (fp32 fused multiply-adds).
  *   x_bf16   bf16 [m, k], row-major, 16-byte aligned, 1 <= m <= 128
  *   packed   codes [n, k/4] as pq_fakequant_fwd writes them, 16-byte aligned
  *   alpha    fp32 [n]
@@ -315,8 +325,9 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  *   workspace, workspace_bytes: device scratch of at least
  *            pq_wq_gemm_workspace_bytes(q, m, n, k) bytes, 256-byte
  *            aligned (may be NULL when that is 0). Split-K partial sums and
- *            counters live there; calls that share a workspace must not
- *            overlap on the GPU. Results are deterministic.
+ *            counters, and in the integer mode the activations' digit planes
+ *            (4 m k bytes) and exponents, live there; calls that share a
+ *            workspace must not overlap on the GPU. Results are deterministic.
  * Waits inside the kernel are bounded; pq_device_status() reports one that
  * gave up. Traffic: k/4 B of codes per output feature (+ x, y). */
 PQ_API pq_status_t pq_wq_gemm(pq_quant_t q, int64_t m, int64_t n, int64_t k,
@@ -352,7 +363,9 @@ PQ_API pq_status_t pq_wq_gemm_batch(pq_quant_t q, int64_t m, int32_t count,
                                     const pq_gemm_problem_t* problems, void* workspace,
                                     int64_t workspace_bytes, void* stream);
 
-/* Workspace bytes pq_wq_gemm_batch needs (0: none), -1 if invalid. */
+/* Workspace bytes pq_wq_gemm_batch needs (0: none), -1 if invalid. In the
+ * integer mode it counts one digit-plane set per matrix; a call whose
+ * matrices share activations (same x_bf16 and k) uses one set for them. */
 PQ_API int64_t pq_wq_gemm_batch_workspace_bytes(pq_quant_t q, int64_t m, int32_t count,
                                                 const pq_gemm_problem_t* problems);
 
