@@ -317,6 +317,11 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  *   m > 16 (bf16 mode): weights decoded to bf16 1 + f'/4 (exact), products
  *     accumulated in fp32 by the tensor cores (kind::f16).
  * A lone matrix with m = 1 runs on the CUDA cores (fp32 fused multiply-adds).
+ * The bf16 and CUDA-core modes form y from sums over all k of x (1 + f'/4)
+ * and of x, so their rounding scales with alpha sum_k |x|; where activations
+ * far larger than the rest of their row meet zero levels (ternary, LSQ2),
+ * that scale, not sum_k |x w|, bounds the error, as 2^-30 max_k |x|
+ * sum_k |w| does in the integer mode.
  *   x_bf16   bf16 [m, k], row-major, 16-byte aligned, 1 <= m <= 128
  *   packed   codes [n, k/4] as pq_fakequant_fwd writes them, 16-byte aligned
  *   alpha    fp32 [n]

@@ -26,17 +26,33 @@ def _case(q, m, n, k, seed):
     return x, packed, a
 
 
-def _check(q, x, packed, a, y):
-    k = x.shape[1]
+def _check(q, x, packed, a, y, grouped=False):
+    """y against the oracle within the matmul tolerance, derived from each
+    mode's arithmetic: bf16 output rounding (2^-8 |ref|) plus an accumulation
+    bound (1e-4 sum_k |x w|), and
+      integer mode (m <= 16, except one row times a lone matrix with
+      k <= 32768): the fixed-point conversion; every activation is rounded to
+      a multiple of 2^(E-29) with 2^E <= max_k |x|, so |error| <=
+      2^-30 max_k |x| sum_k |w|;
+      bf16 and CUDA-core modes: y = alpha (P D + Q Sx) from fp32 sums over
+      all k of x (1 + f'/4) and of x, whose rounding scales with
+      alpha sum_k |x| (it shows where large activations meet zero levels,
+      ternary and LSQ2): 2^-16 alpha sum_k |x|."""
+    m, k = x.shape
     xb = x.view(torch.int16).cpu().numpy()
     pk = packed.cpu().numpy()
     an = a.cpu().numpy()
     ref = pq_oracle.default().wq_matmul(q, xb, pk, an, k)
     # sum_k |x_k * w_k| (for the tolerance only) from the dequantized weights
     wd = pq_oracle.bf16_bits_to_float(pq_oracle.dequant(q, pk, an, k)).astype(np.float64)
-    ones = np.abs(x.float().cpu().numpy().astype(np.float64)) @ np.abs(wd).T
+    xf = np.abs(x.float().cpu().numpy().astype(np.float64))
+    ones = xf @ np.abs(wd).T
     got = y.float().cpu().numpy().astype(np.float64)
     tol = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ones) + 1e-30
+    if m <= 16 and not (m == 1 and not grouped and k <= 32768):
+        tol += 2.0 ** -30 * np.outer(xf.max(axis=1), np.abs(wd).sum(axis=1))
+    else:
+        tol += 2.0 ** -16 * np.outer(xf.sum(axis=1), np.abs(an).astype(np.float64))
     err = np.abs(got - ref)
     worst = np.unravel_index(np.argmax(err / tol), err.shape)
     assert np.all(err <= tol), (f"q={q} shape={x.shape}x{packed.shape}: worst at {worst}: "
@@ -96,7 +112,71 @@ def test_wq_gemm_batch_matches_oracle():
     torch.cuda.synchronize()
     assert pq.pq_device_status() == 0
     for x, packed, a, y in zip(xs, pks, als, ys):
-        _check(q, x, packed, a, y)
+        _check(q, x, packed, a, y, grouped=True)
+
+
+def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.astype(np.uint16).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("q", Q2)
+@pytest.mark.parametrize("m", [1, 6, 18])
+def test_activation_value_ranges(q, m):
+    """Activation rows the integer mode's fixed-point conversion (m = 6), the
+    bf16 mode (m = 18, the six rows repeated) and the CUDA-core path (m = 1,
+    the row with one huge value) must handle: ordinary values, an all-zero
+    row, a row of subnormals only, magnitudes spread over 2^120 (far beyond
+    the 2^22 the integer mode converts exactly), one huge value among tiny
+    ones, and both signs of zero."""
+    n, k = 1000, 2048
+    rng = np.random.default_rng(17)
+    rows = np.zeros((6, k), np.uint16)
+    normal = (rng.standard_normal(k).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    rows[0] = normal
+    rows[1] = 0
+    rows[2] = rng.integers(1, 0x80, k).astype(np.uint16) | (rng.integers(0, 2, k).astype(np.uint16) << 15)
+    e = rng.integers(-60, 61, k)
+    spread = (np.ldexp(1.0, e) * rng.choice([-1.0, 1.0], k) * (1 + rng.random(k))).astype(np.float32)
+    rows[3] = (spread.view(np.uint32) >> 16).astype(np.uint16)
+    tiny = np.full(k, np.float32(1e-20), np.float32) * rng.choice([-1, 1], k).astype(np.float32)
+    tiny[k // 3] = np.float32(1e20)
+    rows[4] = (tiny.view(np.uint32) >> 16).astype(np.uint16)
+    rows[5] = np.where(rng.random(k) < 0.5, 0x8000, 0).astype(np.uint16)  # +0 and -0
+    x = _bf16_from_bits(rows[4:5] if m == 1 else np.tile(rows, (3, 1))[:m])
+    w = I.normal_weights(n, k, seed=9, stream=0, device=DEV)
+    a = I.alpha_init(w, q)
+    _, packed = pq.fakequant_fwd(q, w, a, pack=True)
+    y = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    _check(q, x, packed, a, y)
+    if m > 1:
+        yz = y.float().cpu().numpy()
+        assert np.all(yz[1::6] == 0) and np.all(yz[5::6] == 0)
+
+
+def test_wq_gemm_batch_shared_activations():
+    """Matrices of one launch sharing activation matrices (the integer mode
+    converts each distinct one once) and ones with their own."""
+    q, m = pq.PQ_SEQ2, 9
+    xa = _case(q, m, 8, 4096, seed=201)[0]
+    xb = _case(q, m, 8, 4096, seed=202)[0]
+    xc = _case(q, m, 8, 1536, seed=203)[0]
+    plan = [(xa, 4096, 1000), (xb, 4096, 640), (xa, 4096, 127), (xb, 4096, 4096),
+            (xa, 4096, 300), (xc, 1536, 2000)]
+    xs, pks, als = [], [], []
+    for i, (x, k, n) in enumerate(plan):
+        w = I.normal_weights(n, k, seed=210 + i, stream=0, device=DEV)
+        a = I.alpha_init(w, q)
+        _, packed = pq.fakequant_fwd(q, w, a, pack=True)
+        xs.append(x)
+        pks.append(packed)
+        als.append(a)
+    ys = pq.wq_gemm_batch(q, xs, pks, als)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    for x, packed, a, y in zip(xs, pks, als, ys):
+        _check(q, x, packed, a, y, grouped=True)
 
 
 @pytest.mark.parametrize("q", [pq.PQ_TERNARY, pq.PQ_SEQ2_B])
@@ -116,7 +196,7 @@ def test_wq_gemm_batch_of_64_is_deterministic(q):
     for a_, b_ in zip(y1, y2):
         assert torch.equal(a_.view(torch.int16), b_.view(torch.int16))
     for i in (0, 17, 63):
-        _check(q, xs[i], pks[i], als[i], y1[i])
+        _check(q, xs[i], pks[i], als[i], y1[i], grouped=True)
 
 
 def test_wq_gemm_batch_rejects_bad_counts():
@@ -155,12 +235,11 @@ def test_wq_gemm_wait_timeout_reports_and_recovers():
     _check(q, x, packed, a, y)
 
 
-def _check_rows(q, x, packed, a, y, rows):
+def _check_rows(q, x, packed, a, y, rows, grouped=False):
     """_check on a subset of output features (the oracle runs on those rows)."""
-    k = x.shape[1]
     idx = torch.as_tensor(rows, device=packed.device)
     _check(q, x, packed.index_select(0, idx).contiguous(), a.index_select(0, idx).contiguous(),
-           y.index_select(1, idx).contiguous())
+           y.index_select(1, idx).contiguous(), grouped=grouped)
 
 
 def test_wq_gemm_full_size_grouped_sampled():
@@ -183,12 +262,12 @@ def test_wq_gemm_full_size_grouped_sampled():
     rng = np.random.default_rng(5)
     for (n, k), x, packed, a, y in zip(shapes, xs, pks, als, ys):
         rows = sorted(set([0, n - 1] + list(rng.choice(n, 62, replace=False))))
-        _check_rows(q, x, packed, a, y, rows)
+        _check_rows(q, x, packed, a, y, rows, grouped=True)
 
 
 def test_wq_gemm_batch_single_row_matches_oracle():
-    """One activation row (the CUDA-core path) over matrices of several
-    shapes in one launch."""
+    """One activation row over matrices of several shapes in one launch
+    (the integer tensor-core mode; a lone matrix takes the CUDA-core path)."""
     q, m = pq.PQ_SEQ2_B, 1
     shapes = [(4096, 4096), (1000, 640), (7, 128), (14336, 4096), (300, 14336)]
     xs, pks, als = [], [], []
@@ -203,4 +282,4 @@ def test_wq_gemm_batch_single_row_matches_oracle():
     assert pq.pq_device_status() == pq.PQ_OK
     for x, packed, a, ya, yb in zip(xs, pks, als, y1, y2):
         assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
-        _check(q, x, packed, a, ya)
+        _check(q, x, packed, a, ya, grouped=True)
