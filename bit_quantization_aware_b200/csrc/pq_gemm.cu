@@ -1404,13 +1404,11 @@ static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, voi
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pqv::gemv_kernel<MAXP>, pqv::kThreads,
                                                       smem) != cudaSuccess || per_sm < 1)
         per_sm = 1;
-    // rows per task (x loads are shared by the rows of a task): a lone
-    // matrix takes the largest of 4, 2, 1 that still gives about one task
-    // per warp of the grid; a group takes 4 (measured best: its matrices
-    // follow one another, so fewer instructions per weight win there)
+    // rows per task (x loads are shared by the rows of a task): the largest
+    // of 4, 2, 1 that still gives about one task per warp of the grid
     const int64_t warps = static_cast<int64_t>(sm_count()) * per_sm * (pqv::kThreads / 32);
     for (int i = 0; i < count; ++i)
-        V.prob[i].rows = count > 1 ? 4 : pr[i].n >= 4 * warps ? 4 : pr[i].n >= 2 * warps ? 2 : 1;
+        V.prob[i].rows = pr[i].n >= 4 * warps ? 4 : pr[i].n >= 2 * warps ? 2 : 1;
     if (cudaMemsetAsync(counters, 0, static_cast<size_t>(count) * 4, s) != cudaSuccess)
         return PQ_ERR_CUDA;
     pqv::gemv_kernel<MAXP><<<sm_count() * per_sm, pqv::kThreads, smem, s>>>(V);
@@ -1445,7 +1443,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         const pq_status_t st = check_problem(m, pr[i]);
         if (st != PQ_OK) return st;
     }
-    if (vector_path(m, pr, count)) return run_vector<MAXP>(q, pr, count, workspace, ws_bytes, s);
+    if (vector_path(m, pr, count)) return run_vector<1>(q, pr, 1, workspace, ws_bytes, s);
     const bool i8 = integer_mode(m);
     if (i8 && !coeffs_i8(q, P.c.P4, P.c.PQ)) return PQ_ERR_UNSUPPORTED;
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
