@@ -170,3 +170,32 @@ def test_adamw_argument_errors(L):
         assert f(pq.PQ_SEQ2, 2, arr, ctypes.byref(h), ctypes.byref(h), None) == E
     arr = pq.adamw_matrix_array([dict(rows=0, cols=8)])
     assert f(pq.PQ_SEQ2, 1, arr, ctypes.byref(h), ctypes.byref(h), None) == pq.PQ_OK
+
+
+def test_matmul_workspace_sizes(L):
+    """Workspace sizing of the weight-only matmul (host arithmetic only): the
+    one-row path needs one counter block, the integer mode (m <= 16) at least
+    the activations' digit planes (4 m k bytes), a group one set per matrix;
+    sizes are multiples of 256; bad shapes give -1; the no-alloc scratch
+    holds every decode-sized problem of the Llama-3-8B shapes."""
+    from bit_quantization_aware_b200 import pq
+    q = pq.PQ_SEQ2
+    assert L.pq_wq_gemm_workspace_bytes(q, 1, 16384, 16384) == 256
+    for m in (2, 9, 16):
+        b = L.pq_wq_gemm_workspace_bytes(q, m, 16384, 16384)
+        assert b >= 4 * m * 16384 and b % 256 == 0
+    assert L.pq_wq_gemm_workspace_bytes(q, 0, 128, 128) == -1
+    assert L.pq_wq_gemm_workspace_bytes(q, 4, 128, 100) == -1
+    assert L.pq_wq_gemm_workspace_bytes(pq.PQ_LSQ4, 4, 128, 128) == -1
+    shapes = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
+    xs = [ctypes.c_void_p(16 * (i + 1)) for i in range(len(shapes))]  # never dereferenced
+    arr = (pq.PQGemmProblem * len(shapes))()
+    for i, (n, k) in enumerate(shapes):
+        arr[i].n, arr[i].k, arr[i].x_bf16 = n, k, xs[i].value
+    for m in (1, 8, 16):
+        b = L.pq_wq_gemm_batch_workspace_bytes(q, m, len(shapes), arr)
+        assert b >= sum(4 * m * k for _, k in shapes) and b % 256 == 0
+    cap = pq.WQ_GEMM_NOALLOC_SCRATCH_BYTES
+    for m in range(1, 17):
+        for n, k in shapes:
+            assert L.pq_wq_gemm_workspace_bytes(q, m, n, k) <= cap
