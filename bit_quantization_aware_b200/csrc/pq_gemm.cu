@@ -447,9 +447,9 @@ struct Layout {
 // sum_p acc_p * 256^p, as an exact double (|value| < 2^47).
 __device__ __forceinline__ double planes_value(const float* v) {
     const long long t = static_cast<long long>(__float_as_int(v[0])) +
-                        (static_cast<long long>(__float_as_int(v[1])) << 8) +
-                        (static_cast<long long>(__float_as_int(v[2])) << 16) +
-                        (static_cast<long long>(__float_as_int(v[3])) << 24);
+                        static_cast<long long>(__float_as_int(v[1])) * 256 +
+                        static_cast<long long>(__float_as_int(v[2])) * 65536 +
+                        static_cast<long long>(__float_as_int(v[3])) * 16777216;
     return static_cast<double>(t);
 }
 
@@ -942,6 +942,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
 }
 
+// Sixteen consecutive activations (bf16 pairs hw[0..7]) as the integer
+// mode's four signed base-256 digit words per plane: v = rint(x * 2^(29-E))
+// (ties to even; the product is exact in fp64),
+// v = d0 + 256 d1 + 65536 d2 + 2^24 d3, digits in [-128, 127]; in plane p,
+// byte position 4s + b holds the digit of element s + 4b (the decoded
+// weights' K order).
+__device__ __forceinline__ void digits16(const uint32_t (&hw)[8], int E, uint32_t (&pw)[4][4]) {
+    const double sc = exp2_int(29 - E);
+#pragma unroll
+    for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pw[pp][q] = 0;
+#pragma unroll
+    for (int f = 0; f < 16; ++f) {
+        const uint32_t bits = (f & 1) ? (hw[f >> 1] & 0xFFFF0000u) : (hw[f >> 1] << 16);
+        int v = __double2int_rn(static_cast<double>(__uint_as_float(bits)) * sc);
+        const int pos = 4 * (f & 3) + (f >> 2);
+#pragma unroll
+        for (int pp = 0; pp < 3; ++pp) {
+            const int dgt = ((v + 128) & 255) - 128;
+            v = (v - dgt) >> 8;
+            pw[pp][pos >> 2] |= static_cast<uint32_t>(dgt & 255) << (8 * (pos & 3));
+        }
+        pw[3][pos >> 2] |= static_cast<uint32_t>(v & 255) << (8 * (pos & 3));
+    }
+}
+
+// floor(log2 |x|) of the largest magnitude among bf16 bit patterns given as
+// their sign-cleared magnitude bits (0 for an all-zero row), subnormals included.
+__device__ __forceinline__ int exponent_of_max(uint32_t mag_bits16) {
+    const uint32_t b = mag_bits16 << 16;
+    return b == 0 ? 0 : (b >> 23) ? static_cast<int>(b >> 23) - 127 : -118 - __clz(b);
+}
+
 // ------------------------------------------------- one activation row
 // For m = 1 the tensor cores retire at most 2048 weights per ~46-cycle MMA
 // per SM, far below what the codes' bandwidth allows, so a single row takes
@@ -977,6 +1011,7 @@ template <int MAXP>
 struct VecParams {
     int32_t count;
     float P, Q;
+    double P4, PQ;       // integer kernel: y = alpha * (P4 * sum x f' + PQ * Sx)
     VecProblem prob[MAXP];
 };
 
@@ -1110,6 +1145,158 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const __grid_constant
     }
 }
 
+// Integer one-row kernel: the integer mode's arithmetic on the CUDA cores.
+// Each CTA turns x into four signed base-256 digit planes in shared memory
+// (scale 2^(29 - E) from the row's largest magnitude, as in the pre-pass;
+// chunk c of 64 K at c * 272 bytes, [word w][plane p] 16 bytes each, the K
+// order transposed like the decoded fields) and sums their digits (Sx).
+// A weight word gives four registers of u8 fields (one shift and one
+// three-input op each), and dp4a multiplies each against the matching four
+// digits of every plane: 23 instructions per 16 weights, exact int32 sums.
+template <int R>
+__device__ __forceinline__ void row_task_i8(const VecProblem& pb, int task, int64_t kq, int64_t nchunk,
+                                            int lane, double P4, double PQ, double sxd, double scale,
+                                            const uint4* xs4) {
+    const int64_t row0 = static_cast<int64_t>(task) * R;
+    const uint8_t* rp[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t row = row0 + r < pb.n ? row0 + r : pb.n - 1;
+        rp[r] = pb.codes + row * kq;
+    }
+    int acc[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) acc[r][pp] = 0;
+    uint4 w[R];
+    if (lane < nchunk) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) w[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + lane * 16));
+    }
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        uint4 wn[R];
+        if (c + 32 < nchunk) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) wn[r] = __ldcs(reinterpret_cast<const uint4*>(rp[r] + (c + 32) * 16));
+        }
+        const uint4* xc = xs4 + c * kChunkF4;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 xp[4];
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) xp[pp] = xc[4 * q4 + pp];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint32_t word = q4 == 0 ? w[r].x : q4 == 1 ? w[r].y : q4 == 2 ? w[r].z : w[r].w;
+                uint32_t o[4];
+                decode_word_u8(word, o);
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    int a = acc[r][pp];
+                    a = __dp4a(static_cast<int>(o[0]), static_cast<int>(xp[pp].x), a);
+                    a = __dp4a(static_cast<int>(o[1]), static_cast<int>(xp[pp].y), a);
+                    a = __dp4a(static_cast<int>(o[2]), static_cast<int>(xp[pp].z), a);
+                    a = __dp4a(static_cast<int>(o[3]), static_cast<int>(xp[pp].w), a);
+                    acc[r][pp] = a;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) w[r] = wn[r];
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        long long t = 0;
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            int a = acc[r][pp];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+            t += static_cast<long long>(a) * (1LL << (8 * pp));
+        }
+        const int64_t row = row0 + r;
+        if (lane == r && row < pb.n) {
+            const float v = static_cast<float>((P4 * static_cast<double>(t) + PQ * sxd) * scale);
+            pb.y[row] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldg(pb.alpha + row) * v));
+        }
+    }
+}
+
+template <int MAXP>
+__global__ void __launch_bounds__(kThreads, 1) gemv_i8_kernel(const __grid_constant__ VecParams<MAXP> prm) {
+    extern __shared__ uint4 xq[];  // 64-K chunk c at uint4 c * kChunkF4: [word][plane]
+    __shared__ uint32_t red_mb[kThreads / 32];
+    __shared__ int red_s[kThreads / 32][4];
+    __shared__ int e_sh;
+    __shared__ double sx_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int pi = 0; pi < prm.count; ++pi) {
+        const VecProblem& pb = prm.prob[pi];
+        // max |x| of the row
+        uint32_t mb = 0;
+        for (int64_t i = tid; i < pb.k / 8; i += kThreads) {
+            const uint4 h = __ldg(reinterpret_cast<const uint4*>(pb.x) + i);
+            const uint32_t a = __vmaxu2(__vmaxu2(h.x & 0x7FFF7FFFu, h.y & 0x7FFF7FFFu),
+                                        __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));
+            mb = max(mb, max(a & 0xFFFFu, a >> 16));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        if (lane == 0) red_mb[warp] = mb;
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t t = red_mb[0];
+            for (int w = 1; w < kThreads / 32; ++w) t = max(t, red_mb[w]);
+            e_sh = exponent_of_max(t);
+        }
+        __syncthreads();
+        const int E = e_sh;
+        // digit planes into shared memory, and the planes' digit sums
+        int s4[4] = {0, 0, 0, 0};
+        for (int64_t g = tid; g < pb.k / 16; g += kThreads) {
+            const uint4 h0 = __ldg(reinterpret_cast<const uint4*>(pb.x + 16 * g));
+            const uint4 h1 = __ldg(reinterpret_cast<const uint4*>(pb.x + 16 * g) + 1);
+            const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            uint32_t pw[4][4];
+            digits16(hw, E, pw);
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+                xq[(g >> 2) * kChunkF4 + 4 * (g & 3) + pp] = make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) s4[pp] = __dp4a(static_cast<int>(pw[pp][q]), 0x01010101, s4[pp]);
+            }
+        }
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s4[pp] += __shfl_xor_sync(0xFFFFFFFFu, s4[pp], o);
+            if (lane == 0) red_s[warp][pp] = s4[pp];
+        }
+        __syncthreads();
+        if (tid == 0) {
+            long long t = 0;
+            for (int w = 0; w < kThreads / 32; ++w)
+                for (int pp = 0; pp < 4; ++pp) t += static_cast<long long>(red_s[w][pp]) * (1LL << (8 * pp));
+            sx_sh = static_cast<double>(t);
+        }
+        __syncthreads();
+        const double sxd = sx_sh, scale = exp2_int(E - 29);
+        const int64_t kq = pb.k / 4, nchunk = pb.k / 64;
+        const int64_t ntasks = (pb.n + pb.rows - 1) / pb.rows;
+        for (;;) {
+            int task = 0;
+            if (lane == 0) task = atomicAdd(pb.counter, 1);
+            task = __shfl_sync(0xFFFFFFFFu, task, 0);
+            if (task >= ntasks) break;
+            if (pb.rows == 4) row_task_i8<4>(pb, task, kq, nchunk, lane, prm.P4, prm.PQ, sxd, scale, xq);
+            else if (pb.rows == 2) row_task_i8<2>(pb, task, kq, nchunk, lane, prm.P4, prm.PQ, sxd, scale, xq);
+            else row_task_i8<1>(pb, task, kq, nchunk, lane, prm.P4, prm.PQ, sxd, scale, xq);
+        }
+        __syncthreads();  // the next matrix overwrites the planes
+    }
+}
+
 }  // namespace pqv
 
 // ------------------------------------------------------------------- host
@@ -1142,7 +1329,7 @@ struct XPlanes {
 };
 
 __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XPlanes prm) {
-    __shared__ float red[8];
+    __shared__ uint32_t red[8];
     __shared__ int e_sh;
     const int row = blockIdx.x / prm.slices, slice = blockIdx.x % prm.slices;
     const int xi = row / prm.m, j = row % prm.m;
@@ -1156,21 +1343,18 @@ __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XP
                                     __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));  // per half
         mb = max(mb, max(a & 0xFFFFu, a >> 16));
     }
-    float mx = __uint_as_float(mb << 16);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mb;
     __syncthreads();
     if (threadIdx.x == 0) {
-        float t = red[0];
-        for (int w = 1; w < 8; ++w) t = fmaxf(t, red[w]);
-        const uint32_t b = __float_as_uint(t);
-        // floor(log2 t) from the bits, subnormals included; 0 for an all-zero row
-        e_sh = t == 0.0f ? 0 : (b >> 23) ? static_cast<int>(b >> 23) - 127 : -118 - __clz(b);
+        uint32_t t = red[0];
+        for (int w = 1; w < 8; ++w) t = max(t, red[w]);
+        e_sh = exponent_of_max(t);
         if (slice == 0) prm.exps[xi][j] = e_sh;
     }
     __syncthreads();
-    const double sc = exp2_int(29 - e_sh);
+    const int E = e_sh;
     int8_t* pl = prm.planes[xi] + 4 * j * k;
     const int64_t groups = k / 16;
     const int64_t g1 = groups * (slice + 1) / prm.slices;
@@ -1178,20 +1362,8 @@ __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XP
         const uint4 h0 = reinterpret_cast<const uint4*>(xr + 16 * g)[0];
         const uint4 h1 = reinterpret_cast<const uint4*>(xr + 16 * g)[1];
         const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        uint32_t pw[4][4] = {};
-#pragma unroll
-        for (int f = 0; f < 16; ++f) {
-            const uint32_t bits = (f & 1) ? (hw[f >> 1] & 0xFFFF0000u) : (hw[f >> 1] << 16);
-            int v = __double2int_rn(static_cast<double>(__uint_as_float(bits)) * sc);
-            const int pos = 4 * (f & 3) + (f >> 2);
-#pragma unroll
-            for (int pp = 0; pp < 3; ++pp) {
-                const int dgt = ((v + 128) & 255) - 128;
-                v = (v - dgt) >> 8;
-                pw[pp][pos >> 2] |= static_cast<uint32_t>(dgt & 255) << (8 * (pos & 3));
-            }
-            pw[3][pos >> 2] |= static_cast<uint32_t>(v & 255) << (8 * (pos & 3));
-        }
+        uint32_t pw[4][4];
+        digits16(hw, E, pw);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp)
             *reinterpret_cast<uint4*>(pl + pp * k + 16 * g) = make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
@@ -1359,6 +1531,10 @@ static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Weights from which one row times a lone matrix takes the integer one-row
+// kernel (its x staging costs more per call, its loop less per weight).
+constexpr int64_t kIntegerRowWeights = int64_t{1} << 27;
+
 // A single activation row times a lone matrix, x fitting shared memory, takes
 // the CUDA-core path (measured faster there; a group of matrices runs faster
 // through the integer tensor-core mode, whose pipeline does not restart per
@@ -1374,7 +1550,7 @@ template <int MAXP>
 static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, void* workspace,
                               int64_t ws_bytes, cudaStream_t s) {
     pqv::VecParams<MAXP> V{};
-    if (!coeffs_of(q, V.P, V.Q)) return PQ_ERR_UNSUPPORTED;
+    if (!coeffs_of(q, V.P, V.Q) || !coeffs_i8(q, V.P4, V.PQ)) return PQ_ERR_UNSUPPORTED;
     if (!workspace || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return PQ_ERR_INVALID_ARG;
     int* counters = static_cast<int*>(workspace);
@@ -1395,13 +1571,16 @@ static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, voi
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(pqv::gemv_kernel<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(pqv::kMaxK / 64 * pqv::kChunkF4 * 16)) != cudaSuccess)
+        const int maxs = static_cast<int>(pqv::kMaxK / 64 * pqv::kChunkF4 * 16);
+        if (cudaFuncSetAttribute(pqv::gemv_i8_kernel<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 maxs) != cudaSuccess ||
+            cudaFuncSetAttribute(pqv::gemv_kernel<MAXP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 maxs) != cudaSuccess)
             return PQ_ERR_CUDA;
         attr_set[dev] = true;
     }
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pqv::gemv_kernel<MAXP>, pqv::kThreads,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pqv::gemv_i8_kernel<MAXP>, pqv::kThreads,
                                                       smem) != cudaSuccess || per_sm < 1)
         per_sm = 1;
     // rows per task (x loads are shared by the rows of a task): the largest
@@ -1411,7 +1590,16 @@ static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, voi
         V.prob[i].rows = pr[i].n >= 4 * warps ? 4 : pr[i].n >= 2 * warps ? 2 : 1;
     if (cudaMemsetAsync(counters, 0, static_cast<size_t>(count) * 4, s) != cudaSuccess)
         return PQ_ERR_CUDA;
-    pqv::gemv_kernel<MAXP><<<sm_count() * per_sm, pqv::kThreads, smem, s>>>(V);
+    // every CTA stages x: no more CTAs than the row tasks keep busy
+    int64_t tasks = 0;
+    for (int i = 0; i < count; ++i) tasks += (V.prob[i].n + V.prob[i].rows - 1) / V.prob[i].rows;
+    const int64_t need_ctas = (tasks + pqv::kThreads / 32 - 1) / (pqv::kThreads / 32);
+    const int64_t full = static_cast<int64_t>(sm_count()) * per_sm;
+    const int grid = static_cast<int>(need_ctas < full ? need_ctas : full);
+    if (pr[0].n * pr[0].k >= kIntegerRowWeights)
+        pqv::gemv_i8_kernel<MAXP><<<grid, pqv::kThreads, smem, s>>>(V);
+    else
+        pqv::gemv_kernel<MAXP><<<grid, pqv::kThreads, smem, s>>>(V);
     return cudaGetLastError() == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
 

@@ -316,7 +316,9 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  *     integer sums of digits times fields, combined in fp64.
  *   m > 16 (bf16 mode): weights decoded to bf16 1 + f'/4 (exact), products
  *     accumulated in fp32 by the tensor cores (kind::f16).
- * A lone matrix with m = 1 runs on the CUDA cores (fp32 fused multiply-adds).
+ * A lone matrix with m = 1 runs on the CUDA cores: below 2^27 weights with
+ * fp32 fused multiply-adds, from 2^27 weights with the integer mode's
+ * arithmetic (dp4a on the digit planes).
  * The bf16 and CUDA-core modes form y from sums over all k of x (1 + f'/4)
  * and of x, so their rounding scales with alpha sum_k |x|; where activations
  * far larger than the rest of their row meet zero levels (ternary, LSQ2),

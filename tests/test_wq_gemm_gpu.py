@@ -26,12 +26,23 @@ def _case(q, m, n, k, seed):
     return x, packed, a
 
 
-def _check(q, x, packed, a, y, grouped=False):
+INTEGER_ROW_WEIGHTS = 1 << 27  # one row times a lone matrix this large: integer kernel
+
+
+def _integer_mode(m, n, k, grouped):
+    """The integer arithmetic serves m <= 16, except one row times a lone
+    matrix with k <= 32768 below INTEGER_ROW_WEIGHTS (fp32 CUDA-core kernel)."""
+    if m > 16:
+        return False
+    return not (m == 1 and not grouped and k <= 32768 and n * k < INTEGER_ROW_WEIGHTS)
+
+
+def _check(q, x, packed, a, y, grouped=False, n_total=None):
     """y against the oracle within the matmul tolerance, derived from each
     mode's arithmetic: bf16 output rounding (2^-8 |ref|) plus an accumulation
     bound (1e-4 sum_k |x w|), and
-      integer mode (m <= 16, except one row times a lone matrix with
-      k <= 32768): the fixed-point conversion; every activation is rounded to
+      integer arithmetic (see _integer_mode): the fixed-point conversion;
+      every activation is rounded to
       a multiple of 2^(E-29) with 2^E <= max_k |x|, so |error| <=
       2^-30 max_k |x| sum_k |w|;
       bf16 and CUDA-core modes: y = alpha (P D + Q Sx) from fp32 sums over
@@ -49,7 +60,7 @@ def _check(q, x, packed, a, y, grouped=False):
     ones = xf @ np.abs(wd).T
     got = y.float().cpu().numpy().astype(np.float64)
     tol = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ones) + 1e-30
-    if m <= 16 and not (m == 1 and not grouped and k <= 32768):
+    if _integer_mode(m, packed.shape[0] if n_total is None else n_total, k, grouped):
         tol += 2.0 ** -30 * np.outer(xf.max(axis=1), np.abs(wd).sum(axis=1))
     else:
         tol += 2.0 ** -16 * np.outer(xf.sum(axis=1), np.abs(an).astype(np.float64))
@@ -239,7 +250,26 @@ def _check_rows(q, x, packed, a, y, rows, grouped=False):
     """_check on a subset of output features (the oracle runs on those rows)."""
     idx = torch.as_tensor(rows, device=packed.device)
     _check(q, x, packed.index_select(0, idx).contiguous(), a.index_select(0, idx).contiguous(),
-           y.index_select(1, idx).contiguous(), grouped=grouped)
+           y.index_select(1, idx).contiguous(), grouped=grouped, n_total=packed.shape[0])
+
+
+@pytest.mark.parametrize("q", [pq.PQ_SEQ2, pq.PQ_TERNARY])
+@pytest.mark.parametrize("outlier", [False, True])
+def test_one_row_large_lone_matrix(q, outlier):
+    """One activation row times a lone matrix of 2^27 weights (the integer
+    one-row kernel), with ordinary activations and with one 1e20 value among
+    1e-20 ones; 128 sampled output features against the oracle."""
+    m, n, k = 1, 8192, 16384
+    x, packed, a = _case(q, m, n, k, seed=77)
+    if outlier:
+        t = np.full(k, np.float32(1e-20), np.float32) * np.random.default_rng(3).choice([-1, 1], k).astype(np.float32)
+        t[k // 5] = np.float32(1e20)
+        x = _bf16_from_bits((t.view(np.uint32) >> 16).astype(np.uint16)[None, :])
+    y = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    rows = sorted(set([0, n - 1] + list(np.random.default_rng(9).choice(n, 126, replace=False))))
+    _check_rows(q, x, packed, a, y, rows)
 
 
 def test_wq_gemm_full_size_grouped_sampled():
