@@ -45,9 +45,11 @@
 // (deterministic).
 //
 // Roles (19 warps): 8 decode warps (TMEM lane quarter = warp % 4, K half =
-// warp / 4), 4 epilogue warps, 4 activation permuters, one codes producer,
-// one activation producer, one MMA issuer. The activation ring is deeper
-// than the A ring and has its own barriers, so decoding never waits on it. Every mbarrier wait is bounded: on giving up the kernel
+// warp / 4), 4 epilogue warps, 4 activation permuters (in the integer mode
+// the planes arrive already in MMA order and they only pass the stage on),
+// one codes producer, one activation producer, one MMA issuer. The
+// activation ring is deeper than the A ring and has its own barriers, so
+// decoding never waits on it. Every mbarrier wait is bounded: on giving up the kernel
 // records a device status and an abort flag that ends every role's loop,
 // waits (bounded) for its own copies and MMAs in flight, frees its TMEM and
 // returns.
@@ -1639,6 +1641,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
     const int64_t base = pl.partials ? partial_bytes(pl, m) + round256(pl.blocks * 4) : 0;
     // integer mode: one digit-plane set per distinct activation matrix
     int slot[kMaxBatch];
+    int64_t planes_off[kMaxBatch];  // workspace offsets of each set's planes
     int nslots = 0;
     XPlanes X{};
     int64_t need = base;
@@ -1650,8 +1653,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
             if (t == nslots) {
                 X.x[t] = pr[i].x_bf16;
                 X.k[t] = pr[i].k;
-                X.planes[t] = reinterpret_cast<int8_t*>(need);  // offsets until the base is known
-                X.exps[t] = reinterpret_cast<int*>(need + round256(4 * m * pr[i].k));
+                planes_off[t] = need;  // exponents follow the planes
                 need += xplanes_bytes(m, pr[i].k);
                 ++nslots;
             }
@@ -1669,9 +1671,9 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         P.c.partial = static_cast<float*>(workspace);
         P.c.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + partial_bytes(pl, m));
         for (int t = 0; t < nslots; ++t) {
-            X.planes[t] = static_cast<int8_t*>(workspace) + reinterpret_cast<intptr_t>(X.planes[t]);
-            X.exps[t] = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                               reinterpret_cast<intptr_t>(X.exps[t]));
+            X.planes[t] = static_cast<int8_t*>(workspace) + planes_off[t];
+            X.exps[t] = reinterpret_cast<int*>(static_cast<char*>(workspace) + planes_off[t] +
+                                               round256(4 * m * X.k[t]));
         }
     }
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
