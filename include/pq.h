@@ -86,7 +86,7 @@ typedef enum {
 typedef enum {
     PQ_OK = 0,
     PQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, bad pack shape */
-    PQ_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve */
+    PQ_ERR_UNSUPPORTED = 2, /* valid request the library does not serve */
     PQ_ERR_MISALIGNED = 3,  /* reserved: misaligned input is served by the element path */
     PQ_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
     PQ_ERR_TIMEOUT = 5      /* reserved for bounded device-side waits */

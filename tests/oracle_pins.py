@@ -50,7 +50,7 @@ def printed_levels():
            TERNARY: sorted(frac_f32(v) for v in g["ternary_levels"]["values"])}
     for b, q in (("2", LSQ2), ("3", LSQ3), ("4", LSQ4)):
         out[q] = [float(v) for v in g["lsq_levels"]["values"][b]]
-    # BASELINE-literal 2-bit SEQ: {-1.5,-0.5,0.5,1.5}/1.5
+    # the divisor-1.5 reading of the 2-bit SEQ formula: {-1.5,-0.5,0.5,1.5}/1.5
     out[SEQ2_B] = sorted(f32(Fraction(v).limit_denominator(4) / Fraction(3, 2))
                          for v in g["seq2_code_domain"]["values"])
     out[BINARY] = [-1.0, 1.0]
