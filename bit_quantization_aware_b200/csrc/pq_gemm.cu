@@ -70,7 +70,6 @@ namespace pqg {
 constexpr int kFeat = 127;             // weight rows per tile; TMEM lane 127 = ones
 constexpr int kStageK = 256;           // K per MMA stage: 128 TMEM columns of A, 16 MMAs
 constexpr int kChunkK = 512;           // K per codes chunk: 128 B per row
-constexpr int kStagesPerChunk = kChunkK / kStageK;
 constexpr int kMinK = 128;             // K granularity of the problem
 constexpr int kDecWarps = 8;           // warps 0..7
 constexpr int kEpiWarp0 = 8;           // warps 8..11
@@ -840,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
                 __syncwarp();
                 tmem_ld16(d + c0, v);
-                if (I8) {
+                if constexpr (I8) {
                     // columns 4j .. 4j + 3 are activation row j's digit planes;
                     // x = digits * 2^(E - 29)
                     float o[4];
@@ -861,23 +860,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else if (c0 / 4 < p.m4) {
                         *reinterpret_cast<float4*>(prow + c0 / 4) = make_float4(o[0], o[1], o[2], o[3]);
                     }
-                    continue;
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = fmaf(p.P, v[j], p.Q * sx[c0 + j]);
-                if (!valid_row) continue;
-                if (full) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (c0 + j < p.m)
-                            pb.y[(c0 + j) * pb.n + feat] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[j]));
                 } else {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        if (c0 + 4 * q4 < p.m4)
-                            *reinterpret_cast<float4*>(prow + c0 + 4 * q4) = make_float4(
-                                v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                    for (int j = 0; j < 16; ++j) v[j] = fmaf(p.P, v[j], p.Q * sx[c0 + j]);
+                    if (!valid_row) continue;
+                    if (full) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (c0 + j < p.m)
+                                pb.y[(c0 + j) * pb.n + feat] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[j]));
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            if (c0 + 4 * q4 < p.m4)
+                                *reinterpret_cast<float4*>(prow + c0 + 4 * q4) = make_float4(
+                                    v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                    }
                 }
             }
             tc_fence_before();
