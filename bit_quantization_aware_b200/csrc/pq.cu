@@ -98,11 +98,20 @@ __device__ __forceinline__ void st_stream(T* p, T v) {
 #endif
 }
 
+// Eight consecutive fp32 values (32-byte aligned) as one 256-bit access, so
+// a warp's access covers 1024 contiguous bytes (two 16-byte accesses per
+// lane would each cover only half of every 32-byte sector).
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+#if PQ_LD_HINT == 0
+    asm("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "l"(p));
+#else
     const float4 a = ld_stream(reinterpret_cast<const float4*>(p));
     const float4 b = ld_stream(reinterpret_cast<const float4*>(p) + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+#endif
 }
 
 __device__ __forceinline__ void load8_tail(const float* p, int n, float (&v)[8]) {
@@ -111,8 +120,14 @@ __device__ __forceinline__ void load8_tail(const float* p, int n, float (&v)[8])
 }
 
 __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+#if PQ_ST_HINT == 0
+    asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]),
+                 "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+#else
     st_stream(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
     st_stream(reinterpret_cast<float4*>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+#endif
 }
 
 __device__ __forceinline__ void store8_tail(float* p, int n, const float (&v)[8]) {
@@ -914,13 +929,13 @@ static void launch_dequant(const Batch& b, cudaStream_t s) {
 
 // ------------------------------------------------------- validation
 static bool fwd_vec_ok(const pq_matrix_t& m, int bits) {
-    return m.cols % 8 == 0 && aligned(m.w, 16) &&
+    return m.cols % 8 == 0 && aligned(m.w, 32) &&
            (!m.wq_bf16_out || aligned(m.wq_bf16_out, 16)) &&
            (!m.packed_out || aligned(m.packed_out, bits == 2 ? 2 : 4));
 }
 
 static bool bwd_vec_ok(const pq_matrix_t& m) {
-    return m.cols % 8 == 0 && aligned(m.w, 16) && aligned(m.g_bf16, 16) && aligned(m.dw_out, 16);
+    return m.cols % 8 == 0 && aligned(m.w, 32) && aligned(m.g_bf16, 16) && aligned(m.dw_out, 32);
 }
 
 static pq_status_t check_fwd(int bits, const pq_matrix_t& m) {
@@ -1170,8 +1185,8 @@ static pq_status_t bwd_adamw_impl(int q, int32_t n, const pq_adamw_matrix_t* mat
             if (m.rows == 0) continue;
             // rows without columns still take an AdamW step on alpha with
             // d(alpha) = 0: they go through the element path
-            const bool v = m.cols > 0 && m.cols % 8 == 0 && aligned(m.w, 16) &&
-                           aligned(m.g_bf16, 16) && aligned(m.m_w, 16) && aligned(m.v_w, 16);
+            const bool v = m.cols > 0 && m.cols % 8 == 0 && aligned(m.w, 32) &&
+                           aligned(m.g_bf16, 16) && aligned(m.m_w, 32) && aligned(m.v_w, 32);
             if (v != vec) continue;
             if (b.b.n == kMaxBatch) flush();
             AdamDesc& d = b.b.m[b.b.n++];
@@ -1249,7 +1264,7 @@ static pq_status_t reduce_bwd_adamw_impl(int q, int32_t n_src, const uint16_t* c
             const pq_shard_t& m = sh[i];
             if (m.rows == 0) continue;
             const bool v = src_aligned && m.cols > 0 && m.cols % 8 == 0 && m.g_offset % 8 == 0 &&
-                           aligned(m.w, 16) && aligned(m.m_w, 16) && aligned(m.v_w, 16);
+                           aligned(m.w, 32) && aligned(m.m_w, 32) && aligned(m.v_w, 32);
             if (v != vec) continue;
             if (b.b.n == kMaxBatch) flush();
             ShardDesc& d = b.b.m[b.b.n++];

@@ -21,10 +21,10 @@
  *   - rows == 0 or cols == 0 is valid and launches nothing (array pointers
  *     may then be NULL), except that the backward writes d(alpha) = 0 for
  *     rows > 0, cols == 0 (dalpha_out must then be valid).
- *   - Any alignment is accepted. The fast path needs cols % 8 == 0, 16-byte
- *     aligned fp32/bf16 arrays and a packed buffer aligned to 2 bytes
- *     (2-bit codes) or 4 bytes (4-bit codes); otherwise a slower element
- *     path with the same results runs.
+ *   - Any alignment is accepted. The fast path needs cols % 8 == 0, 32-byte
+ *     aligned fp32 arrays (weights, dW, moments), 16-byte aligned bf16 arrays
+ *     and a packed buffer aligned to 2 bytes (2-bit codes) or 4 bytes (4-bit
+ *     codes); otherwise a slower element path with the same results runs.
  *   - Preconditions not checked on the device: w finite, alpha finite and
  *     > 0, and output buffers that alias no input. Violations give
  *     unspecified results (no fault for in-bounds buffers).
