@@ -9,9 +9,10 @@
 //   one launch per phase, with no per-matrix ramp-up and tail.
 // * A CTA of 256 threads splits into row groups of TPR threads (a power of
 //   two, 1..256, chosen per matrix so that each thread owns about eight
-//   chunks of 8 weights of its row). Each thread issues the 16-byte loads of
-//   several chunks (4 in the forward, 2 in the backward) before computing
-//   any of them.
+//   chunks of 8 weights of its row). Each thread issues the loads of several
+//   chunks (4 in the forward, 2 in the backward) before computing any of
+//   them; a chunk's 8 fp32 values move as one 256-bit access, so a warp
+//   instruction covers 1024 contiguous bytes.
 // * A persistent grid (the occupancy limit; the backward's registers are
 //   capped for 4 CTAs per SM) walks the units in order, so concurrent CTAs
 //   stream neighbouring rows. An optional bulk L2 prefetch of each CTA's
