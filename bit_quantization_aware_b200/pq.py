@@ -313,8 +313,10 @@ def pq_wq_gemm_workspace_bytes(q, m, n, k) -> int:
 
 
 def pq_wq_gemm(q, x, packed, alpha, y_out, workspace=None, stream=None):
-    """Y = X (alpha * levels(codes))^T on the tensor cores; x bf16 [m, k],
-    packed uint8 [n, k/4], alpha fp32 [n], y_out bf16 [m, n]."""
+    """Y = X (alpha * levels(codes))^T; x bf16 [m, k], packed uint8 [n, k/4],
+    alpha fp32 [n], y_out bf16 [m, n]. Tensor cores (integer mode for
+    m <= 16, bf16 beyond), one row times this one matrix on the CUDA cores;
+    include/pq.h states each mode's arithmetic and error bound."""
     m, k = x.shape
     n = packed.shape[0]
     if (packed.dim() != 2 or packed.shape[1] * 8 != k * pq_code_bits(q)
