@@ -104,7 +104,7 @@ def test_small_shapes(q, shape):
 
 
 @pytest.mark.parametrize("q", ALLQ)
-@pytest.mark.parametrize("offset", [1, 2, 3])
+@pytest.mark.parametrize("offset", [1, 2, 3, 4, 8])  # 4: fp32 16-byte aligned only; 8: 32-byte
 def test_misaligned_pointers(q, offset):
     w, a, g = make_case(37, 1024, q, seed=offset)
     wq, pk, pk2, dw, da, gs = run_gpu(q, w, a, g, True, offset=offset)
@@ -559,7 +559,8 @@ def _check_adamw(q, w, a, g, mw, vw, ma, va, gs, t, offset=0):
 
 @pytest.mark.parametrize("q", ALLQ)
 @pytest.mark.parametrize("shape,offset", [((33, 1032), 0), ((7, 1000), 0), ((5, 12), 0),
-                                          ((64, 4096), 0), ((9, 2048), 1), ((3, 0), 0)])
+                                          ((64, 4096), 0), ((9, 2048), 1), ((9, 2048), 4),
+                                          ((9, 2048), 8), ((3, 0), 0)])
 def test_bwd_adamw_two_steps(q, shape, offset):
     """Fused backward + AdamW: two consecutive steps (the second from the
     GPU's state), weights and moments bit-exact against the oracle."""
