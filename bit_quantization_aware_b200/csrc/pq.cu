@@ -10,7 +10,7 @@
 // * A CTA of 256 threads splits into row groups of TPR threads (a power of
 //   two, 1..256, chosen per matrix so that each thread owns about eight
 //   chunks of 8 weights of its row). Each thread issues the loads of several
-//   chunks (4 in the forward, 2 in the backward) before computing any of
+//   chunks (2 in the forward and the backward) before computing any of
 //   them; a chunk's 8 fp32 values move as one 256-bit access, so a warp
 //   instruction covers 1024 contiguous bytes.
 // * A persistent grid (the occupancy limit; the backward's registers are
@@ -51,7 +51,7 @@
 #define PQ_CHUNKS_PER_THREAD 8
 #endif
 #ifndef PQ_FWD_UNROLL
-#define PQ_FWD_UNROLL 4
+#define PQ_FWD_UNROLL 2
 #endif
 #ifndef PQ_BWD_UNROLL
 #define PQ_BWD_UNROLL 2
