@@ -40,12 +40,17 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--op", choices=["quantizer", "dequant", "bwd_adamw", "wq_gemm"],
+    p.add_argument("--op", choices=["quantizer", "dequant", "bwd_adamw", "wq_gemm", "sharded"],
                    default="quantizer",
                    help="quantizer: the forward+backward step (the headline); "
                         "dequant: packed codes -> bf16 over the same layer set; "
                         "bwd_adamw: the backward fused with the AdamW step; "
-                        "wq_gemm: Y = X W^T from the packed 2-bit codes on the tensor cores")
+                        "wq_gemm: Y = X W^T from the packed 2-bit codes on the tensor cores; "
+                        "sharded: the row-sharded step with its ranks emulated on one GPU")
+    p.add_argument("--world", type=int, default=2,
+                   help="sharded: emulated ranks (buffer sets on the one GPU)")
+    p.add_argument("--layers", type=int, default=8,
+                   help="sharded: layers of the Llama-3-8B-shaped set (memory grows with world)")
     p.add_argument("--m", type=int, default=16,
                    help="wq_gemm: activation rows (tokens of a decode batch), 1..128")
     p.add_argument("--shape", default="llama3_8b", choices=["llama3_8b", "16384"],
@@ -811,6 +816,100 @@ def run_wq_gemm(args):
     return 0
 
 
+def sharded_bytes(weights: int, world: int) -> dict:
+    """Algorithmic bytes of one row-sharded step over `weights` weights (all
+    ranks together; scales and d(alpha) are per-row and negligible): pack
+    reads each owned fp32 weight and writes 0.25 B of codes; every rank's
+    gather + dequantization reads all codes and writes all bf16 weights;
+    the reduce step reads `world` bf16 gradient rows per owned weight plus
+    w, m, v and writes w, m, v."""
+    return {"pack": int(4.25 * weights),
+            "gather_dequant": int(world * 2.25 * weights),
+            "reduce_bwd_adamw": int((2 * world + 24) * weights)}
+
+
+def run_sharded(args):
+    """The row-sharded owner-computes step (pack own rows; gather + dequantize
+    everyone's codes; reduce the replicas' gradients + backward + AdamW on
+    own rows) for `--world` ranks emulated as buffer sets on one GPU, over
+    the first `--layers` layers of the Llama-3-8B-shaped set. Peer buffers
+    are local device memory here, so this measures the kernels' HBM
+    efficiency, not NVLink. Each phase runs for every rank in turn, timed by
+    CUDA events. Prints one JSON line."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.sharded import LocalPeers, ShardedQuantStep
+
+    torch.cuda.set_device(0)
+    q, world = pq.PQ_SEQ2, args.world
+    mats = I.llama3_8b_set()[: 7 * args.layers]
+    peers = LocalPeers(world)
+    ranks = [ShardedQuantStep(mats, q, k, world, peers, device="cuda:0") for k in range(world)]
+    for i, m in enumerate(mats):
+        w = I.normal_weights(m.rows, m.cols, seed=3, stream=i, device="cuda:0")
+        a = I.alpha_init(w, q)
+        for r in ranks:
+            r.load_full(i, w, a)
+        del w, a
+    for k, r in enumerate(ranks):
+        for i, m in enumerate(mats):
+            r.g(i).copy_(I.grad_bf16(m.rows, m.cols, seed=4 + k, stream=64 + i, device="cuda:0"))
+    torch.cuda.synchronize()
+    t = [0]
+
+    def phase(fn):
+        for r in ranks:
+            fn(r)
+
+    def step_fns():
+        t[0] += 1
+        hw, ha = pq.adamw(t[0], 2e-5), pq.adamw(t[0], 1e-4)
+        return [("pack", lambda r: r.pack_shards()),
+                ("gather_dequant", lambda r: r.gather_dequant()),
+                ("reduce_bwd_adamw", lambda r: r.reduce_step(hw, ha))]
+
+    for _ in range(max(args.warmup, 1)):
+        for _, fn in step_fns():
+            phase(fn)
+    torch.cuda.synchronize()
+    names = ["pack", "gather_dequant", "reduce_bwd_adamw"]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * args.steps)]
+    for s_ in range(args.steps):
+        for j, (_, fn) in enumerate(step_fns()):
+            ev[4 * s_ + j].record()
+            phase(fn)
+        ev[4 * s_ + 3].record()
+    torch.cuda.synchronize()
+    ms = {n: sum(ev[4 * s_ + j].elapsed_time(ev[4 * s_ + j + 1]) for s_ in range(args.steps)) / args.steps
+          for j, n in enumerate(names)}
+    total = sum(ms.values())
+    weights = I.total_weights(mats)
+    nbytes = sharded_bytes(weights, world)
+    peak, kind = measured_peaks()
+    phases = {n: {"ms_per_step": ms[n], "algorithmic_bytes": nbytes[n],
+                  "GB_s": nbytes[n] / (ms[n] * 1e-3) / 1e9,
+                  "frac_of_peak": nbytes[n] / (ms[n] * 1e-3) / 1e9 / peak} for n in names}
+    allb = sum(nbytes.values())
+    print(json.dumps({
+        "metric": "row-sharded step (ranks emulated on one GPU) Gweights/s", "op": "sharded",
+        "value": weights / (total * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total,
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"llama3_8b_first{args.layers}layers_seq2_sharded_world{world}_emulated",
+                   "weights": weights, "world": world,
+                   "note": "all ranks' work on one GPU in turn; peer reads are local HBM reads"},
+        "roofline": {"bound": "hbm", "kernel": "pack, dequant and reduce_bwd_adamw units kernels",
+                     "achieved": allb / (total * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": allb / (total * 1e-3) / 1e9 / peak, "traffic": None,
+                     "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_step": allb},
+        "phases": phases,
+        # one batched launch per phase per rank (every batch here fits one launch)
+        "gpu_launches": 3 * world * args.steps}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -821,6 +920,8 @@ def main():
         return run_bwd_adamw(args)
     if args.op == "wq_gemm":
         return run_wq_gemm(args)
+    if args.op == "sharded":
+        return run_sharded(args)
     return run_ours(args)
 
 
