@@ -3,12 +3,29 @@ Llama-3-8B-shaped linear set (32 layers of q/o 4096x4096, k/v 1024x4096,
 gate/up 14336x4096, down 4096x14336; 2-bit SEQ, bf16 dequant output).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--op quantizer|dequant|bwd_adamw|wq_gemm|sharded] [--no-extras]
 
 One step = one forward over every matrix, then one backward over every
 matrix, with all inputs resident in HBM (synthetic, seeded; about 84 GB per
 GPU, far larger than L2, so no flush is needed between steps). Each rank
 runs the full set on its own GPU (weak scaling; the quantizer shards by
 matrix and row and needs no collective). Rank 0 prints one JSON line.
+
+With one GPU the default run adds to that line, after the headline's timed
+region:
+
+* ``per_config``: forward, backward and forward + backward of the other
+  four workloads (one 256x1024 weight with packed codes under both 2-bit SEQ
+  readings; one 2048x8192 weight under five quantizers; the 1B-class stack;
+  one 16384x16384 heavy-tailed weight with planted ties and clip bounds,
+  fused packed export and the standalone packer), each phase timed after an
+  L2 flush, with the CPU oracle's rate on the same kind of input beside it;
+* ``next``: the rows built on the quantizer, on the same Llama-3-8B-shaped
+  set: dequantization of packed codes, the backward fused with AdamW (and
+  the unfused backward + torch AdamW beside it), the weight-only 2-bit
+  matmul at 1, 16 and 128 activation rows (and cuBLAS bf16 on the
+  dequantized weights beside it), and the row-sharded step with two ranks
+  emulated on the one GPU.
 
 ``--impl reference`` times the CPU oracle (the plain C reference used by
 the tests) on a bounded sample of the same workload on the host cores.
@@ -32,9 +49,11 @@ UNIT = "Gweights/s"
 WORKLOAD = "llama3_8b_linear_set_seq2_fwd_ste_bwd"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 2 ** 20
+MAX_SHARDED_WORLD = 16  # gradient sources one reduce launch accepts
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=10)
@@ -47,8 +66,14 @@ def parse():
                         "bwd_adamw: the backward fused with the AdamW step; "
                         "wq_gemm: Y = X W^T from the packed 2-bit codes on the tensor cores; "
                         "sharded: the row-sharded step with its ranks emulated on one GPU")
+    p.add_argument("--no-extras", action="store_true",
+                   help="quantizer: print the headline only (no per_config, no next)")
+    p.add_argument("--config-steps", type=int, default=20,
+                   help="timed iterations of each per_config measurement (median reported)")
+    p.add_argument("--extra-steps", type=int, default=10,
+                   help="timed iterations of each next-row measurement")
     p.add_argument("--world", type=int, default=2,
-                   help="sharded: emulated ranks (buffer sets on the one GPU)")
+                   help=f"sharded: emulated ranks (buffer sets on the one GPU), 1..{MAX_SHARDED_WORLD}")
     p.add_argument("--layers", type=int, default=8,
                    help="sharded: layers of the Llama-3-8B-shaped set (memory grows with world)")
     p.add_argument("--m", type=int, default=16,
@@ -59,9 +84,17 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=15.0,
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
-    return p.parse_args()
+    a = p.parse_args(argv)
+    if not 1 <= a.world <= MAX_SHARDED_WORLD:
+        p.error(f"--world must be between 1 and {MAX_SHARDED_WORLD} "
+                f"(the gradient sources one reduce launch sums), got {a.world}")
+    if not 1 <= a.layers <= 32:
+        p.error(f"--layers must be between 1 and 32, got {a.layers}")
+    if not 1 <= a.m <= 128:
+        p.error(f"--m must be between 1 and 128, got {a.m}")
+    return a
 
 
 def config_dict(n_gpus, weights_per_gpu):
@@ -197,51 +230,85 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def physical_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local])
+        except (ValueError, IndexError):
+            pass
+    return local
+
+
 # ---------------------------------------------------------------- reference
 def workload_weights():
     from bit_quantization_aware_b200 import inputs as I
     return I.total_weights(I.llama3_8b_set())
 
 
-def sample_rows_for_oracle(cpu_seconds):
-    """Rows drawn from every matrix kind of one layer so that the oracle's
-    forward + backward takes about ``cpu_seconds`` on one core."""
+def oracle_seconds_per_weight(q, cols, pack=False):
+    """Single-thread oracle time per weight of forward (+ packed codes) +
+    backward, calibrated on 8 full-width rows."""
     import numpy as np
+    import torch
 
     from bit_quantization_aware_b200 import inputs as I
     from oracle import pq_oracle
-    import torch
-
-    mats = [m for m in I.llama3_8b_set() if m.layer == 0]
-    q = I.SEQ2
-    # calibrate with 8 rows of the widest matrix
-    w = I.normal_weights(8, 14336, seed=0, stream=6, device="cpu")
+    w = I.normal_weights(8, cols, seed=0, stream=6, device="cpu")
     a = I.alpha_init(w, q)
-    g = I.grad_bf16(8, 14336, seed=0, stream=70, device="cpu")
+    g = I.grad_bf16(8, cols, seed=0, stream=70, device="cpu")
     gn = g.view(torch.int16).numpy().view(np.uint16)
     t0 = time.perf_counter()
-    pq_oracle.fwd(q, w.numpy(), a.numpy())
+    pq_oracle.fwd(q, w.numpy(), a.numpy(), pack=pack)
     pq_oracle.bwd(q, w.numpy(), a.numpy(), gn, 1.0)
-    per_weight = (time.perf_counter() - t0) / w.numel()
-    total = cpu_seconds / max(per_weight, 1e-12)
-    per_kind = total / len(mats)
+    return (time.perf_counter() - t0) / w.numel()
+
+
+def oracle_sample(mats, q, seconds, *, seed=0, dist="normal", lsq_rule="lsq",
+                  plant=False, pack=False):
+    """Full-width rows of every matrix in ``mats`` (the same draws and
+    scales as the GPU inputs of that workload, on the host) so that the
+    oracle's forward + backward takes about ``seconds`` on one core; whole
+    matrices when they fit."""
+    import numpy as np
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    per_weight = oracle_seconds_per_weight(q, max(m.cols for m in mats), pack)
+    per_mat = seconds / max(per_weight, 1e-12) / len(mats)
     sample = []
     for m in mats:
-        rows = max(1, min(m.rows, int(per_kind // m.cols)))
-        wm = I.normal_weights(rows, m.cols, seed=0, stream=m.proj, device="cpu")
-        am = I.alpha_init(wm, q)
-        gm = I.grad_bf16(rows, m.cols, seed=0, stream=m.proj + 64, device="cpu")
+        rows = max(1, min(m.rows, int(per_mat // m.cols)))
+        sid = 8 * m.layer + m.proj
+        if dist == "normal":
+            wm = I.normal_weights(rows, m.cols, seed=seed, stream=sid, device="cpu")
+        else:
+            wm = I.student_t3_weights(rows, m.cols, seed=seed, stream=sid, device="cpu")
+        am = I.alpha_init(wm, q, lsq_rule=lsq_rule)
+        if plant:
+            I.plant_boundaries(wm, am, frac=0.01, seed=seed)
+        gm = I.grad_bf16(rows, m.cols, seed=seed, stream=sid + 64, device="cpu")
         sample.append((m, wm.numpy(), am.numpy(), gm.view(torch.int16).numpy().view(np.uint16)))
     return sample
 
 
-def time_oracle(sample):
+def sample_rows_for_oracle(cpu_seconds):
+    """Rows drawn from every matrix kind of one layer of the Llama-3-8B-shaped
+    set so that the oracle's forward + backward takes about ``cpu_seconds``
+    on one core."""
+    from bit_quantization_aware_b200 import inputs as I
+    mats = [m for m in I.llama3_8b_set() if m.layer == 0]
+    return oracle_sample(mats, I.SEQ2, cpu_seconds)
+
+
+def time_oracle(sample, q=3, pack=False):
+    """Runs the oracle's forward (+ packed codes) and backward over a sample;
+    returns (weights, seconds)."""
     from oracle import pq_oracle
-    q = 3  # SEQ2
     t0 = time.perf_counter()
     n = 0
     for m, w, a, g in sample:
-        pq_oracle.fwd(q, w, a)
+        pq_oracle.fwd(q, w, a, pack=pack)
         pq_oracle.bwd(q, w, a, g, pq_oracle.default_grad_scale(q, m.cols))
         n += w.size
     dt = time.perf_counter() - t0
@@ -283,6 +350,518 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------- timing helpers
+class L2Flush:
+    """Writes a buffer of twice the L2 size, so that the next kernel finds
+    none of its inputs in L2 (a real step runs a matmul between the
+    quantizer's phases)."""
+
+    def __init__(self, device):
+        import torch
+        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
+        self.k = 0
+
+    def __call__(self):
+        self.k += 1
+        self.buf.fill_(self.k)
+
+
+def timed_phases(fns, steps, warmup, flush):
+    """Runs ``fns`` (name -> callable) in order ``warmup + steps`` times,
+    each call bracketed by CUDA events on the current stream and preceded
+    by an L2 flush (outside the events). Returns, per name, the median
+    milliseconds over the timed iterations, the medians of the sums over
+    all phases, and the library's kernel launches per iteration."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    names = list(fns)
+    for _ in range(max(warmup, 1)):
+        for n in names:
+            flush()
+            fns[n]()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in names] for _ in range(steps)]
+    l0 = pq.pq_launch_count()
+    for it in range(steps):
+        for j, n in enumerate(names):
+            flush()
+            ev[it][j][0].record()
+            fns[n]()
+            ev[it][j][1].record()
+    torch.cuda.synchronize()
+    launches = (pq.pq_launch_count() - l0) / steps
+    per = {n: [ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(steps)]
+           for j, n in enumerate(names)}
+    med = {n: statistics.median(v) for n, v in per.items()}
+    return med, per, launches
+
+
+def phase_entry(ms, weights, nbytes, peak):
+    sec = ms * 1e-3
+    return {"ms": ms, "Gweights_s": weights / sec / 1e9, "GB_s": nbytes / sec / 1e9,
+            "frac_of_peak": nbytes / sec / 1e9 / peak, "algorithmic_bytes": nbytes}
+
+
+def time_graph(fn, steps, warmup):
+    """Captures ``fn`` in a CUDA graph (after two eager runs on a side
+    stream) and times ``steps`` replays; returns (ms per replay, graph,
+    library kernel launches per replay)."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    l0 = pq.pq_launch_count()
+    with torch.cuda.graph(g):
+        fn()
+    launches = pq.pq_launch_count() - l0
+    for _ in range(max(warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, g, launches
+
+
+def time_eager(fn, steps, warmup):
+    """Times ``steps`` back-to-back calls of ``fn`` with CUDA events on the
+    current stream; returns (ms per call, library launches per call)."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    for _ in range(max(warmup, 1)):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = pq.pq_launch_count()
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, (pq.pq_launch_count() - l0) / steps
+
+
+# ---------------------------------------------------------------- per config
+def per_config_cases():
+    """The four workloads besides the headline, with the seeds, draws and
+    scale initialisations of their parity tests (seed = workload number - 1)."""
+    from bit_quantization_aware_b200 import inputs as I
+    Q = I
+    return [
+        dict(key="1_single_256x1024_pack", mats=[I.Matrix("w", 256, 1024, 0, 0)],
+             quantizers=[("seq2", Q.SEQ2, "lsq"), ("seq2_b", Q.SEQ2_B, "lsq")],
+             pack=True, dist="normal", seed=0, plant=False, standalone_pack=False,
+             what="one 256x1024 N(0,0.02) weight, alpha = max|w_row|, forward with packed "
+                  "codes + backward; launch-bound and L2-resident (a parity case)"),
+        dict(key="2_bit_width_sweep_2048x8192", mats=[I.Matrix("w", 2048, 8192, 0, 0)],
+             quantizers=[("binary", Q.BINARY, "lsq"), ("ternary", Q.TERNARY, "lsq"),
+                         ("seq2", Q.SEQ2, "lsq"), ("lsq3", Q.LSQ3, "lsq"),
+                         ("lsq4", Q.LSQ4, "lsq")],
+             pack=False, dist="normal", seed=1, plant=False, standalone_pack=False,
+             what="one 2048x8192 N(0,0.02) weight; alpha = mean|w_row| (binary), "
+                  "max|w_row| (ternary, seq2), 2 mean|w_row|/sqrt(Qp) (lsq3, lsq4)"),
+        dict(key="3_llama_1b_stack", mats=I.llama_1b_stack(),
+             quantizers=[("seq2", Q.SEQ2, "lsq")],
+             pack=False, dist="normal", seed=2, plant=False, standalone_pack=False,
+             what="24 layers: q,o 2048x2048; k,v 512x2048; gate,up 5632x2048; "
+                  "down 2048x5632; one batched launch per phase"),
+        dict(key="5_student_t_16384_planted_pack", mats=[I.Matrix("t3.16384", 16384, 16384, 0, 0)],
+             quantizers=[("seq2", Q.SEQ2, "lsq"), ("ternary", Q.TERNARY, "lsq")],
+             pack=True, dist="student_t", seed=4, plant=True, standalone_pack=True,
+             what="one 16384x16384 Student-t(3)*0.02 weight, 1% of entries planted on "
+                  "clip bounds and rounding ties; forward with fused packed codes + "
+                  "backward; the standalone packer timed beside it"),
+    ]
+
+
+def measure_case(case, steps, warmup, peak, device, flush, oracle_seconds):
+    """One per_config workload: every quantizer's forward, backward and
+    forward + backward (median of ``steps`` after an L2 flush each), the
+    standalone packer where asked, and the oracle's rate on a sample."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.step import QuantStep
+    out = {"what": case["what"], "weights": I.total_weights(case["mats"]),
+           "l2_flush": "before every phase (a buffer of twice the L2 size is written)"}
+    for name, q, rule in case["quantizers"]:
+        step = QuantStep(case["mats"], q, device=device, pack=case["pack"])
+        step.generate(seed=case["seed"], dist=case["dist"], lsq_rule=rule)
+        planted = None
+        if case["plant"]:
+            b = step.bufs[0]
+            n, hit = I.plant_boundaries(b.w, b.alpha, frac=0.01, seed=case["seed"])
+            planted = {"entries": n, "exactly_on_target": hit}
+        fns = {"fwd": step.fwd_all, "bwd": step.bwd_all}
+        if case["standalone_pack"]:  # one matrix: pq_pack_codes into its own buffer
+            b = step.bufs[0]
+            pk_alone = torch.empty_like(b.packed)
+            fns["pack_standalone"] = lambda: pq.pq_pack_codes(step.q, b.w, b.alpha, pk_alone)
+        med, per, launches = timed_phases(fns, steps, warmup, flush)
+        fb = statistics.median([a + b for a, b in zip(per["fwd"], per["bwd"])])
+        w = step.weights
+        entry = {"fwd": phase_entry(med["fwd"], w, step.bytes_fwd(), peak),
+                 "bwd": phase_entry(med["bwd"], w, step.bytes_bwd(), peak),
+                 "fwd_bwd": phase_entry(fb, w, step.bytes_fwd() + step.bytes_bwd(), peak),
+                 "launches_per_iteration": launches,
+                 "packed_codes": bool(case["pack"])}
+        if case["standalone_pack"]:
+            rows = sum(m.rows for m in case["mats"])
+            nb = w * 4 + w * pq.pq_code_bits(q) // 8 + rows * 4
+            entry["pack_standalone"] = phase_entry(med["pack_standalone"], w, nb, peak)
+        if planted:
+            entry["planted"] = planted
+        del step, fns, b
+        torch.cuda.empty_cache()
+        if oracle_seconds > 0:
+            sample = oracle_sample(case["mats"], q, oracle_seconds, seed=case["seed"],
+                                   dist=case["dist"], lsq_rule=rule, plant=case["plant"],
+                                   pack=case["pack"])
+            n, dt = time_oracle(sample, q=q, pack=case["pack"])
+            whole = all(wm.shape[0] == m.rows for m, wm, _, _ in sample)
+            entry["oracle"] = {"Gweights_s": n / dt / 1e9, "cores": 1, "seconds": dt,
+                               "weights": n,
+                               "sample": ("the whole workload" if whole else
+                                          "full-width rows of every matrix"),
+                               "gpu_speedup_fwd_bwd": entry["fwd_bwd"]["Gweights_s"]
+                               / (n / dt / 1e9)}
+        out[name] = entry
+    return out
+
+
+def run_per_config(args, peak, device, oracle_seconds=1.5):
+    flush = L2Flush(device)
+    res = {}
+    for case in per_config_cases():
+        res[case["key"]] = measure_case(case, args.config_steps, args.warmup, peak, device,
+                                        flush, oracle_seconds)
+    del flush
+    return res
+
+
+# ---------------------------------------------------------------- next rows
+def packed_views(step, packed_all):
+    """Per-matrix views of one flat packed-code buffer (2-bit codes)."""
+    views, o = [], 0
+    for b in step.bufs:
+        n = b.m.numel // 4
+        views.append(packed_all[o:o + n].view(b.m.rows, b.m.cols // 4))
+        o += (n + 255) // 256 * 256
+    return views
+
+
+def packed_bytes(step):
+    return sum((b.m.numel // 4 + 255) // 256 * 256 for b in step.bufs)
+
+
+def measure_dequant(step, packed, out, steps, warmup, peak):
+    """Packed codes + alpha -> bf16 for every matrix of the step, one batched
+    call (2.25 B per weight + 4 B per row)."""
+    from bit_quantization_aware_b200 import pq
+    descs = [dict(rows=b.m.rows, cols=b.m.cols, alpha=b.alpha, packed=pk, wq=o)
+             for b, pk, o in zip(step.bufs, packed, out)]
+    mats = pq.matrix_array(descs)
+    ms, launches = time_eager(lambda: pq.pq_dequant_codes_batch(step.q, mats), steps, warmup)
+    nbytes = sum(b.m.numel * 2 + b.m.numel // 4 + b.m.rows * 4 for b in step.bufs)
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "Gweights_s": step.weights / (ms * 1e-3) / 1e9,
+            "launches_per_call": launches,
+            "roofline": {"bound": "hbm", "kernel": "pq::dequant_units_kernel<SEQ2, vector layout>",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "algorithmic_bytes": nbytes}}
+
+
+def measure_bwd_adamw(step, steps, warmup, peak):
+    """The backward fused with one AdamW step over every matrix (one batched
+    launch; 26 B per weight + 24 B per row), then, for context, the unfused
+    sequence: the batched backward writing dW, then torch's fused AdamW. The
+    step's weights and scales are updated in place."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    m_w = torch.zeros_like(step.w_all)
+    v_w = torch.zeros_like(step.w_all)
+    m_a = torch.zeros_like(step.alpha_all)
+    v_a = torch.zeros_like(step.alpha_all)
+    descs = []
+    for b in step.bufs:
+        o = b.w.data_ptr() - step.w_all.data_ptr()
+        o //= 4
+        ro = (b.alpha.data_ptr() - step.alpha_all.data_ptr()) // 4
+        n = b.m.numel
+        descs.append(dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
+                          m_w=m_w[o:o + n], v_w=v_w[o:o + n], m_alpha=m_a[ro:ro + b.m.rows],
+                          v_alpha=v_a[ro:ro + b.m.rows], grad_scale=b.grad_scale))
+    arr = pq.adamw_matrix_array(descs)
+    t = [0]
+
+    def fused():
+        t[0] += 1
+        pq.pq_fakequant_bwd_adamw(step.q, arr, pq.adamw(t[0], 2e-5), pq.adamw(t[0], 2e-5))
+
+    ms, launches = time_eager(fused, steps, warmup)
+    del arr, descs, m_w, v_w, m_a, v_a
+    torch.cuda.empty_cache()
+    # context: backward (dW to memory) + torch fused AdamW on the same data
+    params = []
+    for b in step.bufs:
+        prm = torch.nn.Parameter(b.w, requires_grad=True)
+        prm.grad = b.dw
+        params.append(prm)
+    opt = torch.optim.AdamW(params, lr=2e-5, weight_decay=0.0, fused=True)
+
+    def unfused():
+        step.bwd_all()
+        opt.step()
+
+    ms_unfused, _ = time_eager(unfused, steps, warmup)
+    del opt, params
+    torch.cuda.empty_cache()
+    rows = sum(b.m.rows for b in step.bufs)
+    nbytes = 26 * step.weights + 24 * rows
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "Gweights_s": step.weights / (ms * 1e-3) / 1e9,
+            "launches_per_call": launches,
+            "roofline": {"bound": "hbm", "kernel": "pq::bwd_adamw_units_kernel<SEQ2, vector layout>",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "algorithmic_bytes": nbytes},
+            "unfused": {"ms": ms_unfused,
+                        "what": "pq_fakequant_bwd_batch (dW to memory) + "
+                                "torch.optim.AdamW(fused=True)",
+                        "speedup_of_fused": ms_unfused / ms}}
+
+
+def wq_gemm_kernel_name(m, gsize, max_k):
+    """The kernel a grouped launch of ``gsize`` matrices with ``m`` activation
+    rows runs: one row times a lone matrix (k <= 32768) takes the CUDA-core
+    kernel, 1..16 rows otherwise the integer tensor-core mode (after its
+    activation digit-plane pre-pass), more rows the bf16 tensor-core mode."""
+    if m == 1 and gsize == 1 and max_k <= 32768:
+        return "pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)", False
+    if m <= 16:
+        return ("pqg::wq_gemm_kernel<NT, MAXP, true> (tcgen05.mma kind::i8, TMEM accumulator)"
+                " after pqg::xplanes_kernel"), True
+    return "pqg::wq_gemm_kernel<NT, MAXP, false> (tcgen05.mma kind::f16, TMEM accumulator)", False
+
+
+def measure_wq_gemm(bufs, packed, q, m, steps, warmup, device, with_single=False):
+    """Weight-only 2-bit matmul Y = X (alpha * levels)^T for every matrix in
+    ``bufs`` (grouped launches of up to 64 matrices, captured in one CUDA
+    graph), against cuBLAS (torch.matmul) on the dense bf16 dequantized
+    weights, also graph-captured."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    ks = sorted({b.m.cols for b in bufs})
+    ns = sorted({b.m.rows for b in bufs})
+    gen = torch.Generator(device=device)
+    gen.manual_seed(11)
+    xs = {k: torch.randn((m, k), generator=gen, device=device).to(torch.bfloat16) for k in ks}
+    ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in ns}
+    ys_ref = {n: torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in ns}
+    ngroups = (len(bufs) + 63) // 64
+    gsize = (len(bufs) + ngroups - 1) // ngroups
+    groups = [pq.gemm_problem_array([dict(x=xs[b.m.cols], packed=pk, alpha=b.alpha,
+                                          y=ys[b.m.rows])
+                                     for b, pk in zip(bufs[i:i + gsize], packed[i:i + gsize])])
+              for i in range(0, len(bufs), gsize)]
+    gneed = max(pq.pq_wq_gemm_batch_workspace_bytes(q, m, g) for g in groups)
+    gws = torch.empty(max(gneed, 256), dtype=torch.uint8, device=device)
+
+    def ours():
+        for g in groups:
+            pq.pq_wq_gemm_batch(q, m, g, gws)
+
+    def dense():
+        for b in bufs:
+            torch.matmul(xs[b.m.cols], b.wq.t(), out=ys_ref[b.m.rows])
+
+    ms, g_ours, launches = time_graph(ours, steps, warmup)
+    res = {}
+    if with_single:
+        need = max(pq.pq_wq_gemm_workspace_bytes(q, m, b.m.rows, b.m.cols) for b in bufs)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+
+        def ours_single():
+            for b, pk in zip(bufs, packed):
+                pq.pq_wq_gemm(q, xs[b.m.cols], pk, b.alpha, ys[b.m.rows], ws)
+        ms_single, g_single, l_single = time_graph(ours_single, steps, warmup)
+        res["per_matrix_launches"] = {"ms": ms_single, "launches_per_step": l_single,
+                                      "what": "pq_wq_gemm once per matrix, CUDA graph"}
+        del g_single
+    ms_dense, g_dense, _ = time_graph(dense, steps, warmup)
+    status = pq.pq_device_status()
+    if status != 0:
+        raise RuntimeError(f"weight-only matmul: a bounded device wait gave up ({status})")
+    # the last matrix of the set, both ways (same weights, fp32 sums)
+    b = bufs[-1]
+    yo, yr = ys[b.m.rows].float(), ys_ref[b.m.rows].float()
+    rel = float((yo - yr).abs().max() / yr.abs().max().clamp_min(1e-30))
+    del g_ours, g_dense
+    weights = sum(b.m.numel for b in bufs)
+    nbytes = sum(b.m.numel // 4 + b.m.rows * 4 + m * b.m.cols * 2 + m * b.m.rows * 2
+                 for b in bufs)
+    flops = 2 * m * weights
+    hbm, hbm_kind = measured_peaks()
+    tflops, tf_kind = measured_tensor_peak()
+    if nbytes / (hbm * 1e9) >= flops / (tflops * 1e12):
+        roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s", "peak_source": f"{hbm_kind} hbm_gbs",
+                "algorithmic_bytes": nbytes}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tflops,
+                "unit": "TFLOP/s", "peak_source": f"{tf_kind} bf16_tflops (burst)",
+                "algorithmic_flops": flops}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"], integer_mode = wq_gemm_kernel_name(m, gsize, max(ks))
+    res.update({"m": m, "ms": ms, "Gweights_s": weights / (ms * 1e-3) / 1e9,
+                "tflops": flops / (ms * 1e-3) / 1e12, "launches_per_step": launches,
+                "grouped_launches": len(groups), "matrices_per_launch": gsize,
+                "dtype": ("s8 digit planes of bf16 activations x u8 2-bit code fields, "
+                          "s32 accumulate" if integer_mode else
+                          "bf16 x 2-bit codes, f32 accumulate"),
+                "roofline": roof,
+                "cublas_bf16_dense": {"ms": ms_dense, "speedup_of_ours": ms_dense / ms,
+                                      "what": "torch.matmul(x, W_bf16.t()) per matrix, CUDA graph",
+                                      "max_rel_diff_last_matrix": rel}})
+    return res
+
+
+def sharded_bytes(weights: int, world: int) -> dict:
+    """Algorithmic bytes of one row-sharded step over `weights` weights (all
+    ranks together; scales and d(alpha) are per-row and negligible): pack
+    reads each owned fp32 weight and writes 0.25 B of codes; every rank's
+    gather + dequantization reads all codes and writes all bf16 weights;
+    the reduce step reads `world` bf16 gradient rows per owned weight plus
+    w, m, v and writes w, m, v."""
+    return {"pack": int(4.25 * weights),
+            "gather_dequant": int(world * 2.25 * weights),
+            "reduce_bwd_adamw": int((2 * world + 24) * weights)}
+
+
+def measure_sharded(world, layers, steps, warmup, peak, device):
+    """The row-sharded owner-computes step (pack own rows; gather + dequantize
+    everyone's codes; reduce the replicas' gradients + backward + AdamW on
+    own rows) for ``world`` ranks emulated as buffer sets on one GPU, over
+    the first ``layers`` layers of the Llama-3-8B-shaped set. Peer buffers
+    are local device memory here, so this measures the kernels' HBM
+    efficiency, not NVLink. Each phase runs for every rank in turn, timed by
+    CUDA events."""
+    import torch
+
+    from bit_quantization_aware_b200 import inputs as I
+    from bit_quantization_aware_b200 import pq
+    from bit_quantization_aware_b200.sharded import LocalPeers, ShardedQuantStep
+    q = pq.PQ_SEQ2
+    mats = I.llama3_8b_set()[: 7 * layers]
+    peers = LocalPeers(world)
+    ranks = [ShardedQuantStep(mats, q, k, world, peers, device=device) for k in range(world)]
+    for i, m in enumerate(mats):
+        w = I.normal_weights(m.rows, m.cols, seed=3, stream=i, device=device)
+        a = I.alpha_init(w, q)
+        for r in ranks:
+            r.load_full(i, w, a)
+        del w, a
+    for k, r in enumerate(ranks):
+        for i, m in enumerate(mats):
+            r.g(i).copy_(I.grad_bf16(m.rows, m.cols, seed=4 + k, stream=64 + i, device=device))
+    torch.cuda.synchronize()
+    t = [0]
+
+    def phase(fn):
+        for r in ranks:
+            fn(r)
+
+    def step_fns():
+        t[0] += 1
+        hw, ha = pq.adamw(t[0], 2e-5), pq.adamw(t[0], 1e-4)
+        return [("pack", lambda r: r.pack_shards()),
+                ("gather_dequant", lambda r: r.gather_dequant()),
+                ("reduce_bwd_adamw", lambda r: r.reduce_step(hw, ha))]
+
+    for _ in range(max(warmup, 1)):
+        for _, fn in step_fns():
+            phase(fn)
+    torch.cuda.synchronize()
+    names = ["pack", "gather_dequant", "reduce_bwd_adamw"]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * steps)]
+    l0 = pq.pq_launch_count()
+    for s_ in range(steps):
+        for j, (_, fn) in enumerate(step_fns()):
+            ev[4 * s_ + j].record()
+            phase(fn)
+        ev[4 * s_ + 3].record()
+    torch.cuda.synchronize()
+    launches = pq.pq_launch_count() - l0
+    ms = {n: sum(ev[4 * s_ + j].elapsed_time(ev[4 * s_ + j + 1]) for s_ in range(steps)) / steps
+          for j, n in enumerate(names)}
+    total = sum(ms.values())
+    weights = I.total_weights(mats)
+    nbytes = sharded_bytes(weights, world)
+    phases = {n: {"ms": ms[n], "algorithmic_bytes": nbytes[n],
+                  "GB_s": nbytes[n] / (ms[n] * 1e-3) / 1e9,
+                  "frac_of_peak": nbytes[n] / (ms[n] * 1e-3) / 1e9 / peak} for n in names}
+    allb = sum(nbytes.values())
+    del ranks, peers
+    torch.cuda.empty_cache()
+    return {"ms": total, "Gweights_s": weights / (total * 1e-3) / 1e9, "weights": weights,
+            "world": world, "layers": layers, "launches_per_step": launches / steps,
+            "workload": f"llama3_8b_first{layers}layers_seq2_sharded_world{world}_emulated",
+            "note": "all ranks' work on one GPU in turn; peer reads are local HBM reads",
+            "roofline": {"bound": "hbm", "kernel": "pack, dequant and reduce_bwd_adamw units kernels",
+                         "achieved": allb / (total * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": allb / (total * 1e-3) / 1e9 / peak,
+                         "algorithmic_bytes": allb},
+            "phases": phases, "launches_total": launches}
+
+
+def run_next_rows(step, args, peak, device):
+    """The rows built on the quantizer, on the headline's Llama-3-8B-shaped
+    buffers: packed export -> dequantization -> weight-only matmul at 1, 16
+    and 128 activation rows, then the backward fused with AdamW (which
+    updates the weights in place, so it runs last)."""
+    import torch
+
+    from bit_quantization_aware_b200 import pq
+    res = {}
+    packed_all = torch.empty(packed_bytes(step), dtype=torch.uint8, device=device)
+    packed = packed_views(step, packed_all)
+    # one forward that writes bf16 weights and packed codes
+    pq.pq_fakequant_fwd_batch(step.q, pq.matrix_array([
+        dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, wq=b.wq, packed=pk)
+        for b, pk in zip(step.bufs, packed)]))
+    torch.cuda.synchronize()
+    deq_all = torch.empty_like(step.wq_all)
+    deq_out = [deq_all[(b.wq.data_ptr() - step.wq_all.data_ptr()) // 2:][: b.m.numel]
+               .view(b.m.rows, b.m.cols) for b in step.bufs]
+    res["dequant"] = measure_dequant(step, packed, deq_out, args.extra_steps, args.warmup, peak)
+    same = all(torch.equal(o.view(torch.int16), b.wq.view(torch.int16))
+               for o, b in zip(deq_out, step.bufs))
+    res["dequant"]["equals_forward_bf16"] = bool(same)
+    res["wq_gemm"] = {}
+    for m in (1, 16, 128):
+        res["wq_gemm"][f"m{m}"] = measure_wq_gemm(step.bufs, packed, step.q, m,
+                                                   2 * args.extra_steps, args.warmup, device)
+    del packed, packed_all, deq_out, deq_all
+    torch.cuda.empty_cache()
+    res["bwd_adamw"] = measure_bwd_adamw(step, args.extra_steps, args.warmup, peak)
+    return res
+
+
 # --------------------------------------------------------------------- ours
 def run_ours(args):
     import torch
@@ -296,6 +875,7 @@ def run_ours(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
+    device = f"cuda:{local}"
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=600),
@@ -303,7 +883,7 @@ def run_ours(args):
     pq.lib()  # fail loudly if the CUDA library is missing
 
     mats = I.llama3_8b_set()
-    step = QuantStep(mats, pq.PQ_SEQ2, device=f"cuda:{local}")
+    step = QuantStep(mats, pq.PQ_SEQ2, device=device)
     step.generate(seed=3 + rank)
     stream = torch.cuda.current_stream()
     weights = step.weights
@@ -322,19 +902,13 @@ def run_ours(args):
     bwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     fwd_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    gpu_index = local
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        try:
-            gpu_index = int(vis.split(",")[local])
-        except ValueError:
-            pass
-    sampler = ClockSampler(gpu_index)
+    sampler = ClockSampler(physical_gpu_index(local))
     sampler.start()
     time.sleep(0.3)
 
     barrier()
     torch.cuda.synchronize()
+    l0 = pq.pq_launch_count()
     ev_start.record(stream)
     for k in range(args.steps):
         fwd_ev[k].record(stream)
@@ -344,13 +918,14 @@ def run_ours(args):
         bwd_ev[k][1].record(stream)
     ev_end.record(stream)
     torch.cuda.synchronize()
+    launches = pq.pq_launch_count() - l0
     barrier()
     clocks = sampler.stop()
 
     ms_total = ev_start.elapsed_time(ev_end)
     bwd_ms = sum(a.elapsed_time(b) for a, b in bwd_ev)
     fwd_ms = sum(a.elapsed_time(b[0]) for a, b in zip(fwd_ev, bwd_ev))
-    ms_total, bwd_ms, fwd_ms = reduce_max([ms_total, bwd_ms, fwd_ms], f"cuda:{local}", world)
+    ms_total, bwd_ms, fwd_ms = reduce_max([ms_total, bwd_ms, fwd_ms], device, world)
     ms_step = ms_total / args.steps
     value = step_throughput(weights, world, ms_step)
 
@@ -392,7 +967,27 @@ def run_ours(args):
         sample = sample_rows_for_oracle(args.cpu_seconds)
         n, dt = time_oracle(sample)
         cpu = {"value": n / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": describe_sample(sample), "seconds": dt}
+               "sample": describe_sample(sample), "seconds": dt,
+               "host_cores": os.cpu_count()}
+
+    per_config = nxt = extras_clocks = None
+    if world == 1 and not args.no_extras:
+        # after the headline's timed region: the NEXT rows on its buffers,
+        # then the other workloads and the sharded step on fresh buffers
+        xs = ClockSampler(physical_gpu_index(local))
+        xs.start()
+        nxt = run_next_rows(step, args, peak, device)
+        del step
+        torch.cuda.empty_cache()
+        nxt["sharded"] = measure_sharded(2, 8, args.extra_steps, args.warmup, peak, device)
+        per_config = run_per_config(args, peak, device)
+        extras_clocks = xs.stop()
+        per_config["4_llama3_8b_set"] = {
+            "see": "the line's phases (the headline workload)",
+            "oracle": None if cpu is None else
+            {"Gweights_s": cpu["value"], "cores": 1, "seconds": cpu["seconds"],
+             "sample": cpu["sample"],
+             "gpu_speedup_fwd_bwd": phases["fwd_bwd"]["Gweights_s"] / cpu["value"]}}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -401,9 +996,13 @@ def run_ours(args):
                 "dtype": "f32", "data": "synthetic (seeded N(0,0.02) weights, "
                 "bf16 N(0,1e-3) upstream grads, alpha = max|w_row|)",
                 "config": config_dict(world, weights),
-                "gpu_launches": step.launches_per_step * args.steps,
+                "gpu_launches": launches,
                 "roofline": roofline, "phases": phases, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks}
+        if per_config is not None:
+            line["per_config"] = per_config
+            line["next"] = nxt
+            line["extras_clocks"] = extras_clocks
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -518,58 +1117,42 @@ def run_e2e(step, args, local, world):
                    "Wq, dW, dalpha -> pinned host; three streams, layer-pipelined"}
 
 
-def run_dequant(args):
-    """Packed 2-bit codes + alpha -> bf16 weights for every matrix of the
-    Llama-3-8B-shaped set (the export path's consumer), one batched call,
-    1 GPU. Prints one JSON line with its own roofline (2.25 B/weight)."""
+# ------------------------------------------------------- single-row modes
+def _llama_step_with_codes(device):
+    """The Llama-3-8B-shaped set with bf16 weights and packed codes from
+    one forward (inputs of the dequantization and matmul modes)."""
     import torch
 
     from bit_quantization_aware_b200 import inputs as I
     from bit_quantization_aware_b200 import pq
     from bit_quantization_aware_b200.step import QuantStep
-
-    torch.cuda.set_device(0)
-    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device="cuda:0", pack=True)
+    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device=device, pack=True)
     step.generate(seed=3)
     step.fwd_all()
     torch.cuda.synchronize()
-    out = torch.empty_like(step.wq_all)
-    descs, o = [], 0
-    for b in step.bufs:
-        n = b.m.numel
-        descs.append(dict(rows=b.m.rows, cols=b.m.cols, alpha=b.alpha, packed=b.packed,
-                          wq=out[o:o + n]))
-        o += (n + 63) // 64 * 64
-    mats = pq.matrix_array(descs)
+    return step
 
-    def go():
-        pq.pq_dequant_codes_batch(step.q, mats)
 
-    for _ in range(max(args.warmup, 1)):
-        go()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        go()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    bytes_step = sum(b.m.numel * 2 + b.m.numel // 4 + b.m.rows * 4 for b in step.bufs)
+def run_dequant(args):
+    """Packed 2-bit codes + alpha -> bf16 weights for every matrix of the
+    Llama-3-8B-shaped set (the export path's consumer), one batched call,
+    1 GPU. Prints one JSON line with its own roofline (2.25 B/weight)."""
+    import torch
+    torch.cuda.set_device(0)
+    step = _llama_step_with_codes("cuda:0")
+    out = [torch.empty_like(b.wq) for b in step.bufs]
     peak, kind = measured_peaks()
-    achieved = bytes_step / (ms * 1e-3) / 1e9
+    r = measure_dequant(step, [b.packed for b in step.bufs], out, args.steps, args.warmup, peak)
+    r["roofline"].update(peak_source=f"{kind} hbm_gbs", traffic=None)
     print(json.dumps({
         "metric": "packed-code dequantization Gweights/s", "op": "dequant",
-        "value": step.weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "value": r["Gweights_s"], "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"],
         "higher_is_better": True, "dtype": "u8->bf16", "data": "synthetic",
         "config": {"workload": "llama3_8b_linear_set_seq2_dequant",
-                   "weights": step.weights, "launches_per_step": 1},
-        "roofline": {"bound": "hbm", "kernel": "pq::dequant_units_kernel<SEQ2, vector layout>",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "peak_source": f"{kind} hbm_gbs",
-                     "algorithmic_bytes_per_step": bytes_step}}), flush=True)
+                   "weights": step.weights, "launches_per_step": r["launches_per_call"]},
+        "gpu_launches": r["launches_per_call"] * args.steps,
+        "roofline": r["roofline"]}), flush=True)
     return 0
 
 
@@ -583,330 +1166,82 @@ def run_bwd_adamw(args):
     from bit_quantization_aware_b200 import inputs as I
     from bit_quantization_aware_b200 import pq
     from bit_quantization_aware_b200.step import QuantStep
-
     torch.cuda.set_device(0)
-    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device="cuda:0", alloc_outputs=False)
+    step = QuantStep(I.llama3_8b_set(), pq.PQ_SEQ2, device="cuda:0")
     step.generate(seed=3)
-    m_w = torch.zeros_like(step.w_all)
-    v_w = torch.zeros_like(step.w_all)
-    m_a = torch.zeros_like(step.alpha_all)
-    v_a = torch.zeros_like(step.alpha_all)
-    descs, o, ro = [], 0, 0
-    for b in step.bufs:
-        n = b.m.numel
-        descs.append(dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
-                          m_w=m_w[o:o + n], v_w=v_w[o:o + n], m_alpha=m_a[ro:ro + b.m.rows],
-                          v_alpha=v_a[ro:ro + b.m.rows], grad_scale=b.grad_scale))
-        o += (n + 63) // 64 * 64
-        ro += (b.m.rows + 63) // 64 * 64
-    arr = pq.adamw_matrix_array(descs)
-    t = [0]
-
-    def fused():
-        t[0] += 1
-        pq.pq_fakequant_bwd_adamw(step.q, arr, pq.adamw(t[0], 2e-5), pq.adamw(t[0], 2e-5))
-
-    for _ in range(max(args.warmup, 1)):
-        fused()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        fused()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-
-    # context: backward (dW to memory) + torch fused AdamW on the same data;
-    # our moment buffers make room for torch's
-    del arr, descs, m_w, v_w
-    torch.cuda.empty_cache()
-    dw_all = torch.empty_like(step.w_all)
-    bwd_descs, o = [], 0
-    params = []
-    for b in step.bufs:
-        n = b.m.numel
-        dw = dw_all[o:o + n].view(b.m.rows, b.m.cols)
-        bwd_descs.append(dict(rows=b.m.rows, cols=b.m.cols, w=b.w, alpha=b.alpha, g=b.g,
-                              dw=dw, dalpha=b.dalpha, grad_scale=b.grad_scale))
-        prm = torch.nn.Parameter(b.w, requires_grad=True)
-        prm.grad = dw
-        params.append(prm)
-        o += (n + 63) // 64 * 64
-    bwd_arr = pq.matrix_array(bwd_descs)
-    opt = torch.optim.AdamW(params, lr=2e-5, weight_decay=0.0, fused=True)
-
-    def unfused():
-        pq.pq_fakequant_bwd_batch(step.q, bwd_arr)
-        opt.step()
-
-    for _ in range(max(args.warmup, 1)):
-        unfused()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(args.steps):
-        unfused()
-    e1.record()
-    torch.cuda.synchronize()
-    ms_unfused = e0.elapsed_time(e1) / args.steps
-
-    rows = sum(b.m.rows for b in step.bufs)
-    bytes_step = 26 * step.weights + 24 * rows
     peak, kind = measured_peaks()
-    achieved = bytes_step / (ms * 1e-3) / 1e9
+    r = measure_bwd_adamw(step, args.steps, args.warmup, peak)
+    r["roofline"].update(peak_source=f"{kind} hbm_gbs", traffic=None)
     print(json.dumps({
         "metric": "backward + AdamW step Gweights/s", "op": "bwd_adamw",
-        "value": step.weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "value": r["Gweights_s"], "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"],
         "higher_is_better": True, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "llama3_8b_linear_set_seq2_bwd_adamw", "weights": step.weights,
-                   "launches_per_step": 1},
-        "roofline": {"bound": "hbm", "kernel": "pq::bwd_adamw_units_kernel<SEQ2, vector layout>",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_source": f"{kind} hbm_gbs",
-                     "algorithmic_bytes_per_step": bytes_step},
-        "unfused": {"ms_per_step": ms_unfused,
-                    "what": "pq_fakequant_bwd_batch (dW to memory) + torch.optim.AdamW(fused=True)",
-                    "speedup_of_fused": ms_unfused / ms}}), flush=True)
+                   "launches_per_step": r["launches_per_call"]},
+        "gpu_launches": r["launches_per_call"] * args.steps,
+        "roofline": r["roofline"], "unfused": r["unfused"]}), flush=True)
     return 0
 
 
 def run_wq_gemm(args):
-    """Weight-only 2-bit matmul Y = X (alpha * levels)^T for every matrix of
-    the Llama-3-8B-shaped set (224 matrices in grouped launches of up to 64,
-    captured in one CUDA graph; the 1.75 GB of codes are far larger than L2,
-    so every launch reads its codes from HBM), 1 GPU, X of --m rows. Beside
-    it, for context, the same with one launch per matrix, and cuBLAS
-    (torch.matmul) on the dense bf16 dequantized weights, also
-    graph-captured. Prints one JSON line."""
+    """Weight-only 2-bit matmul for every matrix of the Llama-3-8B-shaped set
+    (or four 16384x16384 weights, so that every replay reads its codes from
+    HBM), X of --m rows, 1 GPU; beside it one launch per matrix and cuBLAS
+    bf16 on the dequantized weights. Prints one JSON line."""
     import torch
 
     from bit_quantization_aware_b200 import inputs as I
     from bit_quantization_aware_b200 import pq
     from bit_quantization_aware_b200.step import QuantStep
-
     torch.cuda.set_device(0)
-    dev = "cuda:0"
-    m = args.m
-    q = pq.PQ_SEQ2
     if args.shape == "16384":
-        # one 16384^2 weight, several copies so that every replay reads HBM
-        # (codes 64 MiB and bf16 weights 512 MiB per copy; L2 is 126 MB)
         mats = [I.Matrix(f"w{i}", 16384, 16384, i, 0) for i in range(4)]
-    else:
-        mats = I.llama3_8b_set()
-    step = QuantStep(mats, q, device=dev, pack=True)
-    step.generate(seed=3)
-    step.fwd_all()
-    torch.cuda.synchronize()
-    ks = sorted({b.m.cols for b in step.bufs})
-    ns = sorted({b.m.rows for b in step.bufs})
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(11)
-    xs = {k: torch.randn((m, k), generator=gen, device=dev).to(torch.bfloat16) for k in ks}
-    ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in ns}
-    ys_ref = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in ns}
-    need = max(pq.pq_wq_gemm_workspace_bytes(q, m, b.m.rows, b.m.cols) for b in step.bufs)
-    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    # grouped launches: up to 64 matrices each, in equal groups
-    ngroups = (len(step.bufs) + 63) // 64
-    gsize = (len(step.bufs) + ngroups - 1) // ngroups
-    groups = [pq.gemm_problem_array([dict(x=xs[b.m.cols], packed=b.packed, alpha=b.alpha,
-                                          y=ys[b.m.rows]) for b in step.bufs[i:i + gsize]])
-              for i in range(0, len(step.bufs), gsize)]
-    gneed = max(pq.pq_wq_gemm_batch_workspace_bytes(q, m, g) for g in groups)
-    gws = torch.empty(max(gneed, 256), dtype=torch.uint8, device=dev)
-
-    def ours_single():
-        for b in step.bufs:
-            pq.pq_wq_gemm(q, xs[b.m.cols], b.packed, b.alpha, ys[b.m.rows], ws)
-
-    def ours():
-        for g in groups:
-            pq.pq_wq_gemm_batch(q, m, g, gws)
-
-    def dense():
-        for b in step.bufs:
-            torch.matmul(xs[b.m.cols], b.wq.t(), out=ys_ref[b.m.rows])
-
-    def timed(fn):
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            for _ in range(2):
-                fn()
-        torch.cuda.current_stream().wait_stream(side)
+        step = QuantStep(mats, pq.PQ_SEQ2, device="cuda:0", pack=True)
+        step.generate(seed=3)
+        step.fwd_all()
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        for _ in range(max(args.warmup, 3)):
-            g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / args.steps, g
-
-    ms, g_ours = timed(ours)
-    ms_single, g_single = timed(ours_single)
-    ms_dense, g_dense = timed(dense)
-    assert pq.pq_device_status() == 0
-    # the last matrix of the set, both ways (same weights, fp32 sums)
-    b = step.bufs[-1]
-    yo, yr = ys[b.m.rows].float(), ys_ref[b.m.rows].float()
-    rel = float((yo - yr).abs().max() / yr.abs().max().clamp_min(1e-30))
-    del g_ours, g_single, g_dense
-
-    weights = step.weights
-    bytes_step = sum(b.m.numel // 4 + b.m.rows * 4 + m * b.m.cols * 2 + m * b.m.rows * 2
-                     for b in step.bufs)
-    flops_step = 2 * m * weights
-    hbm, hbm_kind = measured_peaks()
-    tflops, tf_kind = measured_tensor_peak()
-    t_hbm = bytes_step / (hbm * 1e9)
-    t_tc = flops_step / (tflops * 1e12)
-    if t_hbm >= t_tc:
-        roof = {"bound": "hbm", "achieved": bytes_step / (ms * 1e-3) / 1e9, "peak": hbm,
-                "unit": "GB/s", "peak_source": f"{hbm_kind} hbm_gbs",
-                "algorithmic_bytes_per_step": bytes_step}
+        workload = f"4x16384x16384_seq2_wq_gemm_m{args.m}"
     else:
-        roof = {"bound": "tensor", "achieved": flops_step / (ms * 1e-3) / 1e12, "peak": tflops,
-                "unit": "TFLOP/s", "peak_source": f"{tf_kind} bf16_tflops (burst)",
-                "algorithmic_flops_per_step": flops_step}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
-    # the kernel of the grouped launches: one activation row times a lone
-    # matrix (k <= 32768) takes the CUDA-core kernel, 1..16 rows otherwise the
-    # integer tensor-core mode (after its activation digit-plane pre-pass),
-    # more rows the bf16 tensor-core mode
-    integer_mode = m <= 16 and not (m == 1 and gsize == 1 and max(ks) <= 32768)
-    if m == 1 and gsize == 1 and max(ks) <= 32768:
-        roof["kernel"] = "pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)"
-    elif integer_mode:
-        roof["kernel"] = ("pqg::wq_gemm_kernel<NT, MAXP, true> (tcgen05.mma kind::i8, TMEM accumulator)"
-                          " after pqg::xplanes_kernel")
-    else:
-        roof["kernel"] = "pqg::wq_gemm_kernel<NT, MAXP, false> (tcgen05.mma kind::f16, TMEM accumulator)"
+        step = _llama_step_with_codes("cuda:0")
+        workload = f"llama3_8b_linear_set_seq2_wq_gemm_m{args.m}"
+    r = measure_wq_gemm(step.bufs, [b.packed for b in step.bufs], step.q, args.m, args.steps,
+                        args.warmup, "cuda:0", with_single=True)
+    r["roofline"]["traffic"] = None
     print(json.dumps({
         "metric": "weight-only 2-bit matmul Gweights/s", "op": "wq_gemm",
-        "value": weights / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True,
-        "dtype": ("s8 digit planes of bf16 activations x u8 2-bit code fields, s32 accumulate"
-                  if integer_mode else "bf16 x 2-bit codes, f32 accumulate"),
-        "data": "synthetic",
-        "config": {"workload": (f"llama3_8b_linear_set_seq2_wq_gemm_m{m}" if args.shape != "16384"
-                                else f"4x16384x16384_seq2_wq_gemm_m{m}"), "m": m,
-                   "weights": weights, "launches_per_step": len(groups),
-                   "kernels_per_step": len(groups) * (2 if integer_mode else 1),
-                   "matrices_per_launch": gsize,
+        "value": r["Gweights_s"], "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"],
+        "higher_is_better": True, "dtype": r["dtype"], "data": "synthetic",
+        "config": {"workload": workload, "m": args.m, "weights": step.weights,
+                   "launches_per_step": r["launches_per_step"],
+                   "matrices_per_launch": r["matrices_per_launch"],
                    "l2": f"codes {step.weights / 4e9:.2f} GB per step, larger than L2"},
-        "roofline": roof,
-        "gpu_launches": len(groups) * (2 if integer_mode else 1) * args.steps,
-        "tflops": flops_step / (ms * 1e-3) / 1e12,
-        "per_matrix_launches": {"ms_per_step": ms_single, "launches_per_step": len(step.bufs),
-                                "what": "pq_wq_gemm once per matrix, CUDA graph"},
-        "cublas_bf16_dense": {"ms_per_step": ms_dense, "speedup_of_ours": ms_dense / ms,
-                              "what": "torch.matmul(x, W_bf16.t()) per matrix, CUDA graph",
-                              "max_rel_diff_last_matrix": rel}}), flush=True)
+        "roofline": r["roofline"],
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "tflops": r["tflops"],
+        "per_matrix_launches": r["per_matrix_launches"],
+        "cublas_bf16_dense": r["cublas_bf16_dense"]}), flush=True)
     return 0
 
 
-def sharded_bytes(weights: int, world: int) -> dict:
-    """Algorithmic bytes of one row-sharded step over `weights` weights (all
-    ranks together; scales and d(alpha) are per-row and negligible): pack
-    reads each owned fp32 weight and writes 0.25 B of codes; every rank's
-    gather + dequantization reads all codes and writes all bf16 weights;
-    the reduce step reads `world` bf16 gradient rows per owned weight plus
-    w, m, v and writes w, m, v."""
-    return {"pack": int(4.25 * weights),
-            "gather_dequant": int(world * 2.25 * weights),
-            "reduce_bwd_adamw": int((2 * world + 24) * weights)}
-
-
 def run_sharded(args):
-    """The row-sharded owner-computes step (pack own rows; gather + dequantize
-    everyone's codes; reduce the replicas' gradients + backward + AdamW on
-    own rows) for `--world` ranks emulated as buffer sets on one GPU, over
-    the first `--layers` layers of the Llama-3-8B-shaped set. Peer buffers
-    are local device memory here, so this measures the kernels' HBM
-    efficiency, not NVLink. Each phase runs for every rank in turn, timed by
-    CUDA events. Prints one JSON line."""
+    """The row-sharded step for ``--world`` ranks emulated on one GPU over
+    the first ``--layers`` layers; prints one JSON line."""
     import torch
-
-    from bit_quantization_aware_b200 import inputs as I
-    from bit_quantization_aware_b200 import pq
-    from bit_quantization_aware_b200.sharded import LocalPeers, ShardedQuantStep
-
     torch.cuda.set_device(0)
-    q, world = pq.PQ_SEQ2, args.world
-    mats = I.llama3_8b_set()[: 7 * args.layers]
-    peers = LocalPeers(world)
-    ranks = [ShardedQuantStep(mats, q, k, world, peers, device="cuda:0") for k in range(world)]
-    for i, m in enumerate(mats):
-        w = I.normal_weights(m.rows, m.cols, seed=3, stream=i, device="cuda:0")
-        a = I.alpha_init(w, q)
-        for r in ranks:
-            r.load_full(i, w, a)
-        del w, a
-    for k, r in enumerate(ranks):
-        for i, m in enumerate(mats):
-            r.g(i).copy_(I.grad_bf16(m.rows, m.cols, seed=4 + k, stream=64 + i, device="cuda:0"))
-    torch.cuda.synchronize()
-    t = [0]
-
-    def phase(fn):
-        for r in ranks:
-            fn(r)
-
-    def step_fns():
-        t[0] += 1
-        hw, ha = pq.adamw(t[0], 2e-5), pq.adamw(t[0], 1e-4)
-        return [("pack", lambda r: r.pack_shards()),
-                ("gather_dequant", lambda r: r.gather_dequant()),
-                ("reduce_bwd_adamw", lambda r: r.reduce_step(hw, ha))]
-
-    for _ in range(max(args.warmup, 1)):
-        for _, fn in step_fns():
-            phase(fn)
-    torch.cuda.synchronize()
-    names = ["pack", "gather_dequant", "reduce_bwd_adamw"]
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * args.steps)]
-    for s_ in range(args.steps):
-        for j, (_, fn) in enumerate(step_fns()):
-            ev[4 * s_ + j].record()
-            phase(fn)
-        ev[4 * s_ + 3].record()
-    torch.cuda.synchronize()
-    ms = {n: sum(ev[4 * s_ + j].elapsed_time(ev[4 * s_ + j + 1]) for s_ in range(args.steps)) / args.steps
-          for j, n in enumerate(names)}
-    total = sum(ms.values())
-    weights = I.total_weights(mats)
-    nbytes = sharded_bytes(weights, world)
     peak, kind = measured_peaks()
-    phases = {n: {"ms_per_step": ms[n], "algorithmic_bytes": nbytes[n],
-                  "GB_s": nbytes[n] / (ms[n] * 1e-3) / 1e9,
-                  "frac_of_peak": nbytes[n] / (ms[n] * 1e-3) / 1e9 / peak} for n in names}
-    allb = sum(nbytes.values())
+    r = measure_sharded(args.world, args.layers, args.steps, args.warmup, peak, "cuda:0")
+    r["roofline"].update(peak_source=f"{kind} hbm_gbs", traffic=None)
     print(json.dumps({
         "metric": "row-sharded step (ranks emulated on one GPU) Gweights/s", "op": "sharded",
-        "value": weights / (total * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total,
+        "value": r["Gweights_s"], "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"],
         "higher_is_better": True, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"llama3_8b_first{args.layers}layers_seq2_sharded_world{world}_emulated",
-                   "weights": weights, "world": world,
-                   "note": "all ranks' work on one GPU in turn; peer reads are local HBM reads"},
-        "roofline": {"bound": "hbm", "kernel": "pack, dequant and reduce_bwd_adamw units kernels",
-                     "achieved": allb / (total * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
-                     "frac": allb / (total * 1e-3) / 1e9 / peak, "traffic": None,
-                     "peak_source": f"{kind} hbm_gbs", "algorithmic_bytes_per_step": allb},
-        "phases": phases,
-        # one batched launch per phase per rank (every batch here fits one launch)
-        "gpu_launches": 3 * world * args.steps}), flush=True)
+        "config": {"workload": r["workload"], "weights": r["weights"], "world": r["world"],
+                   "note": r["note"]},
+        "roofline": r["roofline"], "phases": r["phases"],
+        "gpu_launches": r["launches_total"]}), flush=True)
     return 0
 
 

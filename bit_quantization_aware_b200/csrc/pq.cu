@@ -31,6 +31,7 @@
 #include <stdint.h>
 
 #include "pq.h"
+#include "pq_launches.cuh"
 #include "pq_quant.cuh"
 
 // Tuning knobs (compile-time; the defaults are the measured choice):
@@ -65,6 +66,8 @@
 #ifndef PQ_ST_HINT
 #define PQ_ST_HINT 0
 #endif
+
+std::atomic<int64_t> pqc::launches{0};
 
 namespace pq {
 
@@ -908,6 +911,7 @@ static void launch_fwd(const Batch& b, cudaStream_t s) {
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
+    pqc::count_launch();
 }
 
 template <int Q, bool VEC>
@@ -917,6 +921,7 @@ static void launch_bwd(const Batch& b, cudaStream_t s) {
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
+    pqc::count_launch();
 }
 
 template <int Q, bool VEC>
@@ -926,6 +931,7 @@ static void launch_dequant(const Batch& b, cudaStream_t s) {
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
+    pqc::count_launch();
 }
 
 // ------------------------------------------------------- validation
@@ -1149,6 +1155,7 @@ static void launch_bwd_adamw(const AdamBatch& b, cudaStream_t s) {
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.b.total_units < ctas ? b.b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
+    pqc::count_launch();
 }
 
 static pq_status_t bwd_adamw_impl(int q, int32_t n, const pq_adamw_matrix_t* mats,
@@ -1218,6 +1225,7 @@ static void launch_reduce_bwd_adamw(const ReduceBatch& b, cudaStream_t s) {
     const int64_t ctas = persistent_ctas(k, cache);
     const unsigned grid = static_cast<unsigned>(b.b.total_units < ctas ? b.b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
+    pqc::count_launch();
 }
 
 static pq_status_t reduce_bwd_adamw_impl(int q, int32_t n_src, const uint16_t* const* srcs,
@@ -1347,6 +1355,7 @@ pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w, const 
     const int64_t gy = rows < 65535 ? rows : 65535;
     scaled_weights_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kThreads,
                             0, static_cast<cudaStream_t>(stream)>>>(w, alpha, x_out, rows, cols);
+    pqc::count_launch();
     return cuda_status(cudaGetLastError());
 }
 
@@ -1417,5 +1426,7 @@ const char* pq_status_string(pq_status_t s) {
 }
 
 int pq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int64_t pq_launch_count(void) { return pqc::launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

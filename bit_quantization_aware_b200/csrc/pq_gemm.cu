@@ -64,6 +64,7 @@
 #include <mutex>
 
 #include "pq.h"
+#include "pq_launches.cuh"
 
 namespace pqg {
 
@@ -1529,6 +1530,7 @@ static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
         attr_set[dev] = true;
     }
     wq_gemm_kernel<NT, MAXP, I8><<<prm.c.grid, kThreads, L::kBytes, s>>>(prm);
+    pqc::count_launch();
     return cudaGetLastError();
 }
 
@@ -1601,6 +1603,7 @@ static pq_status_t run_vector(int q, const pq_gemm_problem_t* pr, int count, voi
         pqv::gemv_i8_kernel<MAXP><<<grid, pqv::kThreads, smem, s>>>(V);
     else
         pqv::gemv_kernel<MAXP><<<grid, pqv::kThreads, smem, s>>>(V);
+    pqc::count_launch();
     return cudaGetLastError() == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }
 
@@ -1701,7 +1704,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         const int64_t cap = maxk / (16 * 64);
         sl = sl < cap ? sl : cap;
         X.slices = static_cast<int32_t>(sl < 1 ? 1 : sl);
-        xplanes_kernel<<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X);
+        xplanes_kernel<<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X); pqc::count_launch();
         if (cudaGetLastError() != cudaSuccess) return PQ_ERR_CUDA;
     }
     cudaError_t e;

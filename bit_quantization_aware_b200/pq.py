@@ -109,6 +109,8 @@ def _declare(L):
     L.pq_wq_gemm_workspace_bytes.restype = i64
     L.pq_device_status.argtypes = []
     L.pq_device_status.restype = i32
+    L.pq_launch_count.argtypes = []
+    L.pq_launch_count.restype = i64
     L.pq_debug_abort_waits.argtypes = [i32]
     L.pq_debug_abort_waits.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
@@ -397,6 +399,12 @@ def pq_wq_gemm_noalloc(q, x, packed, alpha, y_out, stream=None):
 def pq_device_status() -> int:
     """PQ_OK, or PQ_ERR_TIMEOUT once after a bounded device wait gave up."""
     return int(lib().pq_device_status())
+
+
+def pq_launch_count() -> int:
+    """Kernel launches the library has enqueued since it was loaded (the
+    launches of a call are the difference of two readings)."""
+    return int(lib().pq_launch_count())
 
 
 def pq_debug_abort_waits(on: bool) -> None:

@@ -5,6 +5,7 @@
     python -m bit_quantization_aware_b200.profile_case --rows 16384 --cols 16384 \
         --quant seq2 --iters 3 --gemm-m 1
     python -m bit_quantization_aware_b200.profile_case ... --op dequant | bwd_adamw
+    python -m bit_quantization_aware_b200.profile_case --set llama3_8b --iters 2
 
 Draws seeded synthetic inputs on the device (N(0, 0.02) weights, alpha =
 max|w_row| or the quantizer's init, bf16 N(0, 1e-3) upstream gradient),
@@ -16,6 +17,12 @@ prints the per-iteration CUDA-event times. Sized by the caller; a
 forward), ``--op bwd_adamw`` the backward fused with one AdamW step, and
 ``--gemm-m M`` the weight-only matmul with M activation rows on seeded
 random codes (only codes, scales, X and Y are allocated).
+
+``--set llama3_8b`` (or ``llama_1b``) runs the benchmark's batched forward
+and backward over a whole layer set instead of one matrix: one launch per
+phase, about 84 GB resident for the Llama-3-8B-shaped set. Its backward
+moves 70 GB per launch, so an L2-sized tail of dirty lines left after the
+kernel is below 0.2% of its writes (for one-pass DRAM counters only).
 """
 from __future__ import annotations
 
@@ -37,9 +44,13 @@ def main():
     p.add_argument("--gemm-m", type=int, default=0,
                    help="run the weight-only matmul with this many activation rows")
     p.add_argument("--op", default="quantizer", choices=["quantizer", "dequant", "bwd_adamw"])
+    p.add_argument("--set", default="", choices=["", "llama3_8b", "llama_1b"],
+                   help="a whole layer set in the benchmark's batched launches")
     a = p.parse_args()
     q = pq.QUANTIZERS[a.quant]
     dev = torch.device("cuda")
+    if a.set:
+        return set_case(a, q, dev)
     if a.gemm_m:
         return gemm_case(a, q, dev)
     if a.op != "quantizer":
@@ -67,6 +78,25 @@ def main():
         fb = 6 + (pq.pq_code_bits(q) / 8 if a.pack else 0)
         print(f"iter {i}: fwd {tf * 1e6:.1f} us ({n * fb / tf / 1e9:.0f} GB/s), "
               f"bwd {tb * 1e6:.1f} us ({n * 10 / tb / 1e9:.0f} GB/s)")
+
+
+def set_case(a, q, dev):
+    from .step import QuantStep
+    mats = I.llama3_8b_set() if a.set == "llama3_8b" else I.llama_1b_stack()
+    step = QuantStep(mats, q, device=dev, pack=a.pack)
+    step.generate(seed=3)
+    torch.cuda.synchronize()
+    for i in range(a.iters):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        step.fwd_all()
+        e[1].record()
+        step.bwd_all()
+        e[2].record()
+        torch.cuda.synchronize()
+        tf, tb = e[0].elapsed_time(e[1]) * 1e-3, e[1].elapsed_time(e[2]) * 1e-3
+        print(f"iter {i}: fwd {tf * 1e3:.3f} ms ({step.bytes_fwd() / tf / 1e9:.0f} GB/s), "
+              f"bwd {tb * 1e3:.3f} ms ({step.bytes_bwd() / tb / 1e9:.0f} GB/s)")
 
 
 def next_case(a, q, dev):

@@ -395,7 +395,11 @@ PQ_API int64_t pq_wq_gemm_batch_workspace_bytes(pq_quant_t q, int64_t m, int32_t
  *   Set-up: the first call on each device that passes the argument checks
  *          looks up the array's device address once (cudaGetSymbolAddress;
  *          a failure returns PQ_ERR_CUDA and the next call retries). Make
- *          that first call before any stream capture.
+ *          that first call before any stream capture. The address is kept
+ *          for the life of the process: after cudaDeviceReset on a device
+ *          the library's module is loaded again and the kept address may
+ *          be stale, so do not call this entry point on a device that has
+ *          been reset since its first call.
  *   Zeroing: the split-K counters at the end of the used scratch must be
  *          zero when the kernel starts; every call clears them on `stream`
  *          (cudaMemsetAsync) before its launch. The partial sums need no
@@ -438,6 +442,15 @@ PQ_API const char* pq_status_string(pq_status_t s);
 
 /* cudaError_t of the calling thread's last PQ_ERR_CUDA (0 if none). */
 PQ_API int pq_last_cuda_error(void);
+
+/* Number of kernel launches the library has enqueued since it was loaded,
+ * over all devices, streams and threads (a host-side counter, read without
+ * synchronising). A call's launches are the difference of two readings;
+ * under stream capture it counts the launches captured into the graph,
+ * which every replay of the graph repeats. No counterpart in the pages:
+ * it lets a caller report how many of this library's kernels a timed
+ * region ran. */
+PQ_API int64_t pq_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -386,18 +386,21 @@ int pqo_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alpha,
  * n_src bf16 gradients (one per data-parallel replica, for the same rows):
  * gbar = fl(fl(sum_k g_k) * grad_mult), summed in source order in fp32;
  * then exactly pqo_bwd_adamw's steps with the fp32 gbar in place of g
- * (dW = inside ? gbar : 0; the d(alpha) term is gbar*(level - inside*x)). */
+ * (dW = inside ? gbar : 0; the d(alpha) term is gbar*(level - inside*x)).
+ * row_abs (nullable) receives sum_j |term_j| per row before grad_scale, as
+ * pqo_bwd gives it, for the tolerance floor of rows whose sum cancels. */
 int pqo_reduce_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alpha,
                          int n_src, const uint16_t* const* g_srcs, float grad_mult,
                          float* m_w, float* v_w, float* m_a, float* v_a, float grad_scale,
-                         const pqo_adamw* hw, const pqo_adamw* ha, float* dalpha) {
+                         const pqo_adamw* hw, const pqo_adamw* ha, float* dalpha,
+                         double* row_abs) {
     pqo_params p;
     if (pqo_get_params(q, &p) || rows < 0 || cols < 0 || n_src < 1 || !g_srcs || !hw || !ha)
         return -1;
     const pqo_adamw_k kw = pqo_adamw_consts(hw), ka = pqo_adamw_consts(ha);
     for (int64_t r = 0; r < rows; ++r) {
         const float a = alpha[r];
-        double acc = 0.0;
+        double acc = 0.0, acc_abs = 0.0;
         for (int64_t j = 0; j < cols; ++j) {
             float sum = 0.0f;
             for (int k = 0; k < n_src; ++k) {
@@ -409,13 +412,16 @@ int pqo_reduce_bwd_adamw(int q, int64_t rows, int64_t cols, float* w, float* alp
             float lev, x;
             pqo_quantize_scalar(q, w[r * cols + j], a, 0.0f, NULL, &lev, NULL, &inside, &x);
             const float dw = inside ? gbar : 0.0f;
-            acc += (double)gbar * ((double)lev - (inside ? (double)x : 0.0));
+            const double term = (double)gbar * ((double)lev - (inside ? (double)x : 0.0));
+            acc += term;
+            acc_abs += fabs(term);
             w[r * cols + j] = pqo_adamw_update(&kw, w[r * cols + j], dw, &m_w[r * cols + j],
                                                &v_w[r * cols + j]);
         }
         const float da = (float)(acc * (double)grad_scale);
         alpha[r] = pqo_adamw_update(&ka, a, da, &m_a[r], &v_a[r]);
         if (dalpha) dalpha[r] = da;
+        if (row_abs) row_abs[r] = acc_abs;
     }
     return 0;
 }

@@ -84,7 +84,7 @@ class Oracle:
         L.pqo_bwd_adamw.restype = ctypes.c_int
         L.pqo_reduce_bwd_adamw.argtypes = [ctypes.c_int, i64, i64, p, p, ctypes.c_int, p,
                                            ctypes.c_float, p, p, p, p, ctypes.c_float,
-                                           ctypes.POINTER(AdamW), ctypes.POINTER(AdamW), p]
+                                           ctypes.POINTER(AdamW), ctypes.POINTER(AdamW), p, p]
         L.pqo_reduce_bwd_adamw.restype = ctypes.c_int
         L.pqo_wq_matmul.argtypes = [ctypes.c_int, i64, i64, i64, p, p, p, p]
         L.pqo_wq_matmul.restype = ctypes.c_int
@@ -188,7 +188,8 @@ class Oracle:
     def reduce_bwd_adamw(self, q, w, alpha, g_list, grad_mult, m_w, v_w, m_a, v_a,
                          grad_scale, hw, ha):
         """Backward + AdamW with the upstream gradient summed over the bf16
-        arrays of g_list; returns (w, alpha, m_w, v_w, m_a, v_a, dalpha)."""
+        arrays of g_list; returns (w, alpha, m_w, v_w, m_a, v_a, dalpha,
+        row_abs), row_abs the per-row sum of |term| before grad_scale."""
         w = np.array(w, np.float32, order="C", copy=True)
         rows, cols = w.shape
         alpha = np.array(alpha, np.float32, copy=True).reshape(rows)
@@ -199,14 +200,16 @@ class Oracle:
         m_a = np.array(m_a, np.float32, copy=True).reshape(rows)
         v_a = np.array(v_a, np.float32, copy=True).reshape(rows)
         da = np.empty(rows, np.float32)
+        row_abs = np.empty(rows, np.float64)
         rc = self.lib.pqo_reduce_bwd_adamw(q, rows, cols, _ptr(w), _ptr(alpha), len(gs),
                                            ctypes.cast(ptrs, ctypes.c_void_p),
                                            ctypes.c_float(grad_mult), _ptr(m_w), _ptr(v_w),
                                            _ptr(m_a), _ptr(v_a), ctypes.c_float(grad_scale),
-                                           ctypes.byref(hw), ctypes.byref(ha), _ptr(da))
+                                           ctypes.byref(hw), ctypes.byref(ha), _ptr(da),
+                                           _ptr(row_abs))
         if rc != 0:
             raise ValueError("oracle reduce_bwd_adamw rejected its arguments")
-        return w, alpha, m_w, v_w, m_a, v_a, da
+        return w, alpha, m_w, v_w, m_a, v_a, da, row_abs
 
     def wq_matmul(self, q, x_bf16, packed, alpha, k):
         """Y = X * (alpha * levels(codes))^T in fp64; x_bf16 [M, K] bits,

@@ -57,3 +57,69 @@ def check_bwd(q, w_np, a_np, g_np, gs, dw_gpu, da_gpu):
     assert np.all(err <= tol), (
         f"q={q}: dalpha row {worst}: gpu={da[worst]!r} ref={ref_da[worst]!r}")
     return float(np.max(err / np.maximum(np.abs(ref_da), 1e-30))) if len(err) else 0.0
+
+
+def compare_rows(q, w, a, g, gs, wq_bits, packed, dw_bits, da):
+    """The oracle's forward (+ packed codes) and backward of these rows
+    against the GPU's outputs (host arrays). Returns a list of mismatch
+    descriptions, empty when bf16 weights, packed bytes and dW are
+    bit-exact and d(alpha) is within tolerance."""
+    errs = []
+    ref_wq, _, ref_pk = pq_oracle.fwd(q, w, a, pack=packed is not None)
+    if wq_bits is not None:
+        bad = np.argwhere(wq_bits != ref_wq)
+        if bad.size:
+            r, c = bad[0]
+            errs.append(f"{len(bad)} bf16 weights differ, first at ({r}, {c}): "
+                        f"gpu {wq_bits[r, c]:#06x} oracle {ref_wq[r, c]:#06x}")
+    if packed is not None:
+        bad = np.argwhere(packed != ref_pk)
+        if bad.size:
+            errs.append(f"{len(bad)} packed bytes differ, first at {bad[0].tolist()}")
+    ref_dw, ref_da, row_abs = pq_oracle.bwd(q, w, a, g, gs)
+    bad = np.argwhere(dw_bits != ref_dw.view(np.uint32))
+    if bad.size:
+        errs.append(f"{len(bad)} dW values differ, first at {bad[0].tolist()}")
+    tol = DALPHA_RTOL * np.maximum(np.abs(ref_da).astype(np.float64),
+                                   DALPHA_FLOOR * abs(gs) * row_abs)
+    err = np.abs(da.astype(np.float64) - ref_da.astype(np.float64))
+    if not np.all(err <= tol):
+        r = int(np.argmax(err - tol))
+        errs.append(f"d(alpha) row {r}: gpu {da[r]!r} oracle {ref_da[r]!r}")
+    return errs
+
+
+def check_step_every_element(step, pool, task_weights=1 << 22):
+    """Every element of every matrix of a QuantStep (after one forward and
+    one backward) against the oracle: bf16 weights, packed codes (if the
+    step packs) and dW bit-exact, d(alpha) within tolerance. Matrices come
+    to the host one at a time; the oracle runs on slices of about
+    ``task_weights`` weights in ``pool`` (ctypes releases the interpreter
+    lock), at most two matrices in flight. Returns the number of weights
+    compared."""
+    q = step.q
+    pending, checked = [], 0
+
+    def drain(items):
+        for name, r0, fut in items:
+            errs = fut.result()
+            assert not errs, f"{name} rows from {r0}: " + "; ".join(errs)
+
+    for b in step.bufs:
+        w, a, g = f32(b.w), f32(b.alpha), bits16(b.g)
+        wq = bits16(b.wq)
+        pk = u8(b.packed) if b.packed is not None else None
+        dw = f32(b.dw).view(np.uint32)
+        da = f32(b.dalpha)
+        per = max(1, task_weights // max(1, b.m.cols))
+        futs = []
+        for r0 in range(0, b.m.rows, per):
+            s = slice(r0, min(b.m.rows, r0 + per))
+            futs.append((b.m.name, r0, pool.submit(
+                compare_rows, q, w[s], a[s], g[s], b.grad_scale, wq[s],
+                None if pk is None else pk[s], dw[s], da[s])))
+        drain(pending)
+        pending = futs
+        checked += b.m.numel
+    drain(pending)
+    return checked

@@ -488,11 +488,15 @@ def check_reduce_equals_single_source(O):
               np.abs(rng.normal(0, 1e-7, 4)).astype(np.float32)]
         hw, ha = AdamW.at_step(2, 2e-5), AdamW.at_step(2, 1e-4)
         ref = O.bwd_adamw(q, w, a, gb, *st, 0.5, hw, ha)
+        # the per-row sum of |terms| of the plain backward (a diagnostic
+        # output: the tolerance floor of rows whose sum cancels)
+        _, _, ref_abs = O.bwd(q, w, a, gb, 0.5)
         for n, mult in ((1, 1.0), (2, 0.5), (4, 0.25)):
             got = O.reduce_bwd_adamw(q, w, a, [gb] * n, mult, *st, 0.5, hw, ha)
-            for x, y in zip(got, ref):
+            for x, y in zip(got[:7], ref):
                 assert np.array_equal(np.asarray(x).view(np.uint32),
                                       np.asarray(y).view(np.uint32)), (q, n)
+            assert np.array_equal(got[7], ref_abs), (q, n)
 
 
 def check_reduce_sums_in_fp32(O):

@@ -35,7 +35,7 @@ def test_header_declares_entry_points():
               "pq_wq_gemm", "pq_wq_gemm_workspace_bytes", "pq_device_status",
               "pq_wq_gemm_noalloc", "pq_wq_gemm_batch", "pq_wq_gemm_batch_workspace_bytes", "pq_debug_abort_waits",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
-              "pq_last_cuda_error"):
+              "pq_last_cuda_error", "pq_launch_count"):
         assert n in names
 
 
@@ -69,6 +69,11 @@ def test_host_helpers_match_oracle(L):
     for s in range(6):
         assert pq.status_string(s)
     assert L.pq_last_cuda_error() == 0
+    # argument checks that fail launch nothing, so the counter stays put
+    n0 = pq.pq_launch_count()
+    assert pq.pq_default_grad_scale(pq.PQ_SEQ2, 1024) > 0
+    assert L.pq_fakequant_fwd(99, 4, 8, None, None, None, None, None) == pq.PQ_ERR_INVALID_ARG
+    assert pq.pq_launch_count() == n0 >= 0
 
 
 def test_argument_errors_launch_nothing(L):

@@ -1,10 +1,10 @@
 """GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
 
 Bit-exact for bf16 dequantized weights, packed codes and fp32 dW; d(alpha)
-within 1e-4 relative (floor: 1e-6 of the row's sum of |terms|). Small cases
-compare every element; the full-size workloads run in the launch
-configuration of the benchmark and compare sampled rows, which the oracle
-computes one by one (every output row depends only on its own inputs).
+within 1e-4 relative (floor: 1e-6 of the row's sum of |terms|). Every case
+compares every element, the full-size workloads too: they run in the launch
+configuration of the benchmark, come to the host one matrix at a time, and
+the single-threaded oracle runs on row slices from a thread pool.
 """
 import numpy as np
 import pytest
@@ -14,7 +14,7 @@ from bit_quantization_aware_b200 import inputs as I
 from bit_quantization_aware_b200 import pq
 from bit_quantization_aware_b200.step import QuantStep
 from oracle import pq_oracle
-from tests.gpu_util import bits16, check_bwd, check_fwd, f32
+from tests.gpu_util import bits16, check_bwd, check_fwd, check_step_every_element, f32
 
 pytestmark = pytest.mark.gpu
 
@@ -145,48 +145,28 @@ def test_bit_width_sweep_2048x8192(q, rule):
     check_bwd(q, wn, an, gn, gs, dw, da)
 
 
-def _sampled_rows(step, rows_per_matrix, seed=0):
-    rng = np.random.default_rng(seed)
-    for b in step.bufs:
-        r = b.m.rows
-        pick = sorted(set([0, r - 1] + rng.integers(0, r, rows_per_matrix).tolist()))
-        yield b, pick
-
-
-def _check_step_rows(step, rows_per_matrix):
-    q = step.q
-    for b, pick in _sampled_rows(step, rows_per_matrix):
-        idx = torch.tensor(pick, device=DEV)
-        wn = f32(b.w.index_select(0, idx))
-        an = f32(b.alpha.index_select(0, idx))
-        gn = bits16(b.g.index_select(0, idx))
-        check_fwd(q, wn, an, b.wq.index_select(0, idx),
-                  b.packed.index_select(0, idx) if b.packed is not None else None)
-        check_bwd(q, wn, an, gn, b.grad_scale, b.dw.index_select(0, idx),
-                  b.dalpha.index_select(0, idx))
-
-
 @pytest.mark.parametrize("which", ["llama_1b_stack", "llama3_8b_set"])
-def test_layer_set_full_size_sampled(which):
+def test_layer_set_full_size_every_element(which, oracle_pool):
     """The full layer sets in the benchmark's launch configuration (one
-    forward over all matrices, then one backward over all), SEQ2; sampled
-    rows of every matrix compared with the oracle."""
+    batched forward over all matrices, then one batched backward), SEQ2;
+    every element of every matrix compared with the oracle (the 1B-class
+    stack: 1.08 G weights; the Llama-3-8B-shaped set: 6.98 G weights)."""
     mats = getattr(I, which)()
     step = QuantStep(mats, pq.PQ_SEQ2, device=DEV)
     step.generate(seed=2 if which == "llama_1b_stack" else 3)
     step.run()
     torch.cuda.synchronize()
-    _check_step_rows(step, rows_per_matrix=3)
+    assert check_step_every_element(step, oracle_pool) == I.total_weights(mats)
     del step
     torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("q", [pq.PQ_SEQ2, pq.PQ_TERNARY])
-def test_student_t_16384_planted_ties(q):
+def test_student_t_16384_planted_ties(q, oracle_pool):
     """16384x16384 Student-t(3)*0.02 with 1% of entries planted exactly on
     the clip bounds and on rounding ties; forward + packed codes + backward;
-    512 sampled rows compared; most planted entries hit their target
-    exactly (about 85%)."""
+    every element compared (bf16 weights, packed bytes, dW, d(alpha)); most
+    planted entries hit their target exactly (about 85%)."""
     mats = [I.Matrix("t3.16384", 16384, 16384, 0, 0)]
     step = QuantStep(mats, q, device=DEV, pack=True)
     step.generate(seed=4, dist="student_t")
@@ -198,7 +178,7 @@ def test_student_t_16384_planted_ties(q):
     print(f"planted {n} entries, {hit} exactly on a clip bound or tie")
     step.run()
     torch.cuda.synchronize()
-    _check_step_rows(step, rows_per_matrix=512)
+    assert check_step_every_element(step, oracle_pool) == 16384 * 16384
     del step
     torch.cuda.empty_cache()
 
@@ -603,3 +583,23 @@ def test_bwd_adamw_batch_2048x8192_and_stack():
         for x, y in zip(s1, s2):
             assert torch.equal(x.view(torch.uint8) if x.dtype != torch.bfloat16 else x.view(torch.int16),
                                y.view(torch.uint8) if y.dtype != torch.bfloat16 else y.view(torch.int16))
+
+
+def test_launch_counter_counts_batched_launches():
+    """pq_launch_count: a batched forward over 300 matrices of the vector
+    layout goes out as two launches (256 descriptors per launch), and a
+    rejected call launches nothing."""
+    q = pq.PQ_SEQ2
+    shapes = [(3 + i % 5, 8 * (1 + i % 7)) for i in range(300)]
+    ws = [torch.randn(r, c, device=DEV) for r, c in shapes]
+    descs = [dict(rows=r, cols=c, w=w, alpha=w.abs().amax(1).clamp_min(1e-30).contiguous(),
+                  wq=torch.empty(r, c, dtype=torch.bfloat16, device=DEV))
+             for (r, c), w in zip(shapes, ws)]
+    arr = pq.matrix_array(descs)
+    n0 = pq.pq_launch_count()
+    pq.pq_fakequant_fwd_batch(q, arr)
+    torch.cuda.synchronize()
+    assert pq.pq_launch_count() - n0 == 2
+    with pytest.raises(pq.PQError):
+        pq.pq_fakequant_fwd_batch(99, arr)
+    assert pq.pq_launch_count() - n0 == 2

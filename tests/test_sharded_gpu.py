@@ -13,6 +13,7 @@ from bit_quantization_aware_b200 import pq
 from bit_quantization_aware_b200.sharded import LocalPeers, ShardedQuantStep
 from oracle import pq_oracle
 from oracle.pq_oracle import AdamW
+from tests.gpu_util import DALPHA_FLOOR, DALPHA_RTOL
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -111,6 +112,10 @@ def test_reduce_bwd_adamw_matches_oracle(q):
     for x, y in ((wd, ref[0]), (mwd, ref[2]), (vwd, ref[3])):
         assert np.array_equal(x.cpu().numpy().view(np.uint32), y.view(np.uint32))
     da = dad.cpu().numpy()
-    assert np.allclose(da, ref[6], rtol=1e-4, atol=1e-12)
+    # the d(alpha) tolerance of every parity test: 1e-4 relative, floored at
+    # 1e-6 of the row's sum of |terms| times grad_scale
+    tol = DALPHA_RTOL * np.maximum(np.abs(ref[6]).astype(np.float64),
+                                   DALPHA_FLOOR * abs(gsc) * ref[7])
+    assert np.all(np.abs(da.astype(np.float64) - ref[6].astype(np.float64)) <= tol)
     pa, pma, pva = pq_oracle.default().adamw_step(a.numpy(), da, ma, va, ha_o)
     assert np.array_equal(ad.cpu().numpy().view(np.uint32), pa.view(np.uint32))

@@ -2,9 +2,11 @@
 existing pq_wq_gemm entry point (caller workspace), on two consecutive
 calls each: the second call reuses the scratch the first one left.
 
-Tolerance is that of the weight-only matmul tests: 2^-8 of |Y| plus 1e-4 of
-sum_k |x_k * w_k|. This file is collected last so that it also runs after
-every other GPU test in the same process."""
+Both entry points run the same kernel with the same split plan, so the
+outputs must be the same bits; the check also applies the tolerance of the
+weight-only matmul tests (2^-8 of |Y| plus 1e-4 of sum_k |x_k * w_k|) so
+that a failure says how far off a result is. This file is collected last
+so that it also runs after every other GPU test in the same process."""
 import numpy as np
 import pytest
 import torch
@@ -52,6 +54,9 @@ def test_noalloc_matches_workspace_entry_point(q, m, n, k):
         got = y.float().cpu().numpy().astype(np.float64)
         err = np.abs(got - ref64)
         assert np.all(err <= tol), f"call {call}: max error {err.max()} over tolerance"
+        same = torch.equal(y.view(torch.int16), ref.view(torch.int16))
+        assert same, f"call {call}: {int((y.view(torch.int16) != ref.view(torch.int16)).sum())} " \
+                     "outputs differ in their bits from pq_wq_gemm"
 
 
 def test_noalloc_rejects_problems_over_the_scratch_limit():
