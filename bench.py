@@ -525,7 +525,7 @@ def measure_case(case, steps, warmup, peak, device, flush, oracle_seconds):
             entry["pack_standalone"] = phase_entry(med["pack_standalone"], w, nb, peak)
         if planted:
             entry["planted"] = planted
-        del step, fns, b
+        del step, fns
         torch.cuda.empty_cache()
         if oracle_seconds > 0:
             sample = oracle_sample(case["mats"], q, oracle_seconds, seed=case["seed"],

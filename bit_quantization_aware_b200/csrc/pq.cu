@@ -8,15 +8,20 @@
 //   parameters), so a training step's many small and large matrices cost
 //   one launch per phase, with no per-matrix ramp-up and tail.
 // * A CTA of 256 threads splits into row groups of TPR threads (a power of
-//   two, 1..256, chosen per matrix so that each thread owns about eight
-//   chunks of 8 weights of its row). Each thread issues the loads of several
-//   chunks (2 in the forward and the backward) before computing any of
-//   them; a chunk's 8 fp32 values move as one 256-bit access, so a warp
-//   instruction covers 1024 contiguous bytes.
-// * A persistent grid (the occupancy limit; the backward's registers are
-//   capped for 4 CTAs per SM) walks the units in order, so concurrent CTAs
-//   stream neighbouring rows. An optional bulk L2 prefetch of each CTA's
-//   next unit (cp.async.bulk.prefetch.L2) measured slower and is off.
+//   two, 1..256, chosen per matrix so that each thread owns about sixteen
+//   (forward) or eight (backward) chunks of 8 weights of its row). Each
+//   thread issues the loads of several chunks (3 in the forward, 2 in the
+//   backward) before computing any of them; a chunk's 8 fp32 values move
+//   as one 256-bit access, so a warp instruction covers 1024 contiguous
+//   bytes.
+// * A persistent grid (the occupancy limit; the forward's and backward's
+//   registers are capped for 4 CTAs per SM) walks the units in order, so
+//   concurrent CTAs stream neighbouring rows. An optional bulk L2 prefetch
+//   of each CTA's next unit (cp.async.bulk.prefetch.L2) measured slower and
+//   is off.
+// * The dequantization of packed codes stages each unit's bf16 output (a
+//   block of whole rows, contiguous in memory) in shared memory and writes
+//   it with one bulk copy (cp.async.bulk, the TMA engine), double-buffered.
 // * The backward reduces the scale gradient per row in a fixed order: fp64
 //   partial sums per thread, warp shuffles, then (TPR > 32) one shared-memory
 //   slot per warp summed by the group's first thread after a barrier of the
@@ -38,10 +43,19 @@
 //   PQ_PREFETCH      1: bulk L2 prefetch of each CTA's next unit
 //   PQ_CTAS_PER_SM   persistent CTAs per SM (0: the occupancy limit)
 //   PQ_CHUNKS_PER_THREAD  target chunks of 8 weights per thread and row
+//                    (PQ_FWD_CHUNKS_PER_THREAD: the forward's target)
 //   PQ_FWD_UNROLL, PQ_BWD_UNROLL  chunks whose loads a thread issues
-//                    before computing any of them
+//                    before computing any of them (PQ_PACK_UNROLL: the
+//                    forward instance that writes packed codes only)
 //   PQ_LD_HINT, PQ_ST_HINT  cache hints of the streaming loads and stores
+//                    (loads: 0 evict-first, 1 read-only path, 2 default,
+//                    3 evict-first with a 256-byte L2 prefetch, 4 read-only
+//                    without L1 allocation with a 256-byte L2 prefetch)
 //   PQ_BWD_MIN_CTAS  resident CTAs per SM the backward's registers must allow
+//   PQ_FWD_MIN_CTAS  the same for the forward (0: no register cap)
+//   PQ_DEQ_BULK      1: the dequantization stages each unit's bf16 output in
+//                    shared memory and writes it with one bulk copy
+//   PQ_DEQ_BUF_KB    size of one such staging buffer (two per CTA)
 #ifndef PQ_PREFETCH
 #define PQ_PREFETCH 0
 #endif
@@ -51,8 +65,14 @@
 #ifndef PQ_CHUNKS_PER_THREAD
 #define PQ_CHUNKS_PER_THREAD 8
 #endif
+#ifndef PQ_FWD_CHUNKS_PER_THREAD
+#define PQ_FWD_CHUNKS_PER_THREAD 16
+#endif
 #ifndef PQ_FWD_UNROLL
-#define PQ_FWD_UNROLL 2
+#define PQ_FWD_UNROLL 3
+#endif
+#ifndef PQ_PACK_UNROLL
+#define PQ_PACK_UNROLL 2
 #endif
 #ifndef PQ_BWD_UNROLL
 #define PQ_BWD_UNROLL 2
@@ -65,6 +85,20 @@
 #endif
 #ifndef PQ_ST_HINT
 #define PQ_ST_HINT 0
+#endif
+#ifndef PQ_FWD_MIN_CTAS
+#define PQ_FWD_MIN_CTAS 4
+#endif
+#ifndef PQ_DEQ_BULK
+#define PQ_DEQ_BULK 1
+#endif
+#ifndef PQ_DEQ_BUF_KB
+#define PQ_DEQ_BUF_KB 32
+#endif
+#if PQ_FWD_MIN_CTAS > 0
+#define PQ_FWD_BOUNDS __launch_bounds__(kThreads, PQ_FWD_MIN_CTAS)
+#else
+#define PQ_FWD_BOUNDS __launch_bounds__(kThreads)
 #endif
 
 std::atomic<int64_t> pqc::launches{0};
@@ -108,6 +142,14 @@ __device__ __forceinline__ void st_stream(T* p, T v) {
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 #if PQ_LD_HINT == 0
     asm("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "l"(p));
+#elif PQ_LD_HINT == 3
+    asm("ld.global.cs.L2::256B.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "l"(p));
+#elif PQ_LD_HINT == 4
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
         : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
         : "l"(p));
 #else
@@ -168,6 +210,10 @@ __device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes) {
         c += n;
         bytes -= n;
     }
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
 // Barrier over the `count` threads of one row group (ids 1..8; id 0 is
@@ -322,7 +368,7 @@ __device__ __forceinline__ void prefetch_unit(const Batch& p, int mi, int64_t u)
 
 // ------------------------------------------------------------------ forward
 template <int Q, bool VEC, bool WQ, bool PACK>
-__global__ void __launch_bounds__(kThreads)
+__global__ void PQ_FWD_BOUNDS
 fwd_units_kernel(const __grid_constant__ Batch p) {
     int mi = 0;
     for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x) {
@@ -345,7 +391,9 @@ fwd_units_kernel(const __grid_constant__ Batch p) {
         const float* wr = m.w + row * m.cols;
         uint16_t* qr = WQ ? m.wq + row * m.cols : nullptr;
         uint8_t* pr = PACK ? m.packed + row * (m.cols * Traits<Q>::bits / 8) : nullptr;
-        constexpr int U = VEC ? PQ_FWD_UNROLL : 2;  // element path: fewer registers
+        // chunks in flight: the packed-codes-only instance keeps no bf16
+        // outputs live, so it can hold more; element path: fewer registers
+        constexpr int U = VEC ? (WQ ? PQ_FWD_UNROLL : PQ_PACK_UNROLL) : 2;
         for (int64_t ch = c_begin + lane; ch < c_end; ch += U * tpr) {
             float v[U][8];
 #pragma unroll
@@ -488,6 +536,135 @@ __device__ __forceinline__ uint32_t spread2(uint32_t b) {
     return ((b & 0x33u) * 0x1001u | (b & 0xCCu) * 0x40040u) & 0x03030303u;
 }
 
+// Eight codes of one chunk (2-bit: 16 bits of pk; 4-bit: 32 bits) as eight
+// bf16 outputs. 2-bit: byte permutes of the row's table (lo, hi);
+// 4-bit: arithmetic decode and one fp32 multiply each.
+template <int Q>
+__device__ __forceinline__ uint4 dequant_chunk(uint32_t pk, uint32_t lo, uint32_t hi, float a) {
+    constexpr int B = Traits<Q>::bits;
+    constexpr uint32_t mask = (1u << B) - 1u;
+    uint32_t o[4];
+    if constexpr (B == 2) {
+        const uint32_t t0 = spread2(pk & 0xFFu);
+        const uint32_t t1 = spread2(pk >> 8);
+        o[0] = prmt(lo, hi, t0 * 0x11u + 0x4040u);
+        o[1] = prmt(lo, hi, (t0 >> 16) * 0x11u + 0x4040u);
+        o[2] = prmt(lo, hi, t1 * 0x11u + 0x4040u);
+        o[3] = prmt(lo, hi, (t1 >> 16) * 0x11u + 0x4040u);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = pack_bf16x2(__fmul_rn(level_of_field<Q>((pk >> (8 * j)) & mask), a),
+                               __fmul_rn(level_of_field<Q>((pk >> (8 * j + 4)) & mask), a));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The row's four 2-bit outputs as a byte-planar table (lo = low bytes of
+// entries 0..3, hi = high bytes) for dequant_chunk.
+template <int Q>
+__device__ __forceinline__ void dequant_table(float a, uint32_t& lo, uint32_t& hi) {
+    const uint32_t e01 = pack_bf16x2(__fmul_rn(level_of_field<Q>(0), a),
+                                     __fmul_rn(level_of_field<Q>(1), a));
+    const uint32_t e23 = pack_bf16x2(__fmul_rn(level_of_field<Q>(2), a),
+                                     __fmul_rn(level_of_field<Q>(3), a));
+    lo = prmt(e01, e23, 0x6420);
+    hi = prmt(e01, e23, 0x7531);
+}
+
+// ---------------------------------------------- bulk (TMA engine) stores
+constexpr int kDeqBuf = PQ_DEQ_BUF_KB * 1024;        // bytes of one staging buffer
+constexpr int kDeqChunks = kDeqBuf / (kThreads * 16);  // chunks per thread that fill it
+
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the bulk stores of all but the newest group have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Vector-layout dequantization with staged output: a unit (a block of whole
+// rows, at most kDeqBuf bytes of bf16 output, contiguous in memory) is
+// decoded into one of two shared-memory buffers, then written by a single
+// bulk copy that thread 0 issues; the other buffer is filled meanwhile.
+// Thread 0 waits for a buffer's previous copy to finish reading before the
+// CTA refills it. Every thread reaches both barriers of every unit.
+template <int Q>
+__global__ void __launch_bounds__(kThreads)
+dequant_bulk_kernel(const __grid_constant__ Batch p) {
+    constexpr int B = Traits<Q>::bits;
+    extern __shared__ __align__(128) uint8_t sbuf[];
+    int mi = 0;
+    uint32_t it = 0;
+    for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x, ++it) {
+        mi = find_matrix(p, mi, u);
+        const MatDesc& m = p.m[mi];
+        const int tl = m.tpr_log2;
+        const int tpr = 1 << tl;
+        const int lane = threadIdx.x & (tpr - 1);
+        const int rsub = threadIdx.x >> tl;
+        const int rpb = kThreads >> tl;
+        const int64_t row0 = (u - m.unit_begin) * rpb;
+        const int64_t row = row0 + rsub;
+        const int64_t nrows = (m.rows - row0) < rpb ? (m.rows - row0) : rpb;
+        const int64_t nch = m.cols >> 3;
+        const bool live = row < m.rows;
+        // this thread's codes (at most kDeqChunks chunks of its row)
+        uint32_t pk[kDeqChunks];
+        float a = 0.0f;
+        if (live) {
+            a = __ldg(m.alpha + row);
+            const uint8_t* src = m.packed + row * (m.cols * B / 8);
+#pragma unroll
+            for (int k = 0; k < kDeqChunks; ++k) {
+                const int64_t c = lane + static_cast<int64_t>(k) * tpr;
+                if (c < nch) {
+                    if constexpr (B == 2)
+                        pk[k] = ld_stream(reinterpret_cast<const unsigned short*>(src + c * 2));
+                    else
+                        pk[k] = ld_stream(reinterpret_cast<const unsigned int*>(src + c * 4));
+                }
+            }
+        }
+        uint8_t* buf = sbuf + (it & 1u) * kDeqBuf;
+        if (threadIdx.x == 0) bulk_wait_read_all_but_one();
+        __syncthreads();
+        if (live) {
+            uint32_t lo = 0, hi = 0;
+            if constexpr (B == 2) dequant_table<Q>(a, lo, hi);
+            const uint32_t rbase = smem_addr(buf) + static_cast<uint32_t>(rsub * m.cols * 2);
+#pragma unroll
+            for (int k = 0; k < kDeqChunks; ++k) {
+                const int64_t c = lane + static_cast<int64_t>(k) * tpr;
+                if (c < nch) {
+                    const uint4 o = dequant_chunk<Q>(pk[k], lo, hi, a);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     rbase + static_cast<uint32_t>(c * 16)),
+                                 "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+                                 : "memory");
+                }
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            bulk_store(m.wq + row0 * m.cols, smem_addr(buf),
+                       static_cast<uint32_t>(nrows * m.cols * 2));
+            bulk_commit();
+        }
+    }
+    if (threadIdx.x == 0) bulk_wait_all();
+}
+
 template <int Q, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 dequant_units_kernel(const __grid_constant__ Batch p) {
@@ -510,14 +687,7 @@ dequant_units_kernel(const __grid_constant__ Batch p) {
             // lane l decodes chunks l, l + tpr, ... of 8 codes: each warp
             // store writes 512 contiguous bytes
             uint32_t lo = 0, hi = 0;
-            if constexpr (B == 2) {  // table of the 4 outputs, byte-planar
-                const uint32_t e01 = pack_bf16x2(__fmul_rn(level_of_field<Q>(0), a),
-                                                 __fmul_rn(level_of_field<Q>(1), a));
-                const uint32_t e23 = pack_bf16x2(__fmul_rn(level_of_field<Q>(2), a),
-                                                 __fmul_rn(level_of_field<Q>(3), a));
-                lo = prmt(e01, e23, 0x6420);
-                hi = prmt(e01, e23, 0x7531);
-            }
+            if constexpr (B == 2) dequant_table<Q>(a, lo, hi);  // the 4 outputs, byte-planar
             constexpr int U = 4;
             const int64_t nch = m.cols >> 3;
             for (int64_t ch = lane; ch < nch; ch += U * tpr) {
@@ -535,25 +705,9 @@ dequant_units_kernel(const __grid_constant__ Batch p) {
 #pragma unroll
                 for (int k = 0; k < U; ++k) {
                     const int64_t c = ch + k * tpr;
-                    if (c < nch) {
-                        uint32_t o[4];
-                        if constexpr (B == 2) {
-                            const uint32_t t0 = spread2(pk[k] & 0xFFu);
-                            const uint32_t t1 = spread2(pk[k] >> 8);
-                            o[0] = prmt(lo, hi, t0 * 0x11u + 0x4040u);
-                            o[1] = prmt(lo, hi, (t0 >> 16) * 0x11u + 0x4040u);
-                            o[2] = prmt(lo, hi, t1 * 0x11u + 0x4040u);
-                            o[3] = prmt(lo, hi, (t1 >> 16) * 0x11u + 0x4040u);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                o[j] = pack_bf16x2(
-                                    __fmul_rn(level_of_field<Q>((pk[k] >> (8 * j)) & mask), a),
-                                    __fmul_rn(level_of_field<Q>((pk[k] >> (8 * j + 4)) & mask), a));
-                        }
+                    if (c < nch)
                         st_stream(reinterpret_cast<uint4*>(dst + c * 8),
-                                  make_uint4(o[0], o[1], o[2], o[3]));
-                    }
+                                  dequant_chunk<Q>(pk[k], lo, hi, a));
                 }
             }
         } else {  // element path: groups of 8 codes
@@ -852,10 +1006,13 @@ static inline int ilog2_ceil(int64_t v) {
 
 // Threads per row: a power of two, 1..256, giving each thread about
 // PQ_CHUNKS_PER_THREAD chunks of 8 weights of its row.
-static inline int choose_tpr_log2(int64_t cols) {
-    const int64_t nch = (cols + 7) / 8;
-    const int l = ilog2_ceil((nch + PQ_CHUNKS_PER_THREAD - 1) / PQ_CHUNKS_PER_THREAD);
+static inline int choose_tpr_log2_for(int64_t nch, int chunks_per_thread) {
+    const int l = ilog2_ceil((nch + chunks_per_thread - 1) / chunks_per_thread);
     return l > 8 ? 8 : l;
+}
+
+static inline int choose_tpr_log2(int64_t cols) {
+    return choose_tpr_log2_for((cols + 7) / 8, PQ_CHUNKS_PER_THREAD);
 }
 
 static pq_status_t cuda_status(cudaError_t e) {
@@ -932,6 +1089,33 @@ static void launch_dequant(const Batch& b, cudaStream_t s) {
     const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
     k<<<grid, kThreads, 0, s>>>(b);
     pqc::count_launch();
+}
+
+template <int Q>
+static cudaError_t launch_dequant_bulk(const Batch& b, cudaStream_t s) {
+    static int cache[64] = {0};
+    static bool attr_set[64] = {false};
+    auto k = dequant_bulk_kernel<Q>;
+    constexpr int smem = 2 * kDeqBuf;
+    const int dev = current_device();
+    if (!attr_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    if (cache[dev] == 0) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem) !=
+                cudaSuccess || per_sm <= 0)
+            per_sm = 1;
+        cache[dev] = per_sm * sm_count();
+    }
+    const int64_t ctas = cache[dev];
+    const unsigned grid = static_cast<unsigned>(b.total_units < ctas ? b.total_units : ctas);
+    k<<<grid, kThreads, smem, s>>>(b);
+    pqc::count_launch();
+    return cudaSuccess;
 }
 
 // ------------------------------------------------------- validation
@@ -1029,7 +1213,7 @@ static pq_status_t fwd_batch_impl(int q, int32_t n, const pq_matrix_t* mats, cud
             if (m.rows == 0 || m.cols == 0) continue;
             const int k = (m.wq_bf16_out && m.packed_out) ? 0 : (m.wq_bf16_out ? 1 : 2);
             if (k != kind || fwd_vec_ok(m, bits) != vec) continue;
-            const int tl = choose_tpr_log2(m.cols);
+            const int tl = choose_tpr_log2_for((m.cols + 7) / 8, PQ_FWD_CHUNKS_PER_THREAD);
             const int64_t tpr = int64_t{1} << tl;
             const int64_t rpb = kThreads >> tl;
             const int64_t row_blocks = (m.rows + rpb - 1) / rpb;
@@ -1101,15 +1285,24 @@ static pq_status_t dequant_batch_impl(int q, int32_t n, const pq_matrix_t* mats,
     }
     static thread_local Batch b;
     bool launched = false;
-    for (int cls = 0; cls < 2; ++cls) {
-        const bool vec = cls == 0;
+    cudaError_t err = cudaSuccess;
+    // classes: 0 staged bulk stores (vector layout, a row block's output fits
+    // one staging buffer), 1 vector layout, 2 element path
+    for (int cls = 0; cls < 3; ++cls) {
+        if (cls == 0 && !PQ_DEQ_BULK) continue;
         batch_reset(b);
         auto flush = [&]() {
             if (b.n == 0) return;
             launched = true;
             dispatch_q(q, [&]<int Q>() {
-                if (vec) launch_dequant<Q, true>(b, s);
-                else launch_dequant<Q, false>(b, s);
+                if (cls == 0) {
+                    const cudaError_t e = launch_dequant_bulk<Q>(b, s);
+                    if (e != cudaSuccess) err = e;
+                } else if (cls == 1) {
+                    launch_dequant<Q, true>(b, s);
+                } else {
+                    launch_dequant<Q, false>(b, s);
+                }
             });
             batch_reset(b);
         };
@@ -1118,12 +1311,16 @@ static pq_status_t dequant_batch_impl(int q, int32_t n, const pq_matrix_t* mats,
             if (m.rows == 0 || m.cols == 0) continue;
             const bool v = m.cols % 8 == 0 && aligned(m.packed_out, bits == 2 ? 2 : 4) &&
                            aligned(m.wq_bf16_out, 16);
-            if (v != vec) continue;
+            const int bulk_tl = choose_tpr_log2_for((m.cols + 7) / 8, kDeqChunks);
+            const bool bulk = PQ_DEQ_BULK && v && (int64_t{kDeqChunks} << bulk_tl) * 8 >= m.cols;
+            const int c = bulk ? 0 : (v ? 1 : 2);
+            if (c != cls) continue;
             if (b.n == kMaxBatch) flush();
-            batch_add(b, m, choose_tpr_log2(m.cols), 1);
+            batch_add(b, m, cls == 0 ? bulk_tl : choose_tpr_log2(m.cols), 1);
         }
         flush();
     }
+    if (err != cudaSuccess) return cuda_status(err);
     return launched ? cuda_status(cudaGetLastError()) : PQ_OK;
 }
 

@@ -84,6 +84,11 @@ class PQGemmProblem(ctypes.Structure):
                 ("alpha", ctypes.c_void_p), ("y_bf16", ctypes.c_void_p)]
 
 
+class PQIpcHandle(ctypes.Structure):
+    """``pq_ipc_handle_t``: a CUDA IPC handle of one device allocation."""
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
 def _declare(L):
     i64, p, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.pq_fakequant_fwd_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
@@ -111,6 +116,12 @@ def _declare(L):
     L.pq_device_status.restype = i32
     L.pq_launch_count.argtypes = []
     L.pq_launch_count.restype = i64
+    L.pq_ipc_export.argtypes = [p, ctypes.POINTER(PQIpcHandle), ctypes.POINTER(ctypes.c_int64)]
+    L.pq_ipc_export.restype = i32
+    L.pq_ipc_open.argtypes = [ctypes.POINTER(PQIpcHandle), ctypes.POINTER(ctypes.c_void_p)]
+    L.pq_ipc_open.restype = i32
+    L.pq_ipc_close.argtypes = [p]
+    L.pq_ipc_close.restype = i32
     L.pq_debug_abort_waits.argtypes = [i32]
     L.pq_debug_abort_waits.restype = i32
     L.pq_dequant_codes_batch.argtypes = [i32, i32, ctypes.POINTER(PQMatrix), p]
@@ -399,6 +410,30 @@ def pq_wq_gemm_noalloc(q, x, packed, alpha, y_out, stream=None):
 def pq_device_status() -> int:
     """PQ_OK, or PQ_ERR_TIMEOUT once after a bounded device wait gave up."""
     return int(lib().pq_device_status())
+
+
+def ipc_export(t):
+    """(handle bytes, byte offset) of the device allocation holding the
+    contiguous CUDA tensor ``t`` (pq_ipc_export)."""
+    h = PQIpcHandle()
+    off = ctypes.c_int64()
+    _check("pq_ipc_export", lib().pq_ipc_export(_ptr(t), ctypes.byref(h), ctypes.byref(off)))
+    return bytes(h.bytes), int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Maps another process's exported allocation; returns its base address
+    in this process (pq_ipc_open)."""
+    h = PQIpcHandle()
+    ctypes.memmove(h.bytes, handle, 64)
+    base = ctypes.c_void_p()
+    _check("pq_ipc_open", lib().pq_ipc_open(ctypes.byref(h), ctypes.byref(base)))
+    return int(base.value)
+
+
+def ipc_close(base: int) -> None:
+    """Unmaps a base returned by ``ipc_open`` (pq_ipc_close)."""
+    _check("pq_ipc_close", lib().pq_ipc_close(base))
 
 
 def pq_launch_count() -> int:

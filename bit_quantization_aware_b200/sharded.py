@@ -21,10 +21,19 @@ step, per GPU:
    the STE backward, d(alpha) and AdamW to them, in one kernel
    (the reduce-scatter is fused into the backward).
 
-Peer buffers come from a provider: ``SymmetricPeers`` (torch symmetric
-memory across processes, one GPU each) or ``LocalPeers`` (several buffer
-sets on one GPU standing in for GPUs, for tests). The arithmetic runs in the
-CUDA library (``pq``); this module only lays out buffers and descriptors.
+Ordering: ``forward`` and ``backward`` put the caller's barrier between the
+phases (pack -> barrier -> gather; the model writes the gradient ->
+barrier -> reduce). Two barriers per step suffice when the barrier is a
+stream-ordered collective (or a device synchronise plus a host barrier):
+a rank passes the forward barrier of step t+1 only after every rank's
+reduce of step t is done, and the backward barrier only after every
+rank's gather is done, so no phase overwrites a buffer a peer still reads.
+
+Peer buffers come from a provider: ``IpcPeers`` (CUDA IPC across
+processes, one GPU each; point-to-point mappings, no multicast object) or
+``LocalPeers`` (several buffer sets on one GPU standing in for GPUs, for
+tests). The arithmetic runs in the CUDA library (``pq``); this module only
+lays out buffers and descriptors.
 """
 from __future__ import annotations
 
@@ -102,43 +111,94 @@ class LocalPeers:
         return self.bufs[rank][name]
 
 
-class SymmetricPeers:
-    """Peer buffers in torch symmetric memory: every rank allocates the same
-    buffer and reads the others' through peer mappings (one process per
-    GPU; NVLink / NVSwitch)."""
+class PeerSpan:
+    """A contiguous 1-D range of another process's device memory, mapped by
+    CUDA IPC, typed like a tensor of ``dtype``. Slicing gives a sub-range;
+    the library's kernels take it wherever they take a device tensor. It is
+    never a torch tensor, so nothing reads or copies it on the host."""
 
-    def __init__(self, group):
+    is_cuda = True
+
+    def __init__(self, ptr: int, numel: int, dtype):
+        self.ptr, self.n, self.dtype = int(ptr), int(numel), dtype
+        self.itemsize = torch.empty((), dtype=dtype).element_size()
+
+    def data_ptr(self) -> int:
+        return self.ptr
+
+    def numel(self) -> int:
+        return self.n
+
+    def is_contiguous(self) -> bool:
+        return True
+
+    def __getitem__(self, s):
+        if not isinstance(s, slice) or s.step not in (None, 1):
+            raise TypeError("a peer range takes contiguous slices only")
+        b, e, _ = s.indices(self.n)
+        return PeerSpan(self.ptr + b * self.itemsize, max(0, e - b), self.dtype)
+
+
+class IpcPeers:
+    """Peer buffers for one process per GPU, shared by CUDA IPC: each rank
+    allocates its buffer as an ordinary device tensor, the ranks exchange
+    the IPC handle of the allocation holding it and the buffer's offset (an
+    all-gather of small host objects over the process group), and every
+    rank maps the others' allocations with ``pq.ipc_open`` (once per
+    allocation). These are point-to-point peer mappings over NVLink: no
+    NVLink multicast object is created, so no rank's memory is bound to one.
+
+    Lifetime: a rank's tensors must outlive every other rank's reads. Call
+    ``close`` on every rank after the last kernel that reads a peer buffer
+    has completed on every rank (synchronise, then a barrier); it unmaps the
+    peers' allocations. Only then may the owners free their tensors."""
+
+    def __init__(self, group=None):
         import torch.distributed as dist
-        import torch.distributed._symmetric_memory as symm_mem
-        self.symm_mem = symm_mem
+        self.dist = dist
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
-        self.handles = {}
         self.local = {}
+        self.views = {}
+        self.mapped = {}  # handle bytes -> base address in this process
 
     def allocate(self, rank, name, numel, dtype, device):
         assert rank == self.rank
-        t = self.symm_mem.empty(numel, dtype=dtype, device=device)
-        t.zero_()
-        self.handles[name] = self.symm_mem.rendezvous(t, self.group.group_name)
+        t = torch.zeros(numel, dtype=dtype, device=device)
+        handle, offset = pq.ipc_export(t)
+        info = [None] * self.world
+        self.dist.all_gather_object(info, (handle, offset, numel), group=self.group)
+        views = []
+        for k, (h, off, n) in enumerate(info):
+            if k == self.rank:
+                views.append(t)
+                continue
+            if h not in self.mapped:
+                self.mapped[h] = pq.ipc_open(h)
+            views.append(PeerSpan(self.mapped[h] + off, n, dtype))
         self.local[name] = t
+        self.views[name] = views
         return t
 
     def get(self, rank, name):
-        if rank == self.rank:
-            return self.local[name]
-        t = self.local[name]
-        return self.handles[name].get_buffer(rank, (t.numel(),), t.dtype, 0)
+        return self.views[name][rank]
+
+    def close(self):
+        for base in self.mapped.values():
+            pq.ipc_close(base)
+        self.mapped.clear()
+        self.views.clear()
 
 
 class ShardedQuantStep:
     """One GPU's part of the row-sharded quantizer step over ``mats``."""
 
-    def __init__(self, mats, q: int, rank: int, world: int, peers, device="cuda"):
+    def __init__(self, mats, q: int, rank: int, world: int, peers, device="cuda", lib=pq):
         self.q, self.rank, self.world, self.peers = q, rank, world, peers
+        self.lib = lib  # the library binding (a stand-in in host-only tests)
         self.device = torch.device(device)
-        self.bits = pq.pq_code_bits(q)
+        self.bits = lib.pq_code_bits(q)
         self.layout = Layout(tuple(mats), world, rank, self.bits)
         self.mats = list(mats)
         full, (ne, nr, npk) = self.layout.full_offsets()
@@ -196,7 +256,7 @@ class ShardedQuantStep:
             descs.append(dict(rows=e - b, cols=m.cols, w=self.w_shard(i),
                               alpha=self.alpha_rows(i, b, e),
                               packed=self.packed_full[p0:p0 + (e - b) * m.cols * self.bits // 8]))
-        pq.pq_fakequant_fwd_batch(self.q, pq.matrix_array(descs), stream)
+        self.lib.pq_fakequant_fwd_batch(self.q, self.lib.matrix_array(descs), stream)
 
     def gather_dequant(self, stream=None):
         descs = []
@@ -211,8 +271,7 @@ class ShardedQuantStep:
                                   packed=pk[pb:pb + (e - b) * m.cols * self.bits // 8],
                                   alpha=self.alpha_rows(i, b, e, rank=k),
                                   wq=self.wq_full[e0 + b * m.cols:e0 + e * m.cols]))
-        for s in range(0, len(descs), 256):
-            pq.pq_dequant_codes_batch(self.q, pq.matrix_array(descs[s:s + 256]), stream)
+        self.lib.pq_dequant_codes_batch(self.q, self.lib.matrix_array(descs), stream)
 
     def reduce_step(self, hp_w, hp_alpha, grad_mult=None, stream=None):
         sources = [self.peers.get(k, "g") for k in range(self.world)]
@@ -229,7 +288,24 @@ class ShardedQuantStep:
                                m_w=self.m_w[s0:s0 + n], v_w=self.v_w[s0:s0 + n],
                                m_alpha=self.m_a[r0 + b:r0 + e], v_alpha=self.v_a[r0 + b:r0 + e],
                                dalpha=self.dalpha[r0 + b:r0 + e], g_offset=e0 + b * m.cols,
-                               grad_scale=pq.pq_default_grad_scale(self.q, m.cols)))
+                               grad_scale=self.lib.pq_default_grad_scale(self.q, m.cols)))
         mult = 1.0 / self.world if grad_mult is None else grad_mult
-        pq.pq_reduce_bwd_adamw(self.q, sources, mult, pq.shard_array(shards), hp_w, hp_alpha,
-                               stream)
+        self.lib.pq_reduce_bwd_adamw(self.q, sources, mult, self.lib.shard_array(shards), hp_w,
+                                     hp_alpha, stream)
+
+    # ---------------------------------------------------------- one step
+    def forward(self, barrier, stream=None):
+        """Forward of one step: pack the owned rows, wait at ``barrier``
+        until every rank's codes are written, then gather + dequantize all
+        rows into this rank's bf16 weights."""
+        self.pack_shards(stream)
+        barrier()
+        self.gather_dequant(stream)
+
+    def backward(self, barrier, hp_w, hp_alpha, grad_mult=None, stream=None):
+        """Backward of one step, after the model wrote this rank's full
+        upstream gradient into ``g``: wait at ``barrier`` until every
+        rank's gradient is written, then reduce + backward + AdamW on the
+        owned shards."""
+        barrier()
+        self.reduce_step(hp_w, hp_alpha, grad_mult, stream)

@@ -248,7 +248,7 @@ typedef struct {
  * upstream gradient of each element is the fp32 sum, in source order, of
  * the bf16 gradients g_sources[0..n_src) (one per data-parallel replica,
  * all with the same layout; device pointers, local or another GPU's
- * memory reachable by peer access, e.g. symmetric memory), times
+ * memory reachable by peer access, e.g. mapped with pq_ipc_open), times
  * grad_mult (1/n_src for a mean); then the steps of
  * pq_fakequant_bwd_adamw run with that fp32 gradient. Each GPU calls this
  * on its own shards after every replica's gradient is complete (the
@@ -262,6 +262,35 @@ PQ_API pq_status_t pq_reduce_bwd_adamw(pq_quant_t q, int32_t n_src,
                                        const pq_shard_t* shards,
                                        const pq_adamw_t* hp_w,
                                        const pq_adamw_t* hp_alpha, void* stream);
+
+/* Peer-readable buffers across processes (the row-sharded step's plumbing;
+ * no counterpart in the pages, which leave multi-GPU layout to the training
+ * framework). A CUDA IPC handle of the device allocation that holds a
+ * buffer; another process maps that allocation with pq_ipc_open and reads
+ * the buffer at the exported offset from the mapped base. The mappings are
+ * point-to-point peer mappings (peer access is enabled on first use): no
+ * NVLink multicast object is created or bound.
+ *   pq_ipc_export: dev_ptr is any address inside a cudaMalloc'd allocation
+ *     of the current device (e.g. a tensor of a caching allocator; memory
+ *     from virtual-memory or async pools is rejected with PQ_ERR_CUDA);
+ *     handle_out receives the allocation's handle, offset_out the byte
+ *     offset of dev_ptr from the allocation's base. Several buffers of one
+ *     allocation share a handle: map it once per process.
+ *   pq_ipc_open: maps an exported allocation into this process (current
+ *     device) and returns its base; the owner must keep the allocation
+ *     alive until every mapping is closed. Opening a handle exported by
+ *     this same process fails (PQ_ERR_CUDA).
+ *   pq_ipc_close: unmaps a base returned by pq_ipc_open, after this
+ *     process's last kernel reading it has completed.
+ * Host calls; nothing is enqueued and nothing is allocated. */
+typedef struct {
+    unsigned char bytes[64];
+} pq_ipc_handle_t;
+
+PQ_API pq_status_t pq_ipc_export(const void* dev_ptr, pq_ipc_handle_t* handle_out,
+                                 int64_t* offset_out);
+PQ_API pq_status_t pq_ipc_open(const pq_ipc_handle_t* handle, void** base_out);
+PQ_API pq_status_t pq_ipc_close(void* base);
 
 /* Dequantize packed codes back to bf16 weights: each stored code c (layout
  * of packed_out above) becomes bf16_rn(fl(level(c) * alpha_row)) with the

@@ -35,7 +35,8 @@ def test_header_declares_entry_points():
               "pq_wq_gemm", "pq_wq_gemm_workspace_bytes", "pq_device_status",
               "pq_wq_gemm_noalloc", "pq_wq_gemm_batch", "pq_wq_gemm_batch_workspace_bytes", "pq_debug_abort_waits",
               "pq_status_string", "pq_default_grad_scale", "pq_code_bits",
-              "pq_last_cuda_error", "pq_launch_count"):
+              "pq_last_cuda_error", "pq_launch_count", "pq_ipc_export", "pq_ipc_open",
+              "pq_ipc_close"):
         assert n in names
 
 
