@@ -352,18 +352,21 @@ def run_reference(args):
 
 # ----------------------------------------------------------- timing helpers
 class L2Flush:
-    """Writes a buffer of twice the L2 size, so that the next kernel finds
-    none of its inputs in L2 (a real step runs a matmul between the
-    quantizer's phases)."""
+    """Reads a buffer of twice the L2 size (a sum), so that the next kernel
+    finds none of its inputs in L2 (a real step runs a matmul between the
+    quantizer's phases). A read leaves only clean lines behind: a written
+    flush buffer would leave up to an L2 of dirty lines whose write-back
+    lands in the next kernel's time (for a 268 MB phase, up to half again
+    its own traffic)."""
 
     def __init__(self, device):
         import torch
-        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
-        self.k = 0
+        self.buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+        self.out = torch.empty((), dtype=torch.float32, device=device)
 
     def __call__(self):
-        self.k += 1
-        self.buf.fill_(self.k)
+        import torch
+        torch.sum(self.buf, dim=0, out=self.out)
 
 
 def timed_phases(fns, steps, warmup, flush):
@@ -497,7 +500,7 @@ def measure_case(case, steps, warmup, peak, device, flush, oracle_seconds):
     from bit_quantization_aware_b200 import pq
     from bit_quantization_aware_b200.step import QuantStep
     out = {"what": case["what"], "weights": I.total_weights(case["mats"]),
-           "l2_flush": "before every phase (a buffer of twice the L2 size is written)"}
+           "l2_flush": "before every phase (a buffer of twice the L2 size is read)"}
     for name, q, rule in case["quantizers"]:
         step = QuantStep(case["mats"], q, device=device, pack=case["pack"])
         step.generate(seed=case["seed"], dist=case["dist"], lsq_rule=rule)
