@@ -895,10 +895,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(args.warmup, 0)):
-        step.run()
-    torch.cuda.synchronize()
-
     n_b = step.launches_per_step // 2  # backward launches per step
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
@@ -908,6 +904,11 @@ def run_ours(args):
     sampler = ClockSampler(physical_gpu_index(local))
     sampler.start()
     time.sleep(0.3)
+    # warm-up right before the timed region: after an idle gap the first
+    # few launches run slower while the clocks come back up
+    for _ in range(max(args.warmup, 0)):
+        step.run()
+    torch.cuda.synchronize()
 
     barrier()
     torch.cuda.synchronize()
