@@ -426,7 +426,11 @@ def _dequant_gpu(q, packed_np, alpha_np, cols, offset=0):
 @pytest.mark.parametrize("q", ALLQ)
 @pytest.mark.parametrize("shape,offset", [((1, 32), 0), ((3, 96), 0), ((5, 12), 0),
                                           ((7, 1000), 0), ((33, 1032), 0), ((64, 4096), 0),
-                                          ((9, 4096), 1), ((2, 70000), 0)])
+                                          ((9, 4096), 1), ((2, 70000), 0),
+                                          # staged bulk stores: the widest row a staging
+                                          # buffer holds, one row more (direct stores), and
+                                          # many units per CTA (both buffers reused)
+                                          ((3, 16384), 0), ((2, 16392), 0), ((20000, 1024), 0)])
 def test_dequant_matches_oracle(q, shape, offset):
     """Packed codes -> bf16: every element equals the oracle's decoding
     (random bytes, so every code value of the format appears)."""
