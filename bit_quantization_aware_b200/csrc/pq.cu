@@ -52,7 +52,9 @@
 //                    3 evict-first with a 256-byte L2 prefetch, 4 read-only
 //                    without L1 allocation with a 256-byte L2 prefetch)
 //   PQ_BWD_MIN_CTAS  resident CTAs per SM the backward's registers must allow
-//   PQ_FWD_MIN_CTAS  the same for the forward (0: no register cap)
+//   PQ_FWD_MIN_CTAS  the same for the forward (PQ_PACK_MIN_CTAS: its
+//                    packed-codes-only instance; PQ_RED_MIN_CTAS: the
+//                    sharded reduce + backward + AdamW)
 //   PQ_DEQ_BULK      1: the dequantization stages each unit's bf16 output in
 //                    shared memory and writes it with one bulk copy
 //   PQ_DEQ_BUF_KB    size of one such staging buffer (two per CTA)
@@ -72,7 +74,7 @@
 #define PQ_FWD_UNROLL 3
 #endif
 #ifndef PQ_PACK_UNROLL
-#define PQ_PACK_UNROLL 2
+#define PQ_PACK_UNROLL 4
 #endif
 #ifndef PQ_BWD_UNROLL
 #define PQ_BWD_UNROLL 2
@@ -95,10 +97,11 @@
 #ifndef PQ_DEQ_BUF_KB
 #define PQ_DEQ_BUF_KB 32
 #endif
-#if PQ_FWD_MIN_CTAS > 0
-#define PQ_FWD_BOUNDS __launch_bounds__(kThreads, PQ_FWD_MIN_CTAS)
-#else
-#define PQ_FWD_BOUNDS __launch_bounds__(kThreads)
+#ifndef PQ_PACK_MIN_CTAS
+#define PQ_PACK_MIN_CTAS 3
+#endif
+#ifndef PQ_RED_MIN_CTAS
+#define PQ_RED_MIN_CTAS 3
 #endif
 
 std::atomic<int64_t> pqc::launches{0};
@@ -379,7 +382,7 @@ __device__ __forceinline__ void prefetch_unit(const MatBatch<CAP>& p, int mi, in
 
 // ------------------------------------------------------------------ forward
 template <int Q, bool VEC, bool WQ, bool PACK, int CAP>
-__global__ void PQ_FWD_BOUNDS
+__global__ void __launch_bounds__(kThreads, WQ ? PQ_FWD_MIN_CTAS : PQ_PACK_MIN_CTAS)
 fwd_units_kernel(const __grid_constant__ MatBatch<CAP> p) {
     int mi = 0;
     for (int64_t u = blockIdx.x; u < p.total_units; u += gridDim.x) {
@@ -897,7 +900,7 @@ struct ReduceBatch {
 };
 
 template <int Q, bool VEC>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, PQ_RED_MIN_CTAS)
 reduce_bwd_adamw_units_kernel(const __grid_constant__ ReduceBatch P) {
     const BatchT<ShardDesc>& p = P.b;
     __shared__ double warp_sum[2][kThreads / 32];
