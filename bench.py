@@ -50,6 +50,7 @@ WORKLOAD = "llama3_8b_linear_set_seq2_fwd_ste_bwd"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the roofline uses the measured copy peak)
 MAX_SHARDED_WORLD = 16  # gradient sources one reduce launch accepts
 
 
@@ -950,17 +951,21 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": bwd_bytes_step / n_b,
                 "avg_launch_us": bwd_s_step / n_b * 1e6,
                 "fwd_bwd_frac_of_peak": (step.bytes_fwd() + bwd_bytes_step)
-                / (ms_step * 1e-3) / 1e9 / peak}
+                / (ms_step * 1e-3) / 1e9 / peak,
+                "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                "traffic_frac_of_peak": (None if traffic is None
+                                         else traffic / bwd_s_step * n_b / 1e9 / peak)}
 
     def phase(ms_per_step, nbytes):
         sec = ms_per_step * 1e-3
         return {"ms_per_step": ms_per_step, "Gweights_s": step_throughput(weights, world, ms_per_step),
                 "GB_s": nbytes / sec / 1e9, "frac_of_peak": nbytes / sec / 1e9 / peak,
+                "frac_of_nominal": nbytes / sec / 1e9 / NOMINAL_HBM_GBS,
                 "algorithmic_bytes": nbytes}
     phases = {"fwd": phase(fwd_ms / args.steps, step.bytes_fwd()),
               "bwd": phase(bwd_ms / args.steps, bwd_bytes_step),
               "fwd_bwd": phase(ms_step, step.bytes_fwd() + bwd_bytes_step),
-              "peak_GB_s": peak}
+              "peak_GB_s": peak, "nominal_GB_s": NOMINAL_HBM_GBS}
 
     e2e = None
     if not args.no_e2e:
