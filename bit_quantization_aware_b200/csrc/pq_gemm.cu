@@ -45,9 +45,11 @@
 // (deterministic).
 //
 // Roles (19 warps): 8 decode warps (TMEM lane quarter = warp % 4, K half =
-// warp / 4), 4 epilogue warps, 4 activation permuters (in the integer mode
-// the planes arrive already in MMA order and they only pass the stage on),
-// one codes producer, one activation producer, one MMA issuer. The
+// warp / 4), 4 epilogue warps, 4 activation permuters (bf16 mode only: in
+// the integer mode the planes arrive already in MMA order, and decode warp 0
+// holds each stage until its activations have landed; a permuter pass there
+// measured 7% slower), one codes producer, one activation producer, one MMA
+// issuer. The
 // activation ring is deeper than the A ring and has its own barriers, so
 // decoding never waits on it. Every mbarrier wait is bounded: on giving up the kernel
 // records a device status and an abort flag that ends every role's loop,
@@ -501,7 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < SB; ++s) mbar_init(b_xfull + 8u * s, 1);
         for (int s = 0; s < SA; ++s) {
-            mbar_init(b_afull + 8u * s, kDecWarps + kPermWarps);
+            // integer mode: the decoders alone (warp 0 also waits for the
+            // stage's activations); bf16: decoders and permuters
+            mbar_init(b_afull + 8u * s, I8 ? kDecWarps : kDecWarps + kPermWarps);
             mbar_init(b_aempty + 8u * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -654,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         Ring<SC> cr;
         Ring<SA> ar;
+        Ring<SB> xbr;  // integer mode: the activation ring, followed by warp 0
         int64_t s = rs;
         Piece pc;
         int cur = 0;
@@ -736,6 +741,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                     }
                     __syncwarp();
+                    if constexpr (I8) {
+                        // the planes arrive in MMA order: no permuter pass, so
+                        // warp 0 holds the stage until its activations landed
+                        if (warp == 0 && !warp_wait(b_xfull + 8u * xbr.idx, xbr.phase, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        xbr.next();
+                    }
                     if (lane == 0) mbar_arrive(b_afull + 8u * ar.idx);
                     ar.next();
                 }
@@ -744,8 +758,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cr.next();
             }
         }
-    } else if (warp >= kPermWarp0 && warp < kPermWarp0 + kPermWarps) {
+    } else if (!I8 && warp >= kPermWarp0 && warp < kPermWarp0 + kPermWarps) {
         // ------------------- activation permuters: each group of 16 K -> (j, j + 8)
+        // (bf16 mode only: the integer mode's digit planes arrive in MMA order)
         const int ptid = tid - kPermWarp0 * 32;
         Ring<SB> br;
         Ring<SA> ar;
