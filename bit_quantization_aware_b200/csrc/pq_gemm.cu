@@ -823,9 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!*epi_ok) break;
             tc_fence_after();
             const uint32_t d = tmem + lane_addr + L::kAccStride * ab;
-            // pass 1: Sx (TMEM lane 127) to shared memory
+            // pass 1: Sx (TMEM lane 127) to shared memory, read by the one
+            // warp whose lanes hold it
 #pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) {
+                if (e != kFeat / 32) break;
                 float v[16];
                 __syncwarp();
                 tmem_ld16(d + c0, v);
