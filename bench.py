@@ -463,27 +463,26 @@ def per_config_cases():
     """The four workloads besides the headline, with the seeds, draws and
     scale initialisations of their parity tests (seed = workload number - 1)."""
     from bit_quantization_aware_b200 import inputs as I
-    Q = I
     return [
         dict(key="1_single_256x1024_pack", mats=[I.Matrix("w", 256, 1024, 0, 0)],
-             quantizers=[("seq2", Q.SEQ2, "lsq"), ("seq2_b", Q.SEQ2_B, "lsq")],
+             quantizers=[("seq2", I.SEQ2, "lsq"), ("seq2_b", I.SEQ2_B, "lsq")],
              pack=True, dist="normal", seed=0, plant=False, standalone_pack=False,
              what="one 256x1024 N(0,0.02) weight, alpha = max|w_row|, forward with packed "
                   "codes + backward; launch-bound and L2-resident (a parity case)"),
         dict(key="2_bit_width_sweep_2048x8192", mats=[I.Matrix("w", 2048, 8192, 0, 0)],
-             quantizers=[("binary", Q.BINARY, "lsq"), ("ternary", Q.TERNARY, "lsq"),
-                         ("seq2", Q.SEQ2, "lsq"), ("lsq3", Q.LSQ3, "lsq"),
-                         ("lsq4", Q.LSQ4, "lsq")],
+             quantizers=[("binary", I.BINARY, "lsq"), ("ternary", I.TERNARY, "lsq"),
+                         ("seq2", I.SEQ2, "lsq"), ("lsq3", I.LSQ3, "lsq"),
+                         ("lsq4", I.LSQ4, "lsq")],
              pack=False, dist="normal", seed=1, plant=False, standalone_pack=False,
              what="one 2048x8192 N(0,0.02) weight; alpha = mean|w_row| (binary), "
                   "max|w_row| (ternary, seq2), 2 mean|w_row|/sqrt(Qp) (lsq3, lsq4)"),
         dict(key="3_llama_1b_stack", mats=I.llama_1b_stack(),
-             quantizers=[("seq2", Q.SEQ2, "lsq")],
+             quantizers=[("seq2", I.SEQ2, "lsq")],
              pack=False, dist="normal", seed=2, plant=False, standalone_pack=False,
              what="24 layers: q,o 2048x2048; k,v 512x2048; gate,up 5632x2048; "
                   "down 2048x5632; one batched launch per phase"),
         dict(key="5_student_t_16384_planted_pack", mats=[I.Matrix("t3.16384", 16384, 16384, 0, 0)],
-             quantizers=[("seq2", Q.SEQ2, "lsq"), ("ternary", Q.TERNARY, "lsq")],
+             quantizers=[("seq2", I.SEQ2, "lsq"), ("ternary", I.TERNARY, "lsq")],
              pack=True, dist="student_t", seed=4, plant=True, standalone_pack=True,
              what="one 16384x16384 Student-t(3)*0.02 weight, 1% of entries planted on "
                   "clip bounds and rounding ties; forward with fused packed codes + "
@@ -512,11 +511,11 @@ def measure_case(case, steps, warmup, peak, device, flush, oracle_seconds):
             planted = {"entries": n, "exactly_on_target": hit}
         fns = {"fwd": step.fwd_all, "bwd": step.bwd_all}
         if case["standalone_pack"]:  # one matrix: pq_pack_codes into its own buffer
-            b = step.bufs[0]
-            pk_alone = torch.empty_like(b.packed)
-            fns["pack_standalone"] = lambda: pq.pq_pack_codes(step.q, b.w, b.alpha, pk_alone)
+            b0 = step.bufs[0]
+            pk_alone = torch.empty_like(b0.packed)
+            fns["pack_standalone"] = lambda: pq.pq_pack_codes(step.q, b0.w, b0.alpha, pk_alone)
         med, per, launches = timed_phases(fns, steps, warmup, flush)
-        fb = statistics.median([a + b for a, b in zip(per["fwd"], per["bwd"])])
+        fb = statistics.median([f + g for f, g in zip(per["fwd"], per["bwd"])])
         w = step.weights
         entry = {"fwd": phase_entry(med["fwd"], w, step.bytes_fwd(), peak),
                  "bwd": phase_entry(med["bwd"], w, step.bytes_bwd(), peak),
@@ -529,7 +528,12 @@ def measure_case(case, steps, warmup, peak, device, flush, oracle_seconds):
             entry["pack_standalone"] = phase_entry(med["pack_standalone"], w, nb, peak)
         if planted:
             entry["planted"] = planted
+        # free this quantizer's buffers before the next one allocates
         del step, fns
+        if case["standalone_pack"]:
+            del b0, pk_alone
+        if case["plant"]:
+            del b
         torch.cuda.empty_cache()
         if oracle_seconds > 0:
             sample = oracle_sample(case["mats"], q, oracle_seconds, seed=case["seed"],
