@@ -655,15 +655,23 @@ def measure_bwd_adamw(step, steps, warmup, peak):
 
 def wq_gemm_kernel_name(m, gsize, max_k):
     """The kernel a grouped launch of ``gsize`` matrices with ``m`` activation
-    rows runs: one row times a lone matrix (k <= 32768) takes the CUDA-core
-    kernel, 1..16 rows otherwise the integer tensor-core mode (after its
-    activation digit-plane pre-pass), more rows the bf16 tensor-core mode."""
+    rows runs, and its arithmetic: one row times a lone matrix (k <= 32768)
+    takes the CUDA-core kernel; 1..16 rows otherwise the exact fixed-point
+    mode after its activation digit-plane pre-pass, on packed fp4 MMAs while
+    every k <= 2^20 and on 8-bit MMAs beyond; more rows the bf16 mode."""
     if m == 1 and gsize == 1 and max_k <= 32768:
-        return "pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)", False
+        return "pqg::pqv::gemv_kernel<MAXP> (CUDA cores, paired fp32 FMA)", "bf16 x 2-bit codes, f32 FMA"
+    if m <= 16 and max_k <= (1 << 20):
+        return ("pqg::wq_gemm_kernel<NT, MAXP, kModeF4> (tcgen05.mma kind::mxf4 block-scaled, unit scales, "
+                "TMEM accumulator) after pqg::xplanes_kernel<true>",
+                "e2m1 base-9 digit planes of bf16 activations x e2m1 f'/2 code nibbles, "
+                "f32 accumulate (exact integers)")
     if m <= 16:
-        return ("pqg::wq_gemm_kernel<NT, MAXP, true> (tcgen05.mma kind::i8, TMEM accumulator)"
-                " after pqg::xplanes_kernel"), True
-    return "pqg::wq_gemm_kernel<NT, MAXP, false> (tcgen05.mma kind::f16, TMEM accumulator)", False
+        return ("pqg::wq_gemm_kernel<NT, MAXP, kModeI8> (tcgen05.mma kind::i8, TMEM accumulator)"
+                " after pqg::xplanes_kernel<false>",
+                "s8 digit planes of bf16 activations x u8 2-bit code fields, s32 accumulate")
+    return ("pqg::wq_gemm_kernel<NT, MAXP, kModeBF16> (tcgen05.mma kind::f16, TMEM accumulator)",
+            "bf16 x 2-bit codes, f32 accumulate")
 
 
 def measure_wq_gemm(bufs, packed, q, m, steps, warmup, device, with_single=False):
@@ -735,13 +743,11 @@ def measure_wq_gemm(bufs, packed, q, m, steps, warmup, device, with_single=False
                 "unit": "TFLOP/s", "peak_source": f"{tf_kind} bf16_tflops (burst)",
                 "algorithmic_flops": flops}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"], integer_mode = wq_gemm_kernel_name(m, gsize, max(ks))
+    roof["kernel"], arith = wq_gemm_kernel_name(m, gsize, max(ks))
     res.update({"m": m, "ms": ms, "Gweights_s": weights / (ms * 1e-3) / 1e9,
                 "tflops": flops / (ms * 1e-3) / 1e12, "launches_per_step": launches,
                 "grouped_launches": len(groups), "matrices_per_launch": gsize,
-                "dtype": ("s8 digit planes of bf16 activations x u8 2-bit code fields, "
-                          "s32 accumulate" if integer_mode else
-                          "bf16 x 2-bit codes, f32 accumulate"),
+                "dtype": arith,
                 "roofline": roof,
                 "cublas_bf16_dense": {"ms": ms_dense, "speedup_of_ours": ms_dense / ms,
                                       "what": "torch.matmul(x, W_bf16.t()) per matrix, CUDA graph",

@@ -32,6 +32,21 @@
 // fields (s, s + 4, s + 8, s + 12), so the K order inside every group of 16
 // is a 4 x 4 transpose, which the pre-pass applies to the planes.
 //
+// Packed-fp4 mode (m <= 16, k <= 2^20). Block-scaled fp4 MMAs
+// (kind::mxf4, every scale 1.0) take K = 64 per instruction at about the cost
+// of a K = 32 8-bit one, so the same exact integer sums run at twice the K
+// per MMA. The weights go in as f'/2 (the e2m1 nibbles 0, 0.5, 1, 1.5 are
+// the field's two bits in the low half of a nibble: one mask and one xor per
+// eight weights), the same fixed-point activations v = rint(x 2^(29 - E)) as
+// ten planes of balanced base-9 digits in [-4, 4] (all exact e2m1 values;
+// |v| < 2^30 < 9^10 / 2). Every product is a multiple of 1/2 and every
+// partial sum stays below 2^23 in magnitude for k <= 2^20, so the fp32
+// accumulators hold exact integers, and the epilogue forms
+// sum_k v f' = sum_p 9^p (2 acc_p) exactly in int64: the result is the
+// integer mode's, bit for bit. The decoded nibbles of a code word are its
+// even fields, then its odd fields, so the K order inside every group of 16
+// is (0, 2, .., 14, 1, 3, .., 15), which the pre-pass applies to the planes.
+//
 // Operands. A (decoded weights) lives in TMEM (tcgen05.st from the decode
 // warps; tcgen05.mma reads it there, with no shared-memory round trip);
 // B (activations) arrives by TMA in the 128B-swizzled K-major layout the
@@ -44,12 +59,12 @@
 // workspace and the last CTA to finish the block adds them in K order
 // (deterministic).
 //
-// Roles (19 warps): 8 decode warps (TMEM lane quarter = warp % 4, K half =
-// warp / 4), 4 epilogue warps, 4 activation permuters (bf16 mode only: in
-// the integer mode the planes arrive already in MMA order, and decode warp 0
-// holds each stage until its activations have landed; a permuter pass there
-// measured 7% slower), one codes producer, one activation producer, one MMA
-// issuer. The
+// Roles (19 warps in the bf16 mode, 15 in the integer and fp4 modes): 8
+// decode warps (TMEM lane quarter = warp % 4, K half = warp / 4), 4 epilogue
+// warps, 4 activation permuters (bf16 mode only: in the fixed-point modes the
+// planes arrive already in MMA order, and decode warp 0 holds each stage
+// until its activations have landed; a permuter pass there measured 7%
+// slower), one codes producer, one activation producer, one MMA issuer. The
 // activation ring is deeper than the A ring and has its own barriers, so
 // decoding never waits on it. Every mbarrier wait is bounded: on giving up the kernel
 // records a device status and an abort flag that ends every role's loop,
@@ -78,13 +93,28 @@ constexpr int kDecWarps = 8;           // warps 0..7
 constexpr int kEpiWarp0 = 8;           // warps 8..11
 constexpr int kPermWarp0 = 12;         // warps 12..15
 constexpr int kPermWarps = 4;
-constexpr int kCodesWarp = 16, kXWarp = 17, kMmaWarp = 18;
-constexpr int kThreads = 19 * 32;
+// The single-thread roles follow the permuters (bf16) or the epilogue
+// (integer and fp4 modes, which have no permuters): 19 or 15 warps, so the
+// fixed-point instances get 128 registers a thread instead of 96.
+template <int MODE>
+struct Roles {
+    static constexpr bool kPerm = MODE == 0;  // kModeBF16
+    static constexpr int kCodesWarp = kPerm ? 16 : 12, kXWarp = kCodesWarp + 1, kMmaWarp = kCodesWarp + 2;
+    static constexpr int kThreads = (kCodesWarp + 3) * 32;
+};
 constexpr uint32_t kTmemCols = 512;
 constexpr int kCodesSlotBytes = 16384;
 constexpr uint32_t kCodesTx = kFeat * 128;
 constexpr uint32_t kMaxSpins = 1u << 22;
 constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
+constexpr uint32_t kOnesF4 = 0x22222222u;  // eight e2m1 1.0
+constexpr uint32_t kScaleOne = 0x7F7F7F7Fu;  // four ue8m0 1.0
+constexpr int kF4Planes = 10;            // base-9 digit planes of 30-bit fixed point
+constexpr int64_t kF4MaxK = int64_t{1} << 20;  // exact fp32 sums up to this k
+
+// Arithmetic of a launch: bf16 (kind::f16, m > 16), integer (kind::i8) or
+// packed fp4 (kind::mxf4) on the same fixed-point activations.
+enum : int { kModeBF16 = 0, kModeI8 = 1, kModeF4 = 2 };
 
 // nonzero after a bounded wait gave up (read by pq_device_status)
 __device__ int g_status = 0;
@@ -149,11 +179,29 @@ __host__ __device__ constexpr uint32_t idesc_i8(int nt) {
            (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
-// D (TMEM) (+)= A (TMEM) * B (shared memory)^T; K = 16 (bf16) or 32 (8-bit)
-template <bool I8>
+// Instruction descriptor, kind::mxf4 with 32-element scale blocks: e2m1 A
+// and B, ue8m0 scales, both K-major, M = 128, N = nt, K = 64.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int nt) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// D (TMEM) (+)= A (TMEM) * B (shared memory)^T; K = 16 (bf16), 32 (8-bit) or
+// 64 (fp4; the A and B scale factors come from TMEM columns sf.. and
+// sf + 8.., all of whose bytes are 1.0: the two block scales of an operand's
+// row r sit in column base + r / 32, lane r % 32 of every lane quarter that
+// reads them, so 32 such columns over all 128 lanes serve N up to 192).
+template <int MODE>
 __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    if (I8)
+                                       uint32_t idesc, uint32_t accumulate, uint32_t sf) {
+    if (MODE == kModeF4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], [%1], %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(tmem_d),
+            "r"(tmem_a), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sf), "r"(sf + 8u)
+            : "memory");
+    else if (MODE == kModeI8)
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
@@ -175,17 +223,17 @@ __device__ __forceinline__ void mma_commit(uint32_t mbar) {
                  : "memory");
 }
 
-// NK MMAs over one stage, each reading 32 bytes of K per row (16 bf16 or
-// 32 8-bit values): A columns advance by 8, the B descriptor start address
-// by 32 B inside a 128-B swizzle atom and by one atom (ATOM_B bytes) every
-// 4 MMAs.
-template <int NK, int ATOM_B, bool I8>
+// NK MMAs over one stage, each reading 32 bytes of K per row (16 bf16,
+// 32 8-bit or 64 fp4 values): A columns advance by 8, the B descriptor start
+// address by 32 B inside a 128-B swizzle atom and by one atom (ATOM_B bytes)
+// every 4 MMAs.
+template <int NK, int ATOM_B, int MODE>
 __device__ __forceinline__ void issue_stage(uint32_t d, uint32_t a, uint64_t b0, uint32_t idesc,
-                                            uint32_t acc0) {
+                                            uint32_t acc0, uint32_t sf) {
 #pragma unroll
     for (int kk = 0; kk < NK; ++kk)
-        mma_ts<I8>(d, a + 8u * kk, b0 + static_cast<uint64_t>(((kk >> 2) * ATOM_B + (kk & 3) * 32) >> 4),
-               idesc, kk == 0 ? acc0 : 1u);
+        mma_ts<MODE>(d, a + 8u * kk, b0 + static_cast<uint64_t>(((kk >> 2) * ATOM_B + (kk & 3) * 32) >> 4),
+                     idesc, kk == 0 ? acc0 : 1u, sf);
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
@@ -280,6 +328,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 8 fp32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 32 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
@@ -334,6 +394,14 @@ __device__ __forceinline__ void decode_word_u8(uint32_t w, uint32_t* v) {
     v[1] = mask_flip_or(w >> 2, 0x03030303u, 0x02020202u);
     v[2] = mask_flip_or(w >> 4, 0x03030303u, 0x02020202u);
     v[3] = mask_flip_or(w >> 6, 0x03030303u, 0x02020202u);
+}
+
+// fp4 mode: the 16 fields of a code word as two words of e2m1 nibbles f'/2
+// (f' = f xor 2 in the nibble's low two bits: 0, 0.5, 1, 1.5): the even
+// fields, then the odd ones (K order (0, 2, .., 14, 1, 3, .., 15)).
+__device__ __forceinline__ void decode_word_f4(uint32_t w, uint32_t* v) {
+    v[0] = mask_flip_or(w, 0x33333333u, 0x22222222u);
+    v[1] = mask_flip_or(w >> 2, 0x33333333u, 0x22222222u);
 }
 
 __device__ __forceinline__ void decode_word(uint32_t w, uint32_t* v) {
@@ -424,17 +492,25 @@ __device__ __forceinline__ int64_t cta_of_item(const GemmCommon& p, int64_t i) {
     return ((i + 1) * p.grid + p.items - 1) / p.items - 1;
 }
 
-template <int NT>
+// Shared memory and TMEM of one instance. bf16: 256 K per stage (four
+// 64-K activation atoms), A slots of 128 TMEM columns; integer mode: 512 K
+// per stage (four 128-K atoms), 128 columns; fp4: 512 K per stage (two
+// 256-K atoms), 64 columns, plus 32 columns of unit scale factors.
+template <int NT, int MODE>
 struct Layout {
-    static constexpr int kCodesSlots = NT == 16 ? 8 : NT == 32 ? 6 : 4;
-    static constexpr int kASlots = NT == 128 ? 2 : 3;           // A in TMEM, 128 columns each
-    static constexpr int kBSlots = NT <= 32 ? 6 : NT == 64 ? 4 : 2;
+    static constexpr bool F4 = MODE == kModeF4;
+    static constexpr int kCodesSlots = F4 ? (NT == 80 ? 6 : 4) : NT == 16 ? 8 : NT == 32 ? 6 : 4;
+    static constexpr int kASlots = F4 ? (NT == 80 ? 4 : 2) : NT == 128 ? 2 : 3;
+    static constexpr uint32_t kASlotCols = F4 ? 64 : 128;
+    static constexpr int kBSlots = F4 ? (NT == 80 ? 6 : 3) : NT <= 32 ? 6 : NT == 64 ? 4 : 2;
     static_assert(kBSlots <= 2 * kASlots, "the activation producer reads stage completions "
                                          "from the A ring; deeper B rings would alias phases");
-    static constexpr uint32_t kAccStride = NT == 128 ? 128 : 64;  // two accumulators
+    // two accumulators, 32-column aligned
+    static constexpr uint32_t kAccStride = F4 ? (NT + 31) / 32 * 32 : NT == 128 ? 128 : 64;
     static constexpr uint32_t kACol0 = 2 * kAccStride;
-    static constexpr int kAtomB = NT * 128;             // NT rows x 128 B (64 K)
-    static constexpr int kBSlot = 4 * kAtomB;           // 256 K
+    static constexpr uint32_t kSfCol = kACol0 + kASlotCols * kASlots;  // fp4 only
+    static constexpr int kAtomB = NT * 128;             // NT rows x 128 B
+    static constexpr int kBSlot = (F4 ? 2 : 4) * kAtomB;
     static constexpr int kCodesOff = 0;
     static constexpr int kBOff = kCodesSlots * kCodesSlotBytes;
     static constexpr int kBarOff = kBOff + kBSlots * kBSlot;
@@ -444,7 +520,7 @@ struct Layout {
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort, last, ok
     static constexpr int kSxOff = kMiscOff + 16;              // 128 floats
     static constexpr int kBytes = kSxOff + 128 * 4 + 1024;    // + alignment slack
-    static_assert(kACol0 + 128 * kASlots <= kTmemCols, "TMEM columns");
+    static_assert(kSfCol + (F4 ? 32 : 0) <= kTmemCols, "TMEM columns");
 };
 
 // Integer mode: the four digit-plane accumulators of one activation row,
@@ -457,6 +533,28 @@ __device__ __forceinline__ double planes_value(const float* v) {
     return static_cast<double>(t);
 }
 
+// fp4 mode: 2 sum_p 9^p acc_p for the MP activation rows of this thread's
+// TMEM lane (plane p of row j in column d + p MP + j). Each accumulator is a
+// multiple of 1/2 below 2^23 in magnitude (an exact fp32 value), so twice it
+// converts exactly, and the int64 sum (< 2^52) is exact.
+template <int MP>
+__device__ __forceinline__ void f4_plane_sums(uint32_t d, long long (&s2)[MP]) {
+#pragma unroll
+    for (int j = 0; j < MP; ++j) s2[j] = 0;
+    long long w = 1;
+#pragma unroll
+    for (int pl = 0; pl < kF4Planes; ++pl) {
+        float v[MP];
+        if constexpr (MP == 16)
+            tmem_ld16(d + 16u * pl, v);
+        else
+            tmem_ld8(d + 8u * pl, v);
+#pragma unroll
+        for (int j = 0; j < MP; ++j) s2[j] += w * static_cast<long long>(__float2int_rn(2.0f * v[j]));
+        w *= 9;
+    }
+}
+
 // 2^e as a double, for e in [-1022, 1023].
 __device__ __forceinline__ double exp2_int(int e) {
     return __longlong_as_double(static_cast<long long>(e + 1023) << 52);
@@ -467,15 +565,21 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
                        __fadd_rn(a.w, b.w));
 }
 
-// I8: the integer mode (kind::i8; A = offset-binary fields as u8, B = the
-// activations' signed base-256 digit planes, NT = 4 x activation rows),
-// 512 K per stage; otherwise bf16 (kind::f16), 256 K per stage.
-template <int NT, int MAXP, bool I8>
-__global__ void __launch_bounds__(kThreads, 1)
+// MODE kModeI8: the integer mode (kind::i8; A = offset-binary fields as u8,
+// B = the activations' signed base-256 digit planes, NT = 4 x activation
+// rows), 512 K per stage; kModeF4: the packed-fp4 mode (kind::mxf4; A =
+// f'/2 nibbles, B = ten base-9 digit planes of 8 or 16 rows each, NT = 80 or
+// 160), 512 K per stage; kModeBF16 (kind::f16), 256 K per stage.
+template <int NT, int MAXP, int MODE>
+__global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
     wq_gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
-    using L = Layout<NT>;
-    constexpr int SK = I8 ? 2 * kStageK : kStageK;  // K per stage
-    constexpr int KB = I8 ? 128 : 64;                // K per 128-B activation box
+    using L = Layout<NT, MODE>;
+    constexpr int kCodesWarp = Roles<MODE>::kCodesWarp, kXWarp = Roles<MODE>::kXWarp,
+                  kMmaWarp = Roles<MODE>::kMmaWarp;
+    constexpr bool I8 = MODE == kModeI8, F4 = MODE == kModeF4;
+    constexpr bool INT = MODE != kModeBF16;          // fixed-point activations, exact sums
+    constexpr int SK = INT ? 2 * kStageK : kStageK;  // K per stage
+    constexpr int KB = F4 ? 256 : I8 ? 128 : 64;     // K per 128-B activation box
     const GemmCommon& p = prm.c;
     constexpr int SC = L::kCodesSlots, SA = L::kASlots, SB = L::kBSlots;
     extern __shared__ uint8_t smem_raw[];
@@ -503,9 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < SB; ++s) mbar_init(b_xfull + 8u * s, 1);
         for (int s = 0; s < SA; ++s) {
-            // integer mode: the decoders alone (warp 0 also waits for the
-            // stage's activations); bf16: decoders and permuters
-            mbar_init(b_afull + 8u * s, I8 ? kDecWarps : kDecWarps + kPermWarps);
+            // integer and fp4 modes: the decoders alone (warp 0 also waits
+            // for the stage's activations); bf16: decoders and permuters
+            mbar_init(b_afull + 8u * s, INT ? kDecWarps : kDecWarps + kPermWarps);
             mbar_init(b_aempty + 8u * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -538,6 +642,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if constexpr (F4) {
+        // the unit scale factors every fp4 MMA reads
+        if (warp < 4) {
+            uint32_t one[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) one[j] = kScaleOne;
+            tmem_st32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kSfCol, one);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     const int64_t rs = range_start(p, blockIdx.x), re = range_start(p, blockIdx.x + 1);
 
     if (warp == kCodesWarp) {
@@ -550,13 +667,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int cur = 0;
             bool ok = true;
             while (ok && next_piece(prm, s, re, pc, cur)) {
+                const CUtensorMap* tc = &prm.prob[pc.pi].tc;
                 for (int64_t c = pc.c0; c < pc.c1; ++c) {
                     if (!mbar_wait(b_cempty + 8u * cr.idx, cr.phase ^ 1u, abort)) {
                         ok = false;
                         break;
                     }
                     mbar_expect_tx(b_cfull + 8u * cr.idx, kCodesTx);
-                    tma_load_2d(sbase + L::kCodesOff + cr.idx * kCodesSlotBytes, &prm.prob[pc.pi].tc,
+                    tma_load_2d(sbase + L::kCodesOff + cr.idx * kCodesSlotBytes, tc,
                                 b_cfull + 8u * cr.idx, static_cast<int32_t>(c * (kChunkK / 4)),
                                 static_cast<int32_t>(pc.b * kFeat));
                     cr.next();
@@ -577,8 +695,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int cur = 0;
             bool ok = true;
             while (ok && next_piece(prm, s, re, pc, cur)) {
+                const int64_t pk = prm.prob[pc.pi].k;  // once per piece
+                const CUtensorMap* tx = &prm.prob[pc.pi].tx;
                 for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
+                    const int ns = stages_of_chunk<SK>(pk, c);
                     for (int i = 0; i < ns; ++i, ++gs) {
                         if (gs >= static_cast<uint32_t>(SB)) {  // B slot free: stage gs - SB done
                             if (!mbar_wait(b_aempty + 8u * er.idx, er.phase, abort)) {
@@ -588,12 +708,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             er.next();
                         }
                         const int64_t k0 = c * kChunkK + i * SK;
-                        const int boxes = stage_k<SK>(prm.prob[pc.pi].k, k0) / KB;
+                        const int boxes = (stage_k<SK>(pk, k0) + KB - 1) / KB;
                         const uint32_t dst = sbase + L::kBOff + xr.idx * L::kBSlot;
                         mbar_expect_tx(b_xfull + 8u * xr.idx, static_cast<uint32_t>(boxes * NT * 128));
                         for (int bx = 0; bx < boxes; ++bx)
-                            tma_load_2d(dst + bx * L::kAtomB, &prm.prob[pc.pi].tx, b_xfull + 8u * xr.idx,
-                                        static_cast<int32_t>(k0 + KB * bx), 0);
+                            tma_load_2d(dst + bx * L::kAtomB, tx, b_xfull + 8u * xr.idx,
+                                        static_cast<int32_t>((k0 + KB * bx) / (F4 ? 2 : 1)), 0);
                         xr.next();
                     }
                 }
@@ -603,9 +723,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- MMA issuer
         // The issuing thread blocks on every tcgen05.mma, so its loop keeps
-        // bookkeeping to a few 32-bit operations between MMAs.
+        // bookkeeping to a few 32-bit operations between MMAs: a piece's
+        // stage counts come from one read of the matrix's k (the launch's
+        // parameters are too large for the constant cache, and the MMA asm's
+        // memory clobbers would otherwise reload it on every stage).
         if (lane == 0) {
-            constexpr uint32_t idesc = I8 ? idesc_i8(NT) : idesc_bf16(NT);
+            constexpr uint32_t idesc = F4 ? idesc_mxf4(NT) : I8 ? idesc_i8(NT) : idesc_bf16(NT);
+            const uint32_t sf = tmem + L::kSfCol;
             Ring<SA> ar;
             Ring<SB> br;
             Ring<2> accr;
@@ -618,30 +742,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + L::kAccStride * accr.idx;
                 uint32_t acc0 = 0;
-                for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                    const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
-                    const int tail_k = stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + (ns - 1) * SK);
-                    for (int i = 0; i < ns; ++i) {
-                        if (!mbar_wait(b_afull + 8u * ar.idx, ar.phase, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t a = tmem + L::kACol0 + 128u * ar.idx;
-                        const uint64_t b0 = sw128_desc(sbase + L::kBOff + br.idx * L::kBSlot);
-                        if (tail_k == SK || i != ns - 1)
-                            issue_stage<16, L::kAtomB, I8>(d, a, b0, idesc, acc0);
-                        else if (!I8 || tail_k == 256)
-                            issue_stage<8, L::kAtomB, I8>(d, a, b0, idesc, acc0);
-                        else if (tail_k == 128)
-                            issue_stage<4, L::kAtomB, I8>(d, a, b0, idesc, acc0);
-                        else
-                            issue_stage<12, L::kAtomB, I8>(d, a, b0, idesc, acc0);
-                        acc0 = 1;
-                        mma_commit(b_aempty + 8u * ar.idx);
-                        ar.next();
-                        br.next();
+                // the piece's K range [c0 * 512, min(c1 * 512, k)): whole
+                // stages, then at most one short one (k is a multiple of 128)
+                const int64_t pk = prm.prob[pc.pi].k;
+                const int64_t kspan = (pc.c1 * kChunkK < pk ? pc.c1 * kChunkK : pk) - pc.c0 * kChunkK;
+                const int nfull = static_cast<int>(kspan / SK);
+                const int tail_k = static_cast<int>(kspan % SK);
+                for (int i = 0; i <= nfull; ++i) {
+                    if (i == nfull && tail_k == 0) break;
+                    if (!mbar_wait(b_afull + 8u * ar.idx, ar.phase, abort)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    const uint32_t a = tmem + L::kACol0 + L::kASlotCols * ar.idx;
+                    const uint64_t b0 = sw128_desc(sbase + L::kBOff + br.idx * L::kBSlot);
+                    if (i < nfull)
+                        issue_stage<F4 ? 8 : 16, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                    else if constexpr (F4) {  // 64 K per MMA
+                        if (tail_k == 128)
+                            issue_stage<2, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                        else if (tail_k == 256)
+                            issue_stage<4, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                        else
+                            issue_stage<6, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                    } else if (!I8 || tail_k == 256)
+                        issue_stage<8, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                    else if (tail_k == 128)
+                        issue_stage<4, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                    else
+                        issue_stage<12, L::kAtomB, MODE>(d, a, b0, idesc, acc0, sf);
+                    acc0 = 1;
+                    mma_commit(b_aempty + 8u * ar.idx);
+                    ar.next();
+                    br.next();
                 }
                 if (!ok) break;
                 mma_commit(b_accfull + 8u * accr.idx);
@@ -664,22 +798,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         int cur = 0;
         bool ok = true;
         while (ok && next_piece(prm, s, re, pc, cur)) {
+            const int64_t pk = prm.prob[pc.pi].k;  // once per piece
             for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
                 if (!warp_wait(b_cfull + 8u * cr.idx, cr.phase, abort)) {
                     ok = false;
                     break;
                 }
                 const uint32_t crow = sbase + L::kCodesOff + cr.idx * kCodesSlotBytes + r * 128;
-                const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
+                const int ns = stages_of_chunk<SK>(pk, c);
                 for (int i = 0; i < ns; ++i) {
                     // this warp's half of the stage exists unless the stage is a short tail
-                    const bool mine = stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + i * SK) > SK / 2 * half;
+                    const bool mine = stage_k<SK>(pk, c * kChunkK + i * SK) > SK / 2 * half;
                     // bf16: 128 K of this row (32 code bytes) -> 64 TMEM columns;
-                    // integer mode: 256 K (64 code bytes) -> 64 TMEM columns
-                    const int ch = I8 ? 4 * half : 4 * i + 2 * half;
+                    // integer mode: 256 K (64 code bytes) -> 64 TMEM columns;
+                    // fp4: 256 K (64 code bytes) -> 32 TMEM columns
+                    const int ch = INT ? 4 * half : 4 * i + 2 * half;
                     uint32_t v[32], v2[32];
                     uint4 c2 = make_uint4(0, 0, 0, 0), c3 = c2;
-                    if (I8 && mine) {
+                    if (F4 && mine) {
+                        // the whole stage decoded before waiting for its slot
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 cw = lds128(crow + (((ch + q) ^ (r & 7)) << 4));
+                            decode_word_f4(cw.x, v + 8 * q);
+                            decode_word_f4(cw.y, v + 8 * q + 2);
+                            decode_word_f4(cw.z, v + 8 * q + 4);
+                            decode_word_f4(cw.w, v + 8 * q + 6);
+                        }
+                        if (r == kFeat) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = kOnesF4;
+                        }
+                    } else if (I8 && mine) {
                         // the first half decoded before the wait; the rest after the first store
                         const uint4 c0 = lds128(crow + ((ch ^ (r & 7)) << 4));
                         const uint4 c1 = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
@@ -697,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = 0x01010101u;
                         }
-                    } else if (!I8 && mine) {
+                    } else if (!INT && mine) {
                         // decode the whole stage before waiting for its slot
                         const uint4 c0 = lds128(crow + ((ch ^ (r & 7)) << 4));
                         const uint4 c1 = lds128(crow + (((ch + 1) ^ (r & 7)) << 4));
@@ -718,9 +868,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (mine) {
+                    if (mine && F4) {
                         tc_fence_after();
-                        const uint32_t col = tmem + lane_addr + L::kACol0 + 128u * ar.idx + 64u * half;
+                        tmem_st32(tmem + lane_addr + L::kACol0 + L::kASlotCols * ar.idx + 32u * half, v);
+                        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                        tc_fence_before();
+                    } else if (mine) {
+                        tc_fence_after();
+                        const uint32_t col = tmem + lane_addr + L::kACol0 + L::kASlotCols * ar.idx + 64u * half;
                         tmem_st32(col, v);
                         if (I8) {
                             decode_word_u8(c2.x, v2);
@@ -741,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                     }
                     __syncwarp();
-                    if constexpr (I8) {
+                    if constexpr (INT) {
                         // the planes arrive in MMA order: no permuter pass, so
                         // warp 0 holds the stage until its activations landed
                         if (warp == 0 && !warp_wait(b_xfull + 8u * xbr.idx, xbr.phase, abort)) {
@@ -758,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cr.next();
             }
         }
-    } else if (!I8 && warp >= kPermWarp0 && warp < kPermWarp0 + kPermWarps) {
+    } else if (!INT && warp >= kPermWarp0 && warp < kPermWarp0 + kPermWarps) {
         // ------------------- activation permuters: each group of 16 K -> (j, j + 8)
         // (bf16 mode only: the integer mode's digit planes arrive in MMA order)
         const int ptid = tid - kPermWarp0 * 32;
@@ -769,15 +924,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int cur = 0;
         bool ok = true;
         while (ok && next_piece(prm, s, re, pc, cur)) {
+            const int64_t pk = prm.prob[pc.pi].k;  // once per piece
             for (int64_t c = pc.c0; c < pc.c1 && ok; ++c) {
-                const int ns = stages_of_chunk<SK>(prm.prob[pc.pi].k, c);
+                const int ns = stages_of_chunk<SK>(pk, c);
                 for (int i = 0; i < ns; ++i) {
                     if (!warp_wait(b_xfull + 8u * br.idx, br.phase, abort)) {
                         ok = false;
                         break;
                     }
                     // the integer mode's digit planes arrive already in MMA order
-                    const int groups = I8 ? 0 : stage_k<SK>(prm.prob[pc.pi].k, c * kChunkK + i * SK) / 16;
+                    const int groups = INT ? 0 : stage_k<SK>(pk, c * kChunkK + i * SK) / 16;
                     const uint32_t bslot = sbase + L::kBOff + br.idx * L::kBSlot;
                     for (int it = ptid; it < NT * groups; it += kPermWarps * 32) {
                         const int bro = it % NT, g = it / NT;
@@ -823,11 +979,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!*epi_ok) break;
             tc_fence_after();
             const uint32_t d = tmem + lane_addr + L::kAccStride * ab;
+            constexpr int MP = NT / kF4Planes;  // fp4: activation rows per plane
             // pass 1: Sx (TMEM lane 127) to shared memory, read by the one
-            // warp whose lanes hold it
+            // warp whose lanes hold it (fp4: the ones row's A is 1.0, so its
+            // plane sums are sum v itself, half of 2 sum_p 9^p acc_p)
+            if constexpr (F4) {
+                if (e == kFeat / 32) {
+                    long long s2[MP];
+                    f4_plane_sums<MP>(d, s2);
+                    if (r == kFeat) {
+#pragma unroll
+                        for (int j = 0; j < MP; ++j)
+                            reinterpret_cast<double*>(sx)[j] = 0.5 * static_cast<double>(s2[j]);
+                    }
+                }
+            }
 #pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) {
-                if (e != kFeat / 32) break;
+                if (F4 || e != kFeat / 32) break;
                 float v[16];
                 __syncwarp();
                 tmem_ld16(d + c0, v);
@@ -852,8 +1021,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wslot = (pb.item0 + pc.b * pb.nchunks + pc.c0 == rs) ? 0 : 1;
             float* prow = full ? nullptr
                                : p.partial + ((static_cast<int64_t>(blockIdx.x) * 2 + wslot) * kFeat + r) * p.m4;
+            if constexpr (F4) {
+                // weight row r: sum_k v f' = 2 sum_p 9^p acc_p; x = v 2^(E - 29)
+                long long s2[MP];
+                __syncwarp();
+                f4_plane_sums<MP>(d, s2);
+                float o[MP];
+#pragma unroll
+                for (int j = 0; j < MP; ++j) {
+                    const double scale = j < p.m ? exp2_int(__ldg(pb.xexp + j) - 29) : 0.0;
+                    o[j] = static_cast<float>(
+                        (p.P4 * static_cast<double>(s2[j]) + p.PQ * reinterpret_cast<const double*>(sx)[j]) * scale);
+                }
+                if (valid_row) {
+                    if (full) {
+#pragma unroll
+                        for (int j = 0; j < MP; ++j)
+                            if (j < p.m)
+                                pb.y[j * pb.n + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * o[j]));
+                    } else {
+#pragma unroll
+                        for (int j4 = 0; j4 < MP; j4 += 4)
+                            if (j4 < p.m4)
+                                *reinterpret_cast<float4*>(prow + j4) =
+                                    make_float4(o[j4], o[j4 + 1], o[j4 + 2], o[j4 + 3]);
+                    }
+                }
+            }
 #pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) {
+                if (F4) break;
                 float v[16];
                 __syncwarp();
                 tmem_ld16(d + c0, v);
@@ -985,6 +1182,41 @@ __device__ __forceinline__ void digits16(const uint32_t (&hw)[8], int E, uint32_
             pw[pp][pos >> 2] |= static_cast<uint32_t>(dgt & 255) << (8 * (pos & 3));
         }
         pw[3][pos >> 2] |= static_cast<uint32_t>(v & 255) << (8 * (pos & 3));
+    }
+}
+
+// fp4 mode: sixteen consecutive activations as the ten balanced base-9
+// digit planes of the same fixed point v = rint(x * 2^(29-E)): v = sum_p
+// 9^p d_p, d_p in [-4, 4] (|v| < 2^30 < 9^10 / 2), each digit as an e2m1
+// nibble (0, 1, 2, 3, 4 = 0b0000, 0b0010, 0b0100, 0b0101, 0b0110; sign bit 3).
+// Plane p's first word holds the even elements (element 2i in nibble i),
+// its second word the odd ones: the decoded weights' K order.
+__device__ __forceinline__ void digits16_f4(const uint32_t (&hw)[8], int E, uint32_t (&w0)[kF4Planes],
+                                            uint32_t (&w1)[kF4Planes]) {
+    const double sc = exp2_int(29 - E);
+#pragma unroll
+    for (int pp = 0; pp < kF4Planes; ++pp) w0[pp] = w1[pp] = 0;
+#pragma unroll
+    for (int f = 0; f < 16; ++f) {
+        const uint32_t bits = (f & 1) ? (hw[f >> 1] & 0xFFFF0000u) : (hw[f >> 1] << 16);
+        int v = __double2int_rn(static_cast<double>(__uint_as_float(bits)) * sc);
+        const int sh = 4 * (f >> 1);
+#pragma unroll
+        for (int pp = 0; pp < kF4Planes; ++pp) {
+            int dgt = v;  // the last plane takes what is left (|v| <= 3 there)
+            if (pp + 1 < kF4Planes) {
+                const int t = v + 4;
+                const int q = (t >= 0 ? t : t - 8) / 9;  // floor(t / 9)
+                dgt = t - 9 * q - 4;
+                v = q;
+            }
+            const uint32_t mag = static_cast<uint32_t>(dgt < 0 ? -dgt : dgt);
+            const uint32_t nib = (mag <= 2 ? 2 * mag : mag + 2) | (dgt < 0 ? 8u : 0u);
+            if (f & 1)
+                w1[pp] |= nib << sh;
+            else
+                w0[pp] |= nib << sh;
+        }
     }
 }
 
@@ -1339,20 +1571,37 @@ constexpr int kMaxBatch = 64;  // matrices per launch (their descriptors travel 
 // inside every group of 16 transposed 4 x 4 like the decoded weights.
 // A row is split into `slices` CTAs; each finds the row's max|x| itself
 // (the row is small and in L2) and converts its share of 16-element groups.
+// fp4 mode: the same fixed point as ten base-9 digit planes of packed e2m1
+// nibbles, plane p of row j being row p * mp + j of a [10 mp][k / 2] byte
+// matrix (mp = 8 or 16 rows per plane; rows m..mp-1 are zero).
 struct XPlanes {
     const uint16_t* x[kMaxBatch];
     int8_t* planes[kMaxBatch];
     int* exps[kMaxBatch];
     int64_t k[kMaxBatch];
     int32_t m, slices;
+    int32_t mp;  // fp4 mode: rows per plane (the grid covers mp rows per matrix)
 };
 
+template <bool F4>
 __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XPlanes prm) {
     __shared__ uint32_t red[8];
     __shared__ int e_sh;
+    const int rows = F4 ? prm.mp : prm.m;
     const int row = blockIdx.x / prm.slices, slice = blockIdx.x % prm.slices;
-    const int xi = row / prm.m, j = row % prm.m;
+    const int xi = row / rows, j = row % rows;
     const int64_t k = prm.k[xi];
+    if (F4 && j >= prm.m) {  // padding rows of the planes: zero
+        const int64_t rb = k / 2;
+        const int64_t words = rb / 16;
+        const int64_t w1 = words * (slice + 1) / prm.slices;
+        for (int pp = 0; pp < kF4Planes; ++pp) {
+            uint4* dst = reinterpret_cast<uint4*>(prm.planes[xi] + (pp * prm.mp + j) * rb);
+            for (int64_t i = words * slice / prm.slices + threadIdx.x; i < w1; i += 256)
+                dst[i] = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
     const uint16_t* xr = prm.x[xi] + j * k;
     // max |x| of the row: the bf16 bits with the sign cleared order like the values
     uint32_t mb = 0;
@@ -1374,18 +1623,27 @@ __global__ void __launch_bounds__(256) xplanes_kernel(const __grid_constant__ XP
     }
     __syncthreads();
     const int E = e_sh;
-    int8_t* pl = prm.planes[xi] + 4 * j * k;
     const int64_t groups = k / 16;
     const int64_t g1 = groups * (slice + 1) / prm.slices;
     for (int64_t g = groups * slice / prm.slices + threadIdx.x; g < g1; g += 256) {
         const uint4 h0 = reinterpret_cast<const uint4*>(xr + 16 * g)[0];
         const uint4 h1 = reinterpret_cast<const uint4*>(xr + 16 * g)[1];
         const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        uint32_t pw[4][4];
-        digits16(hw, E, pw);
+        if constexpr (F4) {
+            uint32_t w0[kF4Planes], w1[kF4Planes];
+            digits16_f4(hw, E, w0, w1);
+            const int64_t rb = k / 2;
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp)
-            *reinterpret_cast<uint4*>(pl + pp * k + 16 * g) = make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
+            for (int pp = 0; pp < kF4Planes; ++pp)
+                *reinterpret_cast<uint2*>(prm.planes[xi] + (pp * prm.mp + j) * rb + 8 * g) = make_uint2(w0[pp], w1[pp]);
+        } else {
+            int8_t* pl = prm.planes[xi] + 4 * j * k;
+            uint32_t pw[4][4];
+            digits16(hw, E, pw);
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp)
+                *reinterpret_cast<uint4*>(pl + pp * k + 16 * g) = make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
+        }
     }
 }
 
@@ -1399,10 +1657,14 @@ struct Plan {
 // Work list of a launch: matrix i's items start at item0[i], its block
 // counters at block0[i].
 static Plan plan(int64_t m, const pq_gemm_problem_t* pr, int count, int64_t* item0,
-                 int64_t* block0, int64_t* nchunks, bool i8) {
+                 int64_t* block0, int64_t* nchunks, int mode) {
     Plan pl;
-    const int64_t rows = i8 ? 4 * m : m;  // B rows: activations, or their 4 digit planes
-    pl.nt = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
+    if (mode == kModeF4) {
+        pl.nt = m <= 8 ? 80 : 160;  // ten planes of 8 or 16 rows
+    } else {
+        const int64_t rows = mode == kModeI8 ? 4 * m : m;  // B rows: activations, or their 4 digit planes
+        pl.nt = rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
+    }
     int64_t items = 0, blocks = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t nb = (pr[i].n + kFeat - 1) / kFeat;
@@ -1457,15 +1719,30 @@ static bool coeffs_i8(int q, double& P4, double& PQ) {
     return true;
 }
 
-// The integer mode serves 2..16 activation rows (one row takes the CUDA-core
-// path when its x fits shared memory).
-static bool integer_mode(int64_t m) { return m <= 16; }
+// Up to 16 activation rows take the exact fixed-point arithmetic (one row
+// takes the CUDA-core path when its x fits shared memory): on packed fp4
+// MMAs while every k <= 2^20 (the fp32 accumulators then hold exact
+// integers), else on 8-bit MMAs (s32 accumulators); more rows take bf16.
+static int mode_of(int64_t m, const pq_gemm_problem_t* pr, int count) {
+    if (m > 16) return kModeBF16;
+    for (int i = 0; i < count; ++i)
+        if (pr[i].k > kF4MaxK) return kModeI8;
+    return kModeF4;
+}
 
 static int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
 
-// Workspace of one activation matrix in the integer mode: its digit planes
-// [4m][k] int8 and the exponents [m] int32.
-static int64_t xplanes_bytes(int64_t m, int64_t k) { return round256(4 * m * k) + round256(4 * m); }
+// fp4 mode: rows per digit plane.
+static int64_t f4_rows(int64_t m) { return m <= 8 ? 8 : 16; }
+
+// Digit planes of one activation matrix: [4m][k] int8 (integer mode) or
+// [10 mp][k/2] bytes (fp4 mode); the exponents [m] int32 follow them.
+static int64_t planes_bytes(int mode, int64_t m, int64_t k) {
+    return mode == kModeF4 ? round256(kF4Planes * f4_rows(m) * (k / 2)) : round256(4 * m * k);
+}
+static int64_t xplanes_bytes(int mode, int64_t m, int64_t k) {
+    return planes_bytes(mode, m, k) + round256(4 * m);
+}
 
 static int64_t partial_bytes(const Plan& pl, int64_t m) {
     const int64_t m4 = (m + 3) / 4 * 4;
@@ -1500,7 +1777,7 @@ static pq_status_t check_problem(int64_t m, const pq_gemm_problem_t& pr) {
 // Tensor maps of one matrix: codes [n rows][k/4 bytes] in boxes of 127 rows
 // x 128 B, activations [m rows][k] in boxes of nt rows x 64 K, both with the
 // 128B swizzle the MMA and the decoders read.
-static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt,
+static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt, int mode,
                         const pq_gemm_problem_t& pr, Problem& out, const int8_t* planes) {
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k / 4), static_cast<cuuint64_t>(pr.n)};
@@ -1512,9 +1789,13 @@ static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
-    if (planes) {  // integer mode: digit planes [4m rows][k] int8, boxes of nt rows x 128 K
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.k), static_cast<cuuint64_t>(4 * m)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.k)};
+    if (planes) {
+        // integer mode: digit planes [4m rows][k] int8, boxes of nt rows x 128 K;
+        // fp4: [10 mp rows][k/2] bytes, boxes of nt = 10 mp rows x 256 K
+        const int64_t row_bytes = mode == kModeF4 ? pr.k / 2 : pr.k;
+        const int64_t rows = mode == kModeF4 ? kF4Planes * f4_rows(m) : 4 * m;
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
         const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
         const cuuint32_t es[2] = {1, 1};
         return enc(&out.tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(planes), dims, strides,
@@ -1534,19 +1815,19 @@ static bool encode_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, int64_t m, int nt
     return true;
 }
 
-template <int NT, int MAXP, bool I8>
+template <int NT, int MAXP, int MODE>
 static cudaError_t launch(const GemmParams<MAXP>& prm, cudaStream_t s) {
-    using L = Layout<NT>;
+    using L = Layout<NT, MODE>;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         const cudaError_t e = cudaFuncSetAttribute(
-            wq_gemm_kernel<NT, MAXP, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+            wq_gemm_kernel<NT, MAXP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    wq_gemm_kernel<NT, MAXP, I8><<<prm.c.grid, kThreads, L::kBytes, s>>>(prm);
+    wq_gemm_kernel<NT, MAXP, MODE><<<prm.c.grid, Roles<MODE>::kThreads, L::kBytes, s>>>(prm);
     pqc::count_launch();
     return cudaGetLastError();
 }
@@ -1633,12 +1914,12 @@ static int64_t workspace_bytes(int q, int64_t m, const pq_gemm_problem_t* pr, in
             return -1;
     }
     if (vector_path(m, pr, count)) return 256;  // one task counter per matrix
-    const bool i8 = integer_mode(m);
+    const int mode = mode_of(m, pr, count);
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
-    const Plan pl = plan(m, pr, count, item0, block0, nchunks, i8);
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks, mode);
     int64_t b = pl.partials ? partial_bytes(pl, m) + round256(pl.blocks * 4) : 0;
-    if (i8)  // sized as if every matrix had its own activations
-        for (int i = 0; i < count; ++i) b += xplanes_bytes(m, pr[i].k);
+    if (mode != kModeBF16)  // sized as if every matrix had its own activations
+        for (int i = 0; i < count; ++i) b += xplanes_bytes(mode, m, pr[i].k);
     return b;
 }
 
@@ -1653,12 +1934,13 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         if (st != PQ_OK) return st;
     }
     if (vector_path(m, pr, count)) return run_vector<1>(q, pr, 1, workspace, ws_bytes, s);
-    const bool i8 = integer_mode(m);
+    const int mode = mode_of(m, pr, count);
+    const bool i8 = mode != kModeBF16;  // fixed-point activations (integer or fp4 MMAs)
     if (i8 && !coeffs_i8(q, P.c.P4, P.c.PQ)) return PQ_ERR_UNSUPPORTED;
     int64_t item0[kMaxBatch], block0[kMaxBatch], nchunks[kMaxBatch];
-    const Plan pl = plan(m, pr, count, item0, block0, nchunks, i8);
+    const Plan pl = plan(m, pr, count, item0, block0, nchunks, mode);
     const int64_t base = pl.partials ? partial_bytes(pl, m) + round256(pl.blocks * 4) : 0;
-    // integer mode: one digit-plane set per distinct activation matrix
+    // fixed point: one digit-plane set per distinct activation matrix
     int slot[kMaxBatch];
     int64_t planes_off[kMaxBatch];  // workspace offsets of each set's planes
     int nslots = 0;
@@ -1666,6 +1948,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
     int64_t need = base;
     if (i8) {
         X.m = static_cast<int32_t>(m);
+        X.mp = static_cast<int32_t>(f4_rows(m));
         for (int i = 0; i < count; ++i) {
             int t = 0;
             while (t < nslots && !(X.x[t] == pr[i].x_bf16 && X.k[t] == pr[i].k)) ++t;
@@ -1673,7 +1956,7 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
                 X.x[t] = pr[i].x_bf16;
                 X.k[t] = pr[i].k;
                 planes_off[t] = need;  // exponents follow the planes
-                need += xplanes_bytes(m, pr[i].k);
+                need += xplanes_bytes(mode, m, pr[i].k);
                 ++nslots;
             }
             slot[i] = t;
@@ -1692,14 +1975,14 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         for (int t = 0; t < nslots; ++t) {
             X.planes[t] = static_cast<int8_t*>(workspace) + planes_off[t];
             X.exps[t] = reinterpret_cast<int*>(static_cast<char*>(workspace) + planes_off[t] +
-                                               round256(4 * m * X.k[t]));
+                                               planes_bytes(mode, m, X.k[t]));
         }
     }
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return PQ_ERR_CUDA;
     for (int i = 0; i < count; ++i) {
         Problem& d = P.prob[i];
-        if (!encode_maps(enc, m, pl.nt, pr[i], d, i8 ? X.planes[slot[i]] : nullptr)) return PQ_ERR_CUDA;
+        if (!encode_maps(enc, m, pl.nt, mode, pr[i], d, i8 ? X.planes[slot[i]] : nullptr)) return PQ_ERR_CUDA;
         d.xexp = i8 ? X.exps[slot[i]] : nullptr;
         d.alpha = pr[i].alpha;
         d.y = pr[i].y_bf16;
@@ -1716,23 +1999,29 @@ static pq_status_t run(int q, int64_t m, const pq_gemm_problem_t* pr, int count,
         // at most one CTA per SM over all rows, each converting >= 64 groups
         int64_t maxk = 0;
         for (int t = 0; t < nslots; ++t) maxk = X.k[t] > maxk ? X.k[t] : maxk;
-        const int64_t rows = nslots * m;
+        const int64_t rows = nslots * (mode == kModeF4 ? X.mp : m);
         int64_t sl = sm_count() / rows;
         const int64_t cap = maxk / (16 * 64);
         sl = sl < cap ? sl : cap;
         X.slices = static_cast<int32_t>(sl < 1 ? 1 : sl);
-        xplanes_kernel<<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X); pqc::count_launch();
+        if (mode == kModeF4)
+            xplanes_kernel<true><<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X);
+        else
+            xplanes_kernel<false><<<static_cast<int>(rows * X.slices), 256, 0, s>>>(X);
+        pqc::count_launch();
         if (cudaGetLastError() != cudaSuccess) return PQ_ERR_CUDA;
     }
     cudaError_t e;
-    switch (pl.nt + (i8 ? 1 : 0)) {
-        case 17: e = launch<16, MAXP, true>(P, s); break;
-        case 33: e = launch<32, MAXP, true>(P, s); break;
-        case 65: e = launch<64, MAXP, true>(P, s); break;
-        case 16: e = launch<16, MAXP, false>(P, s); break;
-        case 32: e = launch<32, MAXP, false>(P, s); break;
-        case 64: e = launch<64, MAXP, false>(P, s); break;
-        default: e = launch<128, MAXP, false>(P, s); break;
+    switch (pl.nt * 4 + mode) {
+        case 80 * 4 + kModeF4: e = launch<80, MAXP, kModeF4>(P, s); break;
+        case 160 * 4 + kModeF4: e = launch<160, MAXP, kModeF4>(P, s); break;
+        case 16 * 4 + kModeI8: e = launch<16, MAXP, kModeI8>(P, s); break;
+        case 32 * 4 + kModeI8: e = launch<32, MAXP, kModeI8>(P, s); break;
+        case 64 * 4 + kModeI8: e = launch<64, MAXP, kModeI8>(P, s); break;
+        case 16 * 4 + kModeBF16: e = launch<16, MAXP, kModeBF16>(P, s); break;
+        case 32 * 4 + kModeBF16: e = launch<32, MAXP, kModeBF16>(P, s); break;
+        case 64 * 4 + kModeBF16: e = launch<64, MAXP, kModeBF16>(P, s); break;
+        default: e = launch<128, MAXP, kModeBF16>(P, s); break;
     }
     return e == cudaSuccess ? PQ_OK : PQ_ERR_CUDA;
 }

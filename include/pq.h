@@ -338,11 +338,15 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  * f' = c + 2; the factor (1/4, 1/3, 1/3, 1, 1) times alpha scales the sums,
  * which are rounded once to bf16. Two modes:
  *   m <= 16 (integer mode; m = 1 only for the grouped call): each activation
- *     row is scaled by a power of two to 30-bit fixed point, rounded to the
+ *     row is scaled by a power of two to 30-bit fixed point and rounded to the
  *     nearest integer (exact for every value within 2^22 of the row's largest
- *     magnitude; otherwise off by at most 2^-30 of it) and split into four
- *     signed base-256 digits; the tensor cores (kind::i8) form the exact
- *     integer sums of digits times fields, combined in fp64.
+ *     magnitude; otherwise off by at most 2^-30 of it); the tensor cores form
+ *     the exact integer sums of those integers times the fields, combined in
+ *     fp64. While every k <= 2^20 the integers go in as ten planes of
+ *     balanced base-9 digits on block-scaled fp4 MMAs (kind::mxf4, unit
+ *     scales; the weights as f'/2, every product and partial sum an exact
+ *     fp32 value); beyond, as four signed base-256 digit planes on 8-bit MMAs
+ *     (kind::i8, s32 sums). Both give the same bits.
  *   m > 16 (bf16 mode): weights decoded to bf16 1 + f'/4 (exact), products
  *     accumulated in fp32 by the tensor cores (kind::f16).
  * A lone matrix with m = 1 runs on the CUDA cores: below 2^27 weights with
@@ -362,7 +366,8 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  *            pq_wq_gemm_workspace_bytes(q, m, n, k) bytes, 256-byte
  *            aligned (may be NULL when that is 0). Split-K partial sums and
  *            counters, and in the integer mode the activations' digit planes
- *            (4 m k bytes) and exponents, live there; calls that share a
+ *            (fp4: 10 mp k / 2 bytes, mp = 8 for m <= 8 else 16; 8-bit:
+ *            4 m k bytes) and exponents, live there; calls that share a
  *            workspace must not overlap on the GPU. Results are deterministic.
  * Waits inside the kernel are bounded; pq_device_status() reports one that
  * gave up. Traffic: k/4 B of codes per output feature (+ x, y). */
