@@ -126,6 +126,26 @@ def test_wq_gemm_batch_matches_oracle():
         _check(q, x, packed, a, y, grouped=True)
 
 
+@pytest.mark.parametrize("q", [pq.PQ_SEQ2, pq.PQ_TERNARY])
+def test_rows_longer_than_fp4_exact_range(q):
+    """Rows longer than 2^20 take the 8-bit MMA form of the integer mode
+    (the fp4 form's fp32 sums stay exact only up to that length): a lone
+    matrix with a short K tail and two row blocks (the last ragged), and a
+    group in which one long matrix sends every matrix of the launch there."""
+    m, n, k = 5, 130, (1 << 20) + 128
+    x, packed, a = _case(q, m, n, k, seed=77)
+    y = pq.wq_gemm(q, x, packed, a)
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    _check(q, x, packed, a, y)
+    x2, packed2, a2 = _case(q, m, 300, 1024, seed=78)
+    ys = pq.wq_gemm_batch(q, [x, x2], [packed, packed2], [a, a2])
+    torch.cuda.synchronize()
+    assert pq.pq_device_status() == 0
+    _check(q, x, packed, a, ys[0], grouped=True)
+    _check(q, x2, packed2, a2, ys[1], grouped=True)
+
+
 def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(bits.astype(np.uint16).view(np.int16)).to(DEV).view(torch.bfloat16)
 
