@@ -1100,6 +1100,11 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
                 long long s2[MP];
                 __syncwarp();
                 f4_plane_sums<MP>(d, s2);
+                // the accumulator is read: hand it back before the arithmetic
+                // and the stores
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_accempty + 8u * ab);
                 float o[MP];
 #pragma unroll
                 for (int j = 0; j < MP; ++j) {
@@ -1168,9 +1173,11 @@ __global__ void __launch_bounds__(Roles<MODE>::kThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_accempty + 8u * ab);
+            if (!F4) {  // (fp4: handed back right after its TMEM reads)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_accempty + 8u * ab);
+            }
             if (!full) {
                 // the last of the block's pieces to finish adds them in K order
                 __threadfence();
