@@ -178,18 +178,33 @@ def test_adamw_argument_errors(L):
     assert f(pq.PQ_SEQ2, 1, arr, ctypes.byref(h), ctypes.byref(h), None) == pq.PQ_OK
 
 
+def _planes_bytes(m, k):
+    """The integer mode's digit planes of one activation matrix plus its
+    exponents: ten base-9 planes of packed e2m1 nibbles, mp = 8 or 16 rows
+    each (k <= 2^20, fp4 MMAs), or four int8 planes of m rows (8-bit MMAs)."""
+    r256 = lambda b: (b + 255) // 256 * 256
+    if k <= 1 << 20:
+        return r256(10 * (8 if m <= 8 else 16) * k // 2) + r256(4 * m)
+    return r256(4 * m * k) + r256(4 * m)
+
+
 def test_matmul_workspace_sizes(L):
     """Workspace sizing of the weight-only matmul (host arithmetic only): the
-    one-row path needs one counter block, the integer mode (m <= 16) at least
-    the activations' digit planes (4 m k bytes), a group one set per matrix;
-    sizes are multiples of 256; bad shapes give -1; the no-alloc scratch
-    holds every decode-sized problem of the Llama-3-8B shapes."""
+    one-row path needs one counter block, the integer mode (m <= 16) its
+    activations' digit planes and exponents (plus split-K partial sums), a
+    group one set per matrix; sizes are multiples of 256; bad shapes give
+    -1; the no-alloc scratch holds every decode-sized problem of the
+    Llama-3-8B shapes."""
     from bit_quantization_aware_b200 import pq
     q = pq.PQ_SEQ2
     assert L.pq_wq_gemm_workspace_bytes(q, 1, 16384, 16384) == 256
-    for m in (2, 9, 16):
-        b = L.pq_wq_gemm_workspace_bytes(q, m, 16384, 16384)
-        assert b >= 4 * m * 16384 and b % 256 == 0
+    for m in (2, 8, 9, 16):
+        for n, k in ((16384, 16384), (127, 128), (130, (1 << 20) + 128)):
+            b = L.pq_wq_gemm_workspace_bytes(q, m, n, k)
+            assert b >= _planes_bytes(m, k) and b % 256 == 0, (m, n, k, b)
+    # one row block, one chunk: no split-K scratch, the planes alone
+    for m in (2, 8, 9, 16):
+        assert L.pq_wq_gemm_workspace_bytes(q, m, 127, 512) == _planes_bytes(m, 512)
     assert L.pq_wq_gemm_workspace_bytes(q, 0, 128, 128) == -1
     assert L.pq_wq_gemm_workspace_bytes(q, 4, 128, 100) == -1
     assert L.pq_wq_gemm_workspace_bytes(pq.PQ_LSQ4, 4, 128, 128) == -1
@@ -200,7 +215,7 @@ def test_matmul_workspace_sizes(L):
         arr[i].n, arr[i].k, arr[i].x_bf16 = n, k, xs[i].value
     for m in (1, 8, 16):
         b = L.pq_wq_gemm_batch_workspace_bytes(q, m, len(shapes), arr)
-        assert b >= sum(4 * m * k for _, k in shapes) and b % 256 == 0
+        assert b >= sum(_planes_bytes(m, k) for _, k in shapes) and b % 256 == 0
     cap = pq.WQ_GEMM_NOALLOC_SCRATCH_BYTES
     for m in range(1, 17):
         for n, k in shapes:
