@@ -19,11 +19,13 @@
 // (16 bits apart), so the K order inside every group of 16 is interleaved
 // (j, j + 8); the activation tile is permuted the same way in shared memory.
 //
-// Integer mode (m <= 16). The 8-bit MMA kinds take K = 32 per instruction at
-// the cost of a K = 16 bf16 one, so the weights are decoded instead to their
-// offset-binary fields f' as unsigned bytes (one shift and one three-input
-// logic op per four weights) and multiplied (kind::i8, s32 accumulators) by
-// the activations in fixed point: a pre-pass scales each activation row by
+// Integer mode (m <= 16; this 8-bit form serves rows longer than 2^20, the
+// packed-fp4 form below all others). The 8-bit MMA kinds take K = 32 per
+// instruction at the cost of a K = 16 bf16 one, so the weights are decoded
+// instead to their offset-binary fields f' as unsigned bytes (one shift and
+// one three-input logic op per four weights) and multiplied (kind::i8, s32
+// accumulators) by the activations in fixed point: a pre-pass scales each
+// activation row by
 // 2^(29 - E), E = floor(log2 max|x|), rounds to integers and writes their four
 // signed base-256 digits as four planes, so the tensor cores form the exact
 // integer sums of digits times fields, combined in fp64 in the epilogue:
