@@ -44,10 +44,11 @@
 // |v| < 2^30 < 9^10 / 2). Every product is a multiple of 1/2 and every
 // partial sum stays below 2^23 in magnitude for k <= 2^20, so the fp32
 // accumulators hold exact integers, and the epilogue forms
-// sum_k v f' = sum_p 9^p (2 acc_p) exactly in int64: the result is the
-// integer mode's, bit for bit. The decoded nibbles of a code word are its
-// even fields, then its odd fields, so the K order inside every group of 16
-// is (0, 2, .., 14, 1, 3, .., 15), which the pre-pass applies to the planes.
+// sum_k v f' = sum_p 9^p (2 acc_p) exactly in int64: the same integers as
+// the 8-bit form's, through the same formula. The decoded nibbles of a code
+// word are its even fields, then its odd fields, so the K order inside every
+// group of 16 is (0, 2, .., 14, 1, 3, .., 15), which the pre-pass applies to
+// the planes.
 //
 // Operands. A (decoded weights) lives in TMEM (tcgen05.st from the decode
 // warps; tcgen05.mma reads it there, with no shared-memory round trip);

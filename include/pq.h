@@ -346,7 +346,8 @@ PQ_API pq_status_t pq_scaled_weights(int64_t rows, int64_t cols, const float* w,
  *     balanced base-9 digits on block-scaled fp4 MMAs (kind::mxf4, unit
  *     scales; the weights as f'/2, every product and partial sum an exact
  *     fp32 value); beyond, as four signed base-256 digit planes on 8-bit MMAs
- *     (kind::i8, s32 sums). Both give the same bits.
+ *     (kind::i8, s32 sums). Both form the same exact integers and put them
+ *     through the same formula.
  *   m > 16 (bf16 mode): weights decoded to bf16 1 + f'/4 (exact), products
  *     accumulated in fp32 by the tensor cores (kind::f16).
  * A lone matrix with m = 1 runs on the CUDA cores: below 2^27 weights with
